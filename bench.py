@@ -1,0 +1,394 @@
+"""Benchmark of the GDR-2 chunkwise forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one gdr2_forward call over the 1.3B-layer workload (B=4, H=16,
+T=4096, d_k=d_v=128, chunk 64, bf16 q/k/v/b/w, fp32 log-decay and state),
+with every input resident in HBM. The step's inputs (541 MB read + written)
+are larger than L2 (126 MB), so successive steps cannot reuse cached data.
+
+N > 1 runs one process per GPU (torchrun); every rank processes its own batch
+of independent (batch, head) recurrences (weak scaling, no collective on the
+data path) and the step time is the maximum over ranks.
+
+The JSON line carries:
+  value / ms_per_step  device time of K timed steps (CUDA events on the launch stream)
+  e2e                  same metric through the C ABI with pinned HOST buffers:
+                       host->device copy of the inputs, the forward, device->host
+                       copy of o and S_T, all inside the timed region
+  roofline             HBM roofline of the forward kernel (algorithmic bytes / time)
+  tensor               algorithmic FLOP/s against the dense bf16 peak
+  components           decode step (256 seq x 16 heads, fp32 state) and backward
+                       (B=2, T=4096) timings with their own rooflines
+  cpu_baseline         the fp64 oracle on the host cores (rank 0, N = 1)
+  clocks               SM clocks and throttle reasons sampled during the timed region
+`--impl reference` times the oracle itself on the same workload (sampled heads).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_wy_b200 import inputs as I  # noqa: E402
+
+METRIC = "GDR-2 chunk fwd tokens/s at H=16,d=128 (1×B200) and % tensor-core peak"
+WORKLOAD = "gdr2_forward B=4 H=16 T=4096 dk=dv=128 C=64 bf16 (1.3B-model layer)"
+BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 2 * 256 + 256  # q,k,v bf16 + log_alpha fp32 + b,w bf16 + o bf16
+FLOP_PER_TOKEN_HEAD = 139_264  # chunk products at C=64, d=128, triangular parts counted once
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not dist.is_initialized():
+        import datetime
+
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int):
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch of independent recurrences."""
+    return base + 7 * rank
+
+
+# ----------------------------------------------------------------------------- measurement helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_wy_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("fwd_") or f.endswith(".cuh"):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu capture, if it is of this source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_sha") != kernel_source_sha():
+        return None
+    return float(d["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while active."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_steps(fn, steps: int, stream) -> list:
+    """Per-step device times (ms), CUDA events recorded on the launching stream."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s, e in evs:
+        s.record(stream)
+        fn()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+# ----------------------------------------------------------------------------- the oracle (CPU baseline)
+def oracle_tokens_per_s(x: I.FwdInputs, heads, nthreads):
+    """Time the fp64 oracle on the listed (batch, head) recurrences over the full T."""
+    import numpy as np
+
+    import oracle
+
+    B, T, H, dk = x.q.shape
+    n = x.as_numpy64()
+    sel = {f: np.ascontiguousarray(np.stack([n[f][b, :, h] for b, h in heads], axis=1)[None])
+           for f in ("q", "k", "v", "log_alpha", "b", "w")}
+    t0 = time.perf_counter()
+    oracle.forward(sel["q"], sel["k"], sel["v"], sel["log_alpha"], sel["b"], sel["w"], nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return len(heads) * T / H / dt, dt
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, world, rank):
+    """The oracle as it stands, on the host cores, with this bench's metric and workload."""
+    if rank != 0:
+        return
+    cfg = I.FWD_1P3B_BF16
+    x = I.make_forward_inputs(**cfg)
+    B, T, H = cfg["B"], cfg["T"], cfg["H"]
+    heads = [(b, h) for b in range(B) for h in range(H)][:16]  # a quarter of the workload per step
+    nthr = cores()
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(x, heads[:2], nthr)
+    times = []
+    for _ in range(args.steps):
+        _, dt = oracle_tokens_per_s(x, heads, nthr)
+        times.append(dt)
+    tok = len(heads) * T / H
+    value = tok * len(times) / sum(times)
+    sample = f"{len(heads)} of {B * H} (batch, head) recurrences over the full T={T} per step (fp64, OpenMP)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthr, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def bench_components(dev, stream, peaks):
+    """Decode step and backward timings (each with its own roofline); not part of the step."""
+    from gated_delta_rule_wy_b200 import gdr2_backward, gdr2_decode_step, gdr2_forward
+
+    out = {}
+    cfg = I.DECODE_1P3B
+    N, H, dk, dv = cfg["N"], cfg["H"], cfg["dk"], cfg["dv"]
+    gen = torch.Generator(device=dev).manual_seed(cfg["seed"])
+    S = torch.randn((N, H, dk, dv), device=dev, generator=gen) * cfg["state_std"]
+    pool = [I.make_token_inputs((N, H, dk), (N, H, dv), cfg["dtype"], cfg["decay_shift"], gen) for _ in range(8)]
+    o = torch.empty((N, H, dv), dtype=cfg["dtype"], device=dev)
+    it = [0]
+
+    def dec():
+        gdr2_decode_step(*pool[it[0] % 8], S, out=o)
+        it[0] += 1
+
+    for _ in range(5):
+        dec()
+    ms = time_steps(dec, 200, stream)
+    us = 1e3 * statistics.median(ms)
+    state_bytes = 2 * N * H * dk * dv * 4
+    tok_bytes = N * H * (3 * dk * 2 + dk * 4 + 2 * dv * 2 + dv * 2)  # q,k,b bf16 + log_alpha + v,w + o
+    gbs = (state_bytes + tok_bytes) / (us * 1e-6) / 1e9
+    out["decode"] = {"workload": "256 seq x 16 heads, d=128, fp32 state 256 MiB, one token per call",
+                     "us_per_step": us, "tokens_per_s": N / (us * 1e-6), "gbs": gbs,
+                     "hbm_frac": gbs / peaks["hbm_gbs"]}
+    del S, pool
+    cfg = I.BWD_1P3B_BF16
+    x = I.make_forward_inputs(**cfg).to(dev)
+    dO = I.make_upstream_grad(cfg["B"], cfg["T"], cfg["H"], cfg["dv"], cfg["seed"], dtype=cfg["dtype"]).to(dev)
+    _, _, saved = gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, save_states=True)
+
+    def bwd():
+        gdr2_backward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, dO, None, None, saved)
+
+    bwd()
+    ms = time_steps(bwd, 3, stream)
+    t = statistics.median(ms)
+    out["backward"] = {"workload": "B=2 H=16 T=4096 d=128 bf16, saved chunk states",
+                       "ms_per_call": t, "tokens_per_s": cfg["B"] * cfg["T"] / (t * 1e-3)}
+    return out
+
+
+def run_ours(args, world, rank, local):
+    from gated_delta_rule_wy_b200 import build, gdr2_forward, gdr2_sync_status
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    peaks, peak_src = load_peaks()
+    cfg = dict(I.FWD_1P3B_BF16)
+    cfg["seed"] = shard_seed(cfg["seed"], rank)
+    x_cpu = I.make_forward_inputs(**cfg)
+    x = x_cpu.to(dev)
+    B, T, H, dk, dv = cfg["B"], cfg["T"], cfg["H"], cfg["dk"], cfg["dv"]
+    o = torch.empty((B, T, H, dv), dtype=cfg["dtype"], device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o)
+
+    for _ in range(args.warmup):
+        step()
+    gdr2_sync_status()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = time_steps(step, args.steps, stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    gdr2_sync_status()
+    total_ms = max_over_ranks(sum(ms), world, dev)
+    ms_per_step = total_ms / args.steps
+    tokens = B * T * world
+    value = tokens / (ms_per_step * 1e-3)
+
+    # ---- end to end through the C ABI with host buffers ----
+    pinned = [t.pin_memory() for t in (x_cpu.q, x_cpu.k, x_cpu.v, x_cpu.log_alpha, x_cpu.b, x_cpu.w)]
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    sT_host = torch.empty((B, H, dk, dv), dtype=torch.float32).pin_memory()
+    dbufs = [torch.empty_like(t, device=dev) for t in pinned]
+    h2d = sum(t.numel() * t.element_size() for t in pinned)
+    d2h = o_host.numel() * o_host.element_size() + sT_host.numel() * 4
+
+    def e2e_step():
+        for d, hsrc in zip(dbufs, pinned):
+            d.copy_(hsrc, non_blocking=True)
+        oo, sT, _ = gdr2_forward(*dbufs, None, out=o)
+        o_host.copy_(oo, non_blocking=True)
+        sT_host.copy_(sT, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(time_steps(e2e_step, e2e_steps, stream)), world, dev) / e2e_steps
+    e2e_value = tokens / (e2e_ms * 1e-3)
+
+    # ---- roofline of the forward kernel (one launch per step) ----
+    alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD + B * H * dk * dv * 4
+    alg_flop = B * T * H * FLOP_PER_TOKEN_HEAD
+    t_launch = statistics.mean(ms) * 1e-3
+    achieved = alg_bytes / t_launch / 1e9
+    traffic = committed_traffic("fwd")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": alg_bytes}
+    tflops = alg_flop / t_launch / 1e12
+    tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+              "frac": tflops / peaks["bf16_tflops"], "algorithmic_flop_per_launch": alg_flop,
+              "attainable_frac": max(alg_bytes / (peaks["hbm_gbs"] * 1e9), alg_flop / (peaks["bf16_tflops"] * 1e12))
+              / t_launch}
+
+    comps = None
+    cpu = None
+    if world == 1:
+        comps = bench_components(dev, stream, peaks)
+        heads = [(b, h) for b in range(B) for h in range(H)]
+        val, dt = oracle_tokens_per_s(x_cpu, heads, cores())
+        cpu = {"value": val, "unit": "tokens/s", "cores": cores(), "kind": "oracle",
+               "sample": f"the whole workload ({B * H} recurrences of T={T}) once, fp64, {dt:.1f} s"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+                "config": {"workload": WORKLOAD, "B": B, "H": H, "T": T, "dk": dk, "dv": dv, "chunk": 64,
+                           "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
+                           "l2": "inputs larger than L2 (541 MB per step vs 126 MB)"},
+                "clocks": clk.summary(),
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": args.steps, "roofline": roofline, "tensor": tensor, "components": comps,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

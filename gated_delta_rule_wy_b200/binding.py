@@ -1,0 +1,198 @@
+"""ctypes binding of libgdr2.so: the C ABI in ``include/gdr2.h`` with torch tensors.
+
+Argument marshalling only. Every function here checks shapes, dtypes and
+devices, allocates output tensors with PyTorch (device memory is the one
+thing torch provides), passes raw device pointers and the current CUDA stream
+to the library, and turns a non-OK status into ``GDR2Error``. There is no
+fallback: if ``libgdr2.so`` is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdr2.so")
+
+GDR2_OK, GDR2_ERR_INVALID_ARG, GDR2_ERR_UNSUPPORTED, GDR2_ERR_CUDA, GDR2_ERR_TIMEOUT = range(5)
+GDR2_F32, GDR2_BF16 = 0, 1
+CHUNK = 64
+_STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
+
+# Every symbol include/gdr2.h declares (the ABI tests check the exports).
+EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward", "gdr2_decode_step",
+                    "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_sync_status")
+
+
+class GDR2Error(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"GDR2 {_STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libgdr2.so once and declare the signatures of include/gdr2.h."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with `python -m gated_delta_rule_wy_b200.build` "
+                               "(there is no CPU fallback)")
+        lib = ctypes.CDLL(p)
+        I, P, Z = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+        lib.gdr2_abi_version.restype = I
+        lib.gdr2_abi_version.argtypes = []
+        lib.gdr2_last_error.restype = ctypes.c_char_p
+        lib.gdr2_last_error.argtypes = []
+        lib.gdr2_forward.restype = I
+        lib.gdr2_forward.argtypes = [I, I, I, I, I, I] + [P] * 11
+        lib.gdr2_decode_step.restype = I
+        lib.gdr2_decode_step.argtypes = [I, I, I, I, I] + [P] * 9
+        lib.gdr2_backward_workspace_bytes.restype = Z
+        lib.gdr2_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        lib.gdr2_backward.restype = I
+        lib.gdr2_backward.argtypes = [I, I, I, I, I, I] + [P] * 17 + [Z, P]
+        lib.gdr2_sync_status.restype = I
+        lib.gdr2_sync_status.argtypes = [P]
+        _lib = lib
+        return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDR2_F32
+    if t.dtype == torch.bfloat16:
+        return GDR2_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _check(t, name, shape, dtype):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _raise(lib, st):
+    if st != GDR2_OK:
+        raise GDR2Error(st, lib.gdr2_last_error().decode(errors="replace"))
+
+
+def gdr2_abi_version() -> int:
+    return load_library().gdr2_abi_version()
+
+
+def gdr2_last_error() -> str:
+    return load_library().gdr2_last_error().decode(errors="replace")
+
+
+def gdr2_sync_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel gave up a bounded wait."""
+    lib = load_library()
+    _raise(lib, lib.gdr2_sync_status(_stream(stream)))
+
+
+def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_states=False,
+                 out=None, stream=None):
+    """Chunkwise forward. Returns (o, S_T, saved_states); S_T / saved_states may be None.
+
+    q, k, b: [B, T, H, dk]; v, w: [B, T, H, dv] (fp32 or bf16, one dtype);
+    log_alpha: [B, T, H, dk] fp32; S0: [B, H, dk, dv] fp32 or None.
+    """
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("b", b, (B, T, H, dk)),
+                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H, dv))):
+        _check(t, name, shp, dt)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32)
+    _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    dev = q.device
+    o = out if out is not None else torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(o, "o", (B, T, H, dv), dt)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if final_state else None
+    nc = (T + CHUNK - 1) // CHUNK
+    saved = torch.empty((B, H, nc, dk, dv), dtype=torch.float32, device=dev) if save_states else None
+    st = lib.gdr2_forward(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                          _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _stream(stream))
+    _raise(lib, st)
+    return o, S_T, saved
+
+
+def gdr2_decode_step(q, k, v, log_alpha, b, w, S, *, out=None, stream=None):
+    """One decode token; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv]."""
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    for name, t, shp in (("q", q, (N, H, dk)), ("k", k, (N, H, dk)), ("b", b, (N, H, dk)),
+                         ("v", v, (N, H, dv)), ("w", w, (N, H, dv))):
+        _check(t, name, shp, dt)
+    _check(log_alpha, "log_alpha", (N, H, dk), torch.float32)
+    _check(S, "S", (N, H, dk, dv), torch.float32)
+    o = out if out is not None else torch.empty((N, H, dv), dtype=dt, device=q.device)
+    _check(o, "o", (N, H, dv), dt)
+    st = lib.gdr2_decode_step(N, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                              _ptr(w), _ptr(S), _ptr(o), _stream(stream))
+    _raise(lib, st)
+    return o
+
+
+def gdr2_backward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    lib = load_library()
+    return int(lib.gdr2_backward_workspace_bytes(B, T, H, dk, dv, GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
+
+
+def gdr2_backward(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, saved_states=None, *,
+                  want_dS0=True, workspace=None, stream=None):
+    """Gradients of <o, dO> + <S_T, dS_T>. Returns dict dq, dk, dv, dlog_alpha, db, dw, dS0."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("b", b, (B, T, H, dk)),
+                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H, dv)), ("dO", dO, (B, T, H, dv))):
+        _check(t, name, shp, dt)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32)
+    _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    _check(dS_T, "dS_T", (B, H, dk, dv), torch.float32)
+    nc = (T + CHUNK - 1) // CHUNK
+    _check(saved_states, "saved_states", (B, H, nc, dk, dv), torch.float32)
+    dev = q.device
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+         "dlog_alpha": torch.empty_like(log_alpha), "db": torch.empty_like(b), "dw": torch.empty_like(w),
+         "dS0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dS0 else None}
+    need = gdr2_backward_workspace_bytes(B, T, H, dk, dv, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = lib.gdr2_backward(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                           _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(saved_states), _ptr(g["dq"]),
+                           _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["db"]), _ptr(g["dw"]),
+                           _ptr(g["dS0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _raise(lib, st)
+    return g

@@ -1,0 +1,287 @@
+// bwd_simt.cu -- gate-aware GDR-2 backward on CUDA cores (fp32 arithmetic).
+//
+// Reverse-mode gradient of the recurrence of the Gated DeltaNet-2 note
+// (sec. 3: the backward passes through the asymmetric factor (I - k_t e_t^T);
+// the gate gradients follow the gated key e = b (.) k and the gated value
+// z = w (.) v). With Sb = Diag(a) S_{t-1}, delta = z - Sb^T e,
+// S_t = Sb + k delta^T and o_t = S_t^T q, one reverse token is
+//   dS  += q dO^T            dq = S_t dO
+//   dk   = dS delta          ddelta = dS^T k
+//   dw   = ddelta (.) v      dv = ddelta (.) w
+//   de   = -Sb ddelta        db = de (.) k,   dk += de (.) b
+//   dSb  = dS - e ddelta^T   dlog_alpha = rowsum(dSb (.) Sb)
+//   dS   = Diag(a) dSb
+//
+// Schedule: one CTA per (batch, head). The states entering each chunk of 64
+// tokens come from the forward (saved_states) or from a forward sweep here.
+// For each chunk, last to first, the CTA replays the chunk forward from its
+// entry state, keeping every token's state and delta in the workspace, then
+// walks the chunk backwards. dS lives in registers: thread (c, half) owns the
+// half row dS[c, half*dv/2 : (half+1)*dv/2]. Row reductions (over value
+// columns) finish with one shuffle between the two halves; column
+// reductions (over key channels) use a shuffle transpose-reduce inside a
+// warp, then shared memory across warps.
+
+#include "gdr2_common.cuh"
+#include "gdr2_launch.h"
+
+namespace gdr2 {
+namespace {
+
+constexpr int C = 64;
+
+__host__ __device__ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdLayout {
+    size_t cs_off, ts_off, dl_off, total;
+};
+
+__host__ __device__ inline BwdLayout bwd_layout(int B, int T, int H, int dk, int dv, bool need_cs)
+{
+    const size_t BH = (size_t)B * H;
+    const size_t NC = (size_t)(T + C - 1) / C;
+    BwdLayout L;
+    size_t off = 0;
+    L.cs_off = off;
+    if (need_cs) off += align256(BH * NC * dk * dv * sizeof(float));
+    L.ts_off = off;
+    off += align256(BH * (C + 1) * dk * dv * sizeof(float));
+    L.dl_off = off;
+    off += align256(BH * C * dv * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// Sum `vals` over the 16 lanes that share bit 4 of the lane id. On return
+// lane L (L = lane & 15) holds, in vals[0 .. N/16), the sums of the N/16
+// consecutive entries starting at (N/16) * L.
+template <int N>
+__device__ __forceinline__ void transpose_reduce16(float (&vals)[N], int lane)
+{
+#pragma unroll
+    for (int o = 8, n = N; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? vals[i] : vals[i + n / 2];
+            const float keep = upper ? vals[i + n / 2] : vals[i];
+            vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
+template <int DK, int DV>
+struct BwdSmem {
+    float red[2 * DK / 32][DV];  // per-warp column partials
+    float vec[DV];               // reduced column vector (delta or ddelta)
+    float z[DV], dO[DV], v[DV], w[DV];
+};
+
+template <typename TIn, int DK, int DV>
+__device__ __forceinline__ void load_row_gates(const BwdArgs &a, size_t ok, int c, float &kc, float &bc,
+                                               float &al)
+{
+    kc = to_f32(static_cast<const TIn *>(a.k)[ok + c]);
+    bc = to_f32(static_cast<const TIn *>(a.b)[ok + c]);
+    al = expf(clamp_log_alpha(a.log_alpha[ok + c]));
+}
+
+// One forward token on the register row S (this thread's half row). Leaves
+// delta in sm.vec and writes it to dl (when not null).
+template <typename TIn, int DK, int DV>
+__device__ __forceinline__ void fwd_token(const BwdArgs &a, BwdSmem<DK, DV> &sm, float (&S)[DV / 2], int t,
+                                          int c, int jb, int lane, int warp, int tid, float *dl)
+{
+    constexpr int HJ = DV / 2;
+    const int bb = blockIdx.x / a.H, h = blockIdx.x % a.H;
+    const size_t ok = (((size_t)bb * a.T + t) * a.H + h) * DK;
+    const size_t ov = (((size_t)bb * a.T + t) * a.H + h) * DV;
+    if (tid < DV)
+        sm.z[tid] = to_f32(static_cast<const TIn *>(a.w)[ov + tid]) * to_f32(static_cast<const TIn *>(a.v)[ov + tid]);
+    float kc, bc, al;
+    load_row_gates<TIn, DK, DV>(a, ok, c, kc, bc, al);
+    const float ae = al * bc * kc;
+    float part[HJ];
+#pragma unroll
+    for (int j = 0; j < HJ; ++j) part[j] = ae * S[j];
+    transpose_reduce16<HJ>(part, lane);
+    constexpr int PER = HJ / 16;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) sm.red[warp][jb + PER * (lane & 15) + i] = part[i];
+    __syncthreads();
+    if (tid < DV) {
+        float r = 0.f;
+#pragma unroll
+        for (int wv = 0; wv < 2 * DK / 32; ++wv) r += sm.red[wv][tid];
+        const float d = sm.z[tid] - r;
+        sm.vec[tid] = d;
+        if (dl) dl[tid] = d;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < HJ; ++j) S[j] = fmaf(al, S[j], kc * sm.vec[jb + j]);
+}
+
+template <typename TIn, int DK, int DV>
+__global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, float *TS, float *DL)
+{
+    constexpr int NT = 2 * DK;
+    constexpr int HJ = DV / 2;
+    constexpr int PER = HJ / 16;
+    __shared__ BwdSmem<DK, DV> sm;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = warp * 16 + (lane & 15);
+    const int half = lane >> 4;
+    const int jb = half * HJ;
+    const int bh = blockIdx.x;
+    const int bb = bh / a.H, h = bh % a.H;
+    const int T = a.T, H = a.H;
+    const int NC = (T + C - 1) / C;
+    const size_t SS = (size_t)DK * DV;
+    float *ts = TS + (size_t)bh * (C + 1) * SS;
+    float *dl = DL + (size_t)bh * C * DV;
+    (void)NT;
+
+    float S[HJ];
+    // ---- states entering each chunk ----
+    const float *chunk_states;
+    if (a.saved_states) {
+        chunk_states = a.saved_states + (size_t)bh * NC * SS;
+    } else {
+        float *cs = CS + (size_t)bh * NC * SS;
+#pragma unroll
+        for (int j = 0; j < HJ; ++j) S[j] = a.S0 ? a.S0[(size_t)bh * SS + (size_t)c * DV + jb + j] : 0.f;
+        for (int t = 0; t < T; ++t) {
+            if (t % C == 0) {
+#pragma unroll
+                for (int j = 0; j < HJ; ++j) cs[(size_t)(t / C) * SS + (size_t)c * DV + jb + j] = S[j];
+            }
+            fwd_token<TIn, DK, DV>(a, sm, S, t, c, jb, lane, warp, tid, nullptr);
+        }
+        chunk_states = cs;
+    }
+
+    float dS[HJ];
+#pragma unroll
+    for (int j = 0; j < HJ; ++j) dS[j] = a.dS_T ? a.dS_T[(size_t)bh * SS + (size_t)c * DV + jb + j] : 0.f;
+
+    for (int n = NC - 1; n >= 0; --n) {
+        const int t0 = n * C;
+        const int Cn = min(C, T - t0);
+        // ---- replay the chunk forward, keeping every state and delta ----
+#pragma unroll
+        for (int j = 0; j < HJ; ++j) {
+            S[j] = chunk_states[(size_t)n * SS + (size_t)c * DV + jb + j];
+            ts[(size_t)c * DV + jb + j] = S[j];
+        }
+        for (int t = 0; t < Cn; ++t) {
+            fwd_token<TIn, DK, DV>(a, sm, S, t0 + t, c, jb, lane, warp, tid, dl + (size_t)t * DV);
+#pragma unroll
+            for (int j = 0; j < HJ; ++j) ts[(size_t)(t + 1) * SS + (size_t)c * DV + jb + j] = S[j];
+        }
+        // Each thread reads back only the rows and deltas it wrote itself.
+        __syncthreads();
+        // ---- reverse tokens ----
+        for (int t = Cn - 1; t >= 0; --t) {
+            const int tg = t0 + t;
+            const size_t ok = (((size_t)bb * T + tg) * H + h) * DK;
+            const size_t ov = (((size_t)bb * T + tg) * H + h) * DV;
+            if (tid < DV) {
+                sm.dO[tid] = to_f32(static_cast<const TIn *>(a.dO)[ov + tid]);
+                sm.v[tid] = to_f32(static_cast<const TIn *>(a.v)[ov + tid]);
+                sm.w[tid] = to_f32(static_cast<const TIn *>(a.w)[ov + tid]);
+                sm.vec[tid] = dl[(size_t)t * DV + tid];  // delta_t
+            }
+            const float qc = to_f32(static_cast<const TIn *>(a.q)[ok + c]);
+            float kc, bc, al;
+            load_row_gates<TIn, DK, DV>(a, ok, c, kc, bc, al);
+            const float ec = bc * kc;
+            __syncthreads();
+            const float *St = ts + (size_t)(t + 1) * SS + (size_t)c * DV + jb;
+            const float *Sp = ts + (size_t)t * SS + (size_t)c * DV + jb;
+            float dq = 0.f, dk = 0.f;
+            float part[HJ];
+#pragma unroll
+            for (int j = 0; j < HJ; ++j) {
+                const float dOj = sm.dO[jb + j];
+                dq = fmaf(St[j], dOj, dq);
+                dS[j] = fmaf(qc, dOj, dS[j]);
+                dk = fmaf(dS[j], sm.vec[jb + j], dk);
+                part[j] = dS[j] * kc;
+            }
+            transpose_reduce16<HJ>(part, lane);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) sm.red[warp][jb + PER * (lane & 15) + i] = part[i];
+            __syncthreads();
+            if (tid < DV) {
+                float dd = 0.f;
+#pragma unroll
+                for (int wv = 0; wv < 2 * DK / 32; ++wv) dd += sm.red[wv][tid];
+                sm.vec[tid] = dd;  // ddelta_t
+                static_cast<TIn *>(a.gw)[ov + tid] = from_f32<TIn>(dd * sm.v[tid]);
+                static_cast<TIn *>(a.gv)[ov + tid] = from_f32<TIn>(dd * sm.w[tid]);
+            }
+            __syncthreads();
+            float de = 0.f, dla = 0.f;
+#pragma unroll
+            for (int j = 0; j < HJ; ++j) {
+                const float dd = sm.vec[jb + j];
+                const float sb = al * Sp[j];
+                de = fmaf(-sb, dd, de);
+                const float g = fmaf(-ec, dd, dS[j]);
+                dla = fmaf(g, sb, dla);
+                dS[j] = al * g;
+            }
+            dq += __shfl_xor_sync(0xffffffffu, dq, 16);
+            dk += __shfl_xor_sync(0xffffffffu, dk, 16);
+            de += __shfl_xor_sync(0xffffffffu, de, 16);
+            dla += __shfl_xor_sync(0xffffffffu, dla, 16);
+            if (half == 0) {
+                static_cast<TIn *>(a.gq)[ok + c] = from_f32<TIn>(dq);
+                static_cast<TIn *>(a.gk)[ok + c] = from_f32<TIn>(fmaf(de, bc, dk));
+                static_cast<TIn *>(a.gb)[ok + c] = from_f32<TIn>(de * kc);
+                a.glog_alpha[ok + c] = dla;
+            }
+            __syncthreads();
+        }
+    }
+    if (a.gS0) {
+#pragma unroll
+        for (int j = 0; j < HJ; ++j) a.gS0[(size_t)bh * SS + (size_t)c * DV + jb + j] = dS[j];
+    }
+}
+
+template <typename TIn, int DK, int DV>
+cudaError_t launch_t(const BwdArgs &a, cudaStream_t s)
+{
+    const BwdLayout L = bwd_layout(a.B, a.T, a.H, a.dk, a.dv, a.saved_states == nullptr);
+    char *ws = static_cast<char *>(a.workspace);
+    bwd_kernel<TIn, DK, DV><<<a.B * a.H, 2 * DK, 0, s>>>(
+        a, reinterpret_cast<float *>(ws + L.cs_off), reinterpret_cast<float *>(ws + L.ts_off),
+        reinterpret_cast<float *>(ws + L.dl_off));
+    return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t launch_dt(const BwdArgs &a, cudaStream_t s)
+{
+    if (a.dk == 128 && a.dv == 128) return launch_t<TIn, 128, 128>(a, s);
+    if (a.dk == 128 && a.dv == 64) return launch_t<TIn, 128, 64>(a, s);
+    if (a.dk == 64 && a.dv == 128) return launch_t<TIn, 64, 128>(a, s);
+    return launch_t<TIn, 64, 64>(a, s);
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool /*bf16*/)
+{
+    return bwd_layout(B, T, H, dk, dv, true).total;
+}
+
+cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s)
+{
+    if (a.B * a.H == 0) return cudaSuccess;
+    return a.bf16 ? launch_dt<__nv_bfloat16>(a, s) : launch_dt<float>(a, s);
+}
+
+}  // namespace gdr2

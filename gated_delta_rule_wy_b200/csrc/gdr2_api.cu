@@ -1,0 +1,221 @@
+// gdr2_api.cu -- the extern "C" entry points of libgdr2.so.
+//
+// Host-side argument validation, the per-device status word and the
+// dispatch to the kernels. Nothing here allocates device memory.
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gdr2.h"
+#include "gdr2_common.cuh"
+#include "gdr2_launch.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+gdr2_status fail(gdr2_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+// One status word per device. Kernels OR bits into it (gdr2::kStatus*).
+__device__ unsigned g_status_word;
+
+constexpr int kMaxDevices = 64;
+unsigned *g_status_ptr[kMaxDevices];
+std::once_flag g_status_once[kMaxDevices];
+
+unsigned *status_ptr(int dev)
+{
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_status_once[dev], [dev] {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) g_status_ptr[dev] = static_cast<unsigned *>(p);
+    });
+    return g_status_ptr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdr2_status check_dims(int B, int T, int H, int dk, int dv)
+{
+    if (B < 0 || T < 0 || H < 0) return fail(GDR2_ERR_INVALID_ARG, "negative size (B=%d T=%d H=%d)", B, T, H);
+    if (dk <= 0 || dv <= 0) return fail(GDR2_ERR_INVALID_ARG, "dk and dv must be positive (dk=%d dv=%d)", dk, dv);
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(GDR2_ERR_UNSUPPORTED, "dk and dv must be 64 or 128 (dk=%d dv=%d)", dk, dv);
+    if ((long long)B * T * H * (dk > dv ? dk : dv) > (1ll << 40))
+        return fail(GDR2_ERR_INVALID_ARG, "problem too large");
+    return GDR2_OK;
+}
+
+gdr2_status check_ptr(const void *p, const char *name, bool nullable)
+{
+    if (!p) return nullable ? GDR2_OK : fail(GDR2_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(GDR2_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return GDR2_OK;
+}
+
+#define GDR2_TRY(expr)                      \
+    do {                                    \
+        gdr2_status st_ = (expr);           \
+        if (st_ != GDR2_OK) return st_;     \
+    } while (0)
+
+gdr2_status check_dtype(gdr2_dtype dt)
+{
+    if (dt != GDR2_F32 && dt != GDR2_BF16) return fail(GDR2_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    return GDR2_OK;
+}
+
+gdr2_status device_status(unsigned **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GDR2_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    *out = status_ptr(dev);
+    if (!*out) return fail(GDR2_ERR_CUDA, "cannot resolve the device status word on device %d", dev);
+    return GDR2_OK;
+}
+
+gdr2_status launched(cudaError_t e, const char *what)
+{
+    if (e != cudaSuccess) return fail(GDR2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    g_last_error[0] = '\0';
+    return GDR2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr2_abi_version(void) { return GDR2_ABI_VERSION; }
+
+const char *gdr2_last_error(void) { return g_last_error; }
+
+gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                         const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                         void *o, float *S_T, float *saved_states, void *stream)
+{
+    GDR2_TRY(check_dims(B, T, H, dk, dv));
+    GDR2_TRY(check_dtype(dt));
+    const bool has_tokens = (long long)B * T * H > 0;
+    GDR2_TRY(check_ptr(q, "q", !has_tokens));
+    GDR2_TRY(check_ptr(k, "k", !has_tokens));
+    GDR2_TRY(check_ptr(v, "v", !has_tokens));
+    GDR2_TRY(check_ptr(log_alpha, "log_alpha", !has_tokens));
+    GDR2_TRY(check_ptr(b, "b", !has_tokens));
+    GDR2_TRY(check_ptr(w, "w", !has_tokens));
+    GDR2_TRY(check_ptr(o, "o", !has_tokens));
+    GDR2_TRY(check_ptr(S0, "S0", true));
+    GDR2_TRY(check_ptr(S_T, "S_T", true));
+    GDR2_TRY(check_ptr(saved_states, "saved_states", true));
+    if ((long long)B * H == 0) return GDR2_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // No tokens: S_T = S0 (or zeros); nothing to save.
+        if (S_T && S_T != S0) {
+            const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+            cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(S_T, 0, bytes, s);
+            return launched(e, "gdr2_forward (T = 0)");
+        }
+        return GDR2_OK;
+    }
+    gdr2::FwdArgs a{B, T, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S0, o, S_T, saved_states, nullptr};
+    GDR2_TRY(device_status(&a.status));
+    if (gdr2::forward_tc_supported(a)) return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward (tcgen05)");
+    return launched(gdr2::launch_forward_simt(a, s), "gdr2_forward (simt)");
+}
+
+gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                             const void *v, const float *log_alpha, const void *b, const void *w, float *S,
+                             void *o, void *stream)
+{
+    GDR2_TRY(check_dims(N, 1, H, dk, dv));
+    GDR2_TRY(check_dtype(dt));
+    const bool any = (long long)N * H > 0;
+    GDR2_TRY(check_ptr(q, "q", !any));
+    GDR2_TRY(check_ptr(k, "k", !any));
+    GDR2_TRY(check_ptr(v, "v", !any));
+    GDR2_TRY(check_ptr(log_alpha, "log_alpha", !any));
+    GDR2_TRY(check_ptr(b, "b", !any));
+    GDR2_TRY(check_ptr(w, "w", !any));
+    GDR2_TRY(check_ptr(S, "S", !any));
+    GDR2_TRY(check_ptr(o, "o", !any));
+    if (!any) return GDR2_OK;
+    gdr2::DecodeArgs a{N, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S, o, nullptr};
+    GDR2_TRY(device_status(&a.status));
+    return launched(gdr2::launch_decode(a, static_cast<cudaStream_t>(stream)), "gdr2_decode_step");
+}
+
+size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt)
+{
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return 0;
+    return gdr2::backward_workspace_bytes(B, T, H, dk, dv, dt == GDR2_BF16);
+}
+
+gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                          const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                          const void *dO, const float *dS_T, const float *saved_states, void *dq, void *dk_,
+                          void *dv_, float *dlog_alpha, void *db, void *dw, float *dS0, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    GDR2_TRY(check_dims(B, T, H, dk, dv));
+    GDR2_TRY(check_dtype(dt));
+    const bool has_tokens = (long long)B * T * H > 0;
+    const char *names[] = {"q", "k", "v", "log_alpha", "b", "w", "dO", "dq", "dk", "dv", "dlog_alpha", "db", "dw"};
+    const void *ptrs[] = {q, k, v, log_alpha, b, w, dO, dq, dk_, dv_, dlog_alpha, db, dw};
+    for (int i = 0; i < 13; ++i) GDR2_TRY(check_ptr(ptrs[i], names[i], !has_tokens));
+    GDR2_TRY(check_ptr(S0, "S0", true));
+    GDR2_TRY(check_ptr(dS_T, "dS_T", true));
+    GDR2_TRY(check_ptr(saved_states, "saved_states", true));
+    GDR2_TRY(check_ptr(dS0, "dS0", true));
+    if ((long long)B * H == 0) return GDR2_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (dS0) {
+            const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+            cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, bytes, cudaMemcpyDeviceToDevice, s)
+                                 : cudaMemsetAsync(dS0, 0, bytes, s);
+            return launched(e, "gdr2_backward (T = 0)");
+        }
+        return GDR2_OK;
+    }
+    const size_t need = gdr2::backward_workspace_bytes(B, T, H, dk, dv, dt == GDR2_BF16);
+    if (!workspace || workspace_bytes < need)
+        return fail(GDR2_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    gdr2::BwdArgs a{B, T, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S0, dO, dS_T, saved_states,
+                    dq, dk_, dv_, dlog_alpha, db, dw, dS0, workspace, workspace_bytes, nullptr};
+    GDR2_TRY(device_status(&a.status));
+    return launched(gdr2::launch_backward(a, s), "gdr2_backward");
+}
+
+gdr2_status gdr2_sync_status(void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(GDR2_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    unsigned *dev_word = nullptr;
+    GDR2_TRY(device_status(&dev_word));
+    unsigned word = 0;
+    e = cudaMemcpyFromSymbolAsync(&word, g_status_word, sizeof(word), 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dev_word, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(GDR2_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(e));
+    if (word & gdr2::kStatusTimeout)
+        return fail(GDR2_ERR_TIMEOUT, "a kernel gave up a bounded device wait (status 0x%x)", word);
+    g_last_error[0] = '\0';
+    return GDR2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// gdr2_launch.h -- host-side launchers behind the C ABI (internal).
+// Each returns cudaSuccess or the launch error; argument checks happen in
+// gdr2_api.cu before any of these is called.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdr2 {
+
+struct FwdArgs {
+    int B, T, H, dk, dv;
+    bool bf16;
+    const void *q, *k, *v;
+    const float *log_alpha;
+    const void *b, *w;
+    const float *S0;
+    void *o;
+    float *S_T;
+    float *saved_states;
+    unsigned *status;  // device status word
+};
+
+struct DecodeArgs {
+    int N, H, dk, dv;
+    bool bf16;
+    const void *q, *k, *v;
+    const float *log_alpha;
+    const void *b, *w;
+    float *S;
+    void *o;
+    unsigned *status;
+};
+
+struct BwdArgs {
+    int B, T, H, dk, dv;
+    bool bf16;
+    const void *q, *k, *v;
+    const float *log_alpha;
+    const void *b, *w;
+    const float *S0;
+    const void *dO;
+    const float *dS_T;
+    const float *saved_states;
+    void *gq, *gk, *gv;  // gradient outputs dq, dk, dv
+    float *glog_alpha;
+    void *gb, *gw;
+    float *gS0;
+    void *workspace;
+    size_t workspace_bytes;
+    unsigned *status;
+};
+
+cudaError_t launch_forward_simt(const FwdArgs &a, cudaStream_t s);
+cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s);
+bool forward_tc_supported(const FwdArgs &a);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf16);
+cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s);
+
+}  // namespace gdr2

@@ -66,13 +66,17 @@ def _l2norm_rows(x: torch.Tensor) -> torch.Tensor:
 
 
 def make_token_inputs(shape_k, shape_v, dtype, decay_shift, gen, normalise_qk=True):
-    """Draw q, k, v, log_alpha, b, w with the distributions in the module docstring."""
-    q = torch.randn(shape_k, generator=gen)
-    k = torch.randn(shape_k, generator=gen)
-    v = torch.randn(shape_v, generator=gen)
-    la = -torch.nn.functional.softplus(torch.randn(shape_k, generator=gen) + decay_shift)
-    b = torch.sigmoid(torch.randn(shape_k, generator=gen))
-    w = torch.sigmoid(torch.randn(shape_v, generator=gen))
+    """Draw q, k, v, log_alpha, b, w with the distributions in the module docstring.
+
+    Tensors are drawn on the generator's device (CPU, or CUDA for long decode runs).
+    """
+    dev = gen.device
+    q = torch.randn(shape_k, generator=gen, device=dev)
+    k = torch.randn(shape_k, generator=gen, device=dev)
+    v = torch.randn(shape_v, generator=gen, device=dev)
+    la = -torch.nn.functional.softplus(torch.randn(shape_k, generator=gen, device=dev) + decay_shift)
+    b = torch.sigmoid(torch.randn(shape_k, generator=gen, device=dev))
+    w = torch.sigmoid(torch.randn(shape_v, generator=gen, device=dev))
     if normalise_qk:
         q, k = _l2norm_rows(q), _l2norm_rows(k)
     return (q.to(dtype), k.to(dtype), v.to(dtype), la.to(torch.float32), b.to(dtype), w.to(dtype))

@@ -1,0 +1,158 @@
+/*
+ * gdr2.h -- C ABI of libgdr2.so, the B200 (sm_100a) implementation of the
+ * Gated Delta Rule-2 (GDR-2) token mixer from "Gated DeltaNet-2: Decoupling
+ * Erase and Write in Linear Attention" (Hatamizadeh, Choi, Kautz).
+ *
+ * The operation (per batch index b and head h, independently):
+ *
+ *   e_t = b_t (.) k_t,   z_t = w_t (.) v_t,   a_t = exp(log_alpha_t)
+ *   S_t = (I - k_t e_t^T) Diag(a_t) S_{t-1} + k_t z_t^T          (dk x dv state)
+ *   o_t = S_t^T q_t
+ *
+ * Sources: the note's sec. 3 forward-pass paragraph (gated key and value,
+ * decay, read), sec. 2 fast-weight objective and the sec. 3 gate-aware
+ * backward paragraph (erase outer product along k: the asymmetric factor
+ * (I - k_t e_t^T)); sec. 3 chunkwise paragraph (decay-normalised state and
+ * WY form used by the forward kernel); sec. 1 (constant-memory recurrent
+ * decoding).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers:   all tensor pointers are DEVICE pointers (CUDA global memory) of
+ *             the current device, contiguous in the layouts below, 16-byte
+ *             aligned. The caller owns every buffer; the library allocates no
+ *             device memory. Scratch, where an entry point needs any, is a
+ *             caller buffer sized by the matching *_workspace_bytes query.
+ * Layouts:    token tensors are token-major:
+ *               q, k, log_alpha, b          [B, T, H, dk]
+ *               v, w, o                     [B, T, H, dv]
+ *             states are [B, H, dk, dv] fp32, row = key channel c,
+ *             column = value channel j (dv contiguous).
+ * Dtypes:     q, k, v, b, w, o and their gradients have the dtype `dt`
+ *             (fp32 or bf16); log_alpha, its gradient and every state are
+ *             fp32. Arithmetic is fp32 throughout; bf16 outputs are rounded
+ *             to nearest even from fp32.
+ * Decay:      log_alpha must not be NaN; values below -64 are treated as
+ *             -64 (alpha = 1.6e-28, a reset to fp32 precision).
+ * Streams:    `stream` is a cudaStream_t (NULL = legacy default stream).
+ *             Every call is asynchronous on that stream and returns once
+ *             the work is enqueued.
+ * Errors:     argument errors are detected on the host before any launch and
+ *             return GDR2_ERR_INVALID_ARG or GDR2_ERR_UNSUPPORTED with no
+ *             work enqueued; launch failures return GDR2_ERR_CUDA. Kernels
+ *             that wait on hardware barriers bound every wait; a kernel that
+ *             gives up records it in a device status word that
+ *             gdr2_sync_status() reports as GDR2_ERR_TIMEOUT. No exception
+ *             or abort crosses the ABI. gdr2_last_error() describes the last
+ *             non-OK status of the calling thread.
+ * Sizes:      dk and dv must each be 64 or 128; B, T, H >= 0 (an empty
+ *             problem is a no-op apart from copying S0 to S_T).
+ */
+#ifndef GDR2_H
+#define GDR2_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDR2_ABI_VERSION 1
+#define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
+
+typedef enum {
+    GDR2_OK = 0,
+    GDR2_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, ... */
+    GDR2_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. dk = 96)   */
+    GDR2_ERR_CUDA = 3,        /* launch or runtime failure                  */
+    GDR2_ERR_TIMEOUT = 4      /* a kernel gave up a bounded device wait     */
+} gdr2_status;
+
+typedef enum {
+    GDR2_F32 = 0,
+    GDR2_BF16 = 1
+} gdr2_dtype;
+
+/* ABI version of the loaded library (GDR2_ABI_VERSION it was built with). */
+int gdr2_abi_version(void);
+
+/* Human-readable description of the calling thread's last non-OK status
+ * (empty string if none). The pointer stays valid until the next call from
+ * the same thread. */
+const char *gdr2_last_error(void);
+
+/*
+ * gdr2_forward -- chunkwise forward over whole sequences (prefill/training).
+ *   Computes o_t for every token and the final state S_T, starting from S0.
+ *   Gated DeltaNet-2 note sec. 3: per chunk of GDR2_CHUNK tokens the decay
+ *   is absorbed into the gated keys (decay-normalised state), the
+ *   strictly-lower system (I + A) is solved in UT form, the WY factors give
+ *   the chunk's pseudo-values, and the state is carried between chunks in
+ *   fp32.
+ * in:  q, k [B,T,H,dk] dt; v [B,T,H,dv] dt; log_alpha [B,T,H,dk] fp32;
+ *      b [B,T,H,dk] dt; w [B,T,H,dv] dt;
+ *      S0 [B,H,dk,dv] fp32 or NULL (zero initial state).
+ * out: o [B,T,H,dv] dt; S_T [B,H,dk,dv] fp32 or NULL (not written);
+ *      saved_states [B,H,ceil(T/64),dk,dv] fp32 or NULL: the state entering
+ *      each chunk (chunk 0 receives S0), for gdr2_backward.
+ * Input and output buffers must not overlap (S0 == S_T is allowed).
+ */
+gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
+                         const void *q, const void *k, const void *v,
+                         const float *log_alpha, const void *b, const void *w,
+                         const float *S0, void *o, float *S_T, float *saved_states,
+                         void *stream);
+
+/*
+ * gdr2_decode_step -- one recurrent token for N*H resident states
+ *   (constant-memory decoding, Gated DeltaNet-2 note sec. 1; the per-token
+ *   steps of sec. 3). One read and one write of S: with r = S^T(a (.) e) and
+ *   s = S^T(a (.) q) taken from the old state, o = s + (z - r)(k . q) and
+ *   S <- Diag(a) S + k (z - r)^T.
+ * in:  q, k, b [N,H,dk] dt; v, w [N,H,dv] dt; log_alpha [N,H,dk] fp32.
+ * in/out: S [N,H,dk,dv] fp32, updated in place.
+ * out: o [N,H,dv] dt.
+ */
+gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt,
+                             const void *q, const void *k, const void *v,
+                             const float *log_alpha, const void *b, const void *w,
+                             float *S, void *o, void *stream);
+
+/* Bytes of device scratch gdr2_backward needs for this problem. */
+size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt);
+
+/*
+ * gdr2_backward -- gate-aware backward (Gated DeltaNet-2 note sec. 3):
+ *   gradients of L = <o, dO> + <S_T, dS_T> with respect to q, k, v,
+ *   log_alpha, b, w and S0, through the asymmetric factor (I - k_t e_t^T).
+ * in:  forward inputs as in gdr2_forward (S0 NULL = zeros); dO [B,T,H,dv] dt;
+ *      dS_T [B,H,dk,dv] fp32 or NULL (zero);
+ *      saved_states as written by gdr2_forward for the same inputs, or NULL
+ *      (the states are recomputed).
+ * out: dq, dk_, db [B,T,H,dk] dt; dv_, dw [B,T,H,dv] dt;
+ *      dlog_alpha [B,T,H,dk] fp32; dS0 [B,H,dk,dv] fp32 or NULL.
+ * scratch: workspace of at least gdr2_backward_workspace_bytes(...) bytes,
+ *      256-byte aligned; its contents on entry do not matter.
+ */
+gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
+                          const void *q, const void *k, const void *v,
+                          const float *log_alpha, const void *b, const void *w,
+                          const float *S0, const void *dO, const float *dS_T,
+                          const float *saved_states,
+                          void *dq, void *dk_, void *dv_, float *dlog_alpha,
+                          void *db, void *dw, float *dS0,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdr2_sync_status -- wait for `stream`, then report and clear the device
+ * status word: GDR2_ERR_TIMEOUT if any kernel of this library gave up a
+ * bounded wait since the last call, GDR2_ERR_CUDA on an asynchronous CUDA
+ * error, GDR2_OK otherwise.
+ */
+gdr2_status gdr2_sync_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR2_H */

@@ -1,0 +1,96 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+``include/gdr2.h`` declares, and rejects bad arguments on the host before any
+launch (so no device work is enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_wy_b200 as g
+from gated_delta_rule_wy_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_wy_b200 import build
+
+    build.build()
+    return g.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "gdr2.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdr2_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == sorted(binding.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libgdr2.so does not export {name}"
+
+
+def test_abi_version(lib):
+    assert lib.gdr2_abi_version() == 1
+
+
+NULL11 = [None] * 11
+
+
+@pytest.mark.parametrize("dims,dt,status", [
+    ((1, 4, 1, 96, 64), 1, binding.GDR2_ERR_UNSUPPORTED),
+    ((1, 4, 1, 64, 32), 1, binding.GDR2_ERR_UNSUPPORTED),
+    ((-1, 4, 1, 64, 64), 1, binding.GDR2_ERR_INVALID_ARG),
+    ((1, -4, 1, 64, 64), 1, binding.GDR2_ERR_INVALID_ARG),
+    ((1, 4, 1, 0, 64), 1, binding.GDR2_ERR_INVALID_ARG),
+    ((1, 4, 1, 64, 64), 7, binding.GDR2_ERR_INVALID_ARG),
+    ((1, 4, 1, 64, 64), 1, binding.GDR2_ERR_INVALID_ARG),  # NULL q with tokens
+])
+def test_forward_rejects_bad_arguments(lib, dims, dt, status):
+    assert lib.gdr2_forward(*dims, dt, *NULL11) == status
+    assert lib.gdr2_last_error()
+
+
+def test_forward_rejects_misaligned_pointer(lib):
+    p = [ctypes.c_void_p(0x10000)] * 11
+    p[2] = ctypes.c_void_p(0x10008)  # v
+    assert lib.gdr2_forward(1, 4, 1, 64, 64, 1, *p) == binding.GDR2_ERR_INVALID_ARG
+    assert b"v is not 16-byte aligned" in lib.gdr2_last_error()
+
+
+def test_decode_rejects_bad_arguments(lib):
+    assert lib.gdr2_decode_step(2, 2, 128, 96, 1, *([None] * 9)) == binding.GDR2_ERR_UNSUPPORTED
+    assert lib.gdr2_decode_step(2, 2, 128, 128, 1, *([None] * 9)) == binding.GDR2_ERR_INVALID_ARG
+    # an empty batch is a no-op, even with NULL pointers
+    assert lib.gdr2_decode_step(0, 16, 128, 128, 1, *([None] * 9)) == binding.GDR2_OK
+
+
+def test_empty_problems_need_no_pointers(lib):
+    assert lib.gdr2_forward(0, 128, 16, 128, 128, 1, *NULL11) == binding.GDR2_OK
+    assert lib.gdr2_forward(4, 64, 0, 128, 128, 1, *NULL11) == binding.GDR2_OK
+
+
+def test_backward_workspace_query_and_checks(lib):
+    n = lib.gdr2_backward_workspace_bytes(2, 4096, 16, 128, 128, 1)
+    # chunk states + one chunk of token states + deltas, per (batch, head)
+    BH, NC, SS = 32, 64, 128 * 128 * 4
+    assert n >= BH * NC * SS + BH * 65 * SS
+    assert n % 256 == 0
+    p = [ctypes.c_void_p(0x10000)] * 17
+    st = lib.gdr2_backward(2, 64, 16, 128, 128, 1, *p, ctypes.c_size_t(16), ctypes.c_void_p(0))
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
+    assert lib.gdr2_backward_workspace_bytes(-1, 1, 1, 64, 64, 1) == 0
+
+
+def test_binding_validates_before_calling():
+    import torch
+
+    q = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdr2_forward(q, q, q, q, q, q)

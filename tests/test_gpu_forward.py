@@ -1,0 +1,153 @@
+"""GPU parity of gdr2_forward against the fp64 oracle (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_wy_b200 import gdr2_forward, gdr2_sync_status
+from gated_delta_rule_wy_b200 import inputs as I
+from parity import TOL, assert_close, head_slice, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(x: I.FwdInputs, **kw):
+    d = x.to("cuda")
+    o, S_T, saved = gdr2_forward(d.q, d.k, d.v, d.log_alpha, d.b, d.w, d.S0, **kw)
+    gdr2_sync_status()
+    return o, S_T, saved
+
+
+def run_oracle(x: I.FwdInputs):
+    n = x.as_numpy64()
+    return oracle.forward(n["q"], n["k"], n["v"], n["log_alpha"], n["b"], n["w"], S0=n["S0"])
+
+
+def check(x, what, tol=None):
+    tol = tol or TOL[x.q.dtype]
+    o, S_T, _ = run_gpu(x)
+    o_ref, S_ref = run_oracle(x)
+    eo = assert_close(o, o_ref, tol, f"{what}: o")
+    es = assert_close(S_T, S_ref, tol, f"{what}: S_T")
+    return eo, es
+
+
+def test_small_f32_workload():
+    """B=1 H=1 T=256 d=64 fp32 (the oracle-scale workload), bound 1e-4."""
+    check(I.make_forward_inputs(**I.FWD_SMALL_F32), "fp32 T=256 d=64")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("T", [1, 5, 63, 64, 65, 130])
+def test_f32_ragged_with_initial_state(dk, dv, T):
+    x = I.make_forward_inputs(B=2, H=2, T=T, dk=dk, dv=dv, dtype=torch.float32, seed=10 + T, with_S0=True)
+    check(x, f"fp32 T={T} dk={dk} dv={dv}")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64)])
+def test_bf16_multi_chunk_ragged(dk, dv):
+    x = I.make_forward_inputs(B=2, H=3, T=200, dk=dk, dv=dv, dtype=torch.bfloat16, decay_shift=2.0,
+                              seed=21, with_S0=True)
+    check(x, f"bf16 T=200 dk={dk} dv={dv}")
+
+
+def test_bf16_slow_decay():
+    """Decay law of the small workload (log alpha = -softplus(N(0,1))) on the bf16 path."""
+    x = I.make_forward_inputs(B=1, H=4, T=333, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=0.0, seed=22)
+    check(x, "bf16 slow decay")
+
+
+def test_empty_sequence_copies_state():
+    x = I.make_forward_inputs(B=2, H=2, T=0, dk=128, dv=128, dtype=torch.bfloat16, seed=3, with_S0=True)
+    o, S_T, _ = run_gpu(x)
+    assert o.shape == (2, 0, 2, 128)
+    assert torch.equal(S_T.cpu(), x.S0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_saved_states_are_chunk_entry_states(dtype):
+    T = 150
+    x = I.make_forward_inputs(B=1, H=2, T=T, dk=128, dv=128, dtype=dtype, decay_shift=2.0, seed=4, with_S0=True)
+    _, _, saved = run_gpu(x, save_states=True)
+    n = x.as_numpy64()
+    for c, t0 in enumerate(range(0, T, 64)):
+        _, S_ref = oracle.forward(n["q"][:, :t0], n["k"][:, :t0], n["v"][:, :t0], n["log_alpha"][:, :t0],
+                                  n["b"][:, :t0], n["w"][:, :t0], S0=n["S0"])
+        assert_close(saved[:, :, c], S_ref, TOL[dtype], f"saved state of chunk {c}")
+
+
+def _edit(x: I.FwdInputs, **fields) -> I.FwdInputs:
+    d = dict(x.__dict__)
+    d.update(fields)
+    return I.FwdInputs(**d)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("case", ["reset", "no_erase", "full_erase", "erase_range_2", "no_decay",
+                                  "strong_decay", "one_hot_keys", "kda_gates"])
+def test_degenerate_cases(dtype, case):
+    x = I.make_forward_inputs(B=1, H=2, T=160, dk=128, dv=128, dtype=dtype, decay_shift=1.0, seed=5, with_S0=True)
+    la, b, k, w = x.log_alpha.clone(), x.b.clone(), x.k.clone(), x.w.clone()
+    if case == "reset":  # alpha = 0 at a few tokens: the memory clears
+        la[:, [3, 64, 100, 159]] = float("-inf")
+    elif case == "no_erase":
+        b.zero_()
+    elif case == "full_erase":
+        b.fill_(1.0)
+    elif case == "erase_range_2":  # the erase-range ablation, b in [0, 2]
+        b = (b.float() * 2.0).to(dtype)
+    elif case == "no_decay":
+        la.zero_()
+    elif case == "strong_decay":  # alpha ~ 1e-13 per token: exercises the decay-range handling
+        la = la - 30.0
+    elif case == "one_hot_keys":
+        k = torch.nn.functional.one_hot(torch.randint(0, 128, k.shape[:-1], generator=torch.Generator().manual_seed(0)),
+                                        128).to(dtype)
+    elif case == "kda_gates":  # b = w = beta * 1
+        beta = torch.rand(b.shape[:-1], generator=torch.Generator().manual_seed(1))
+        b = beta[..., None].expand_as(b).contiguous().to(dtype)
+        w = beta[..., None].expand_as(w).contiguous().to(dtype)
+    check(_edit(x, log_alpha=la, b=b, k=k, w=w), f"{case} ({dtype})")
+
+
+def test_split_sequence_resumes_from_state():
+    """forward(x) equals forward of the tail started from the head's final state."""
+    x = I.make_forward_inputs(B=2, H=4, T=300, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=2.0, seed=6)
+    d = x.to("cuda")
+    o, S_T, _ = gdr2_forward(d.q, d.k, d.v, d.log_alpha, d.b, d.w, None)
+    cut = 137
+    o1, S1, _ = gdr2_forward(*(t[:, :cut].contiguous() for t in (d.q, d.k, d.v, d.log_alpha, d.b, d.w)), None)
+    o2, S2, _ = gdr2_forward(*(t[:, cut:].contiguous() for t in (d.q, d.k, d.v, d.log_alpha, d.b, d.w)), S1)
+    gdr2_sync_status()
+    assert rel_err(torch.cat([o1, o2], 1), o.double().cpu().numpy()) <= 2e-2
+    assert rel_err(S2, S_T.double().cpu().numpy()) <= 2e-2
+
+
+def _sampled_heads(x: I.FwdInputs, pairs, what):
+    """Run the GPU on the whole workload; check the listed (b, h) against the oracle."""
+    o, S_T, _ = run_gpu(x)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S_T).all()
+    n = x.as_numpy64()
+    errs = []
+    for (b, h) in pairs:
+        args = [head_slice(n[f], b, h) for f in ("q", "k", "v", "log_alpha", "b", "w")]
+        o_ref, S_ref = oracle.forward(*args, S0=head_slice(n["S0"], b, h, token_major=False))
+        errs.append(assert_close(o[b:b + 1, :, h:h + 1], o_ref, TOL[x.q.dtype], f"{what} o[b={b},h={h}]"))
+        errs.append(assert_close(S_T[b:b + 1, h:h + 1], S_ref, TOL[x.q.dtype], f"{what} S_T[b={b},h={h}]"))
+    return max(errs)
+
+
+@pytest.mark.slow
+def test_full_size_1p3b_layer_sampled_heads():
+    """B=4 H=16 T=4096 d=128 bf16, the benchmarked launch; oracle on sampled heads."""
+    x = I.make_forward_inputs(**I.FWD_1P3B_BF16)
+    _sampled_heads(x, [(0, 0), (1, 7), (3, 15)], "1.3B layer")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", I.SWEEP_T)
+def test_sequence_sweep_sampled_heads(T):
+    """65,536 tokens per call at T in {2K..32K}; oracle on two heads of the last sequence."""
+    x = I.make_forward_inputs(**I.sweep_config(T))
+    B = x.q.shape[0]
+    _sampled_heads(x, [(B - 1, 0), (0, 9)], f"sweep T={T}")
