@@ -60,7 +60,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_backward_workspace_bytes.restype = Z
         lib.gdr2_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.gdr2_backward.restype = I
-        lib.gdr2_backward.argtypes = [I, I, I, I, I, I] + [P] * 17 + [Z, P]
+        lib.gdr2_backward.argtypes = [I, I, I, I, I, I] + [P] * 18 + [Z, P]
         lib.gdr2_sync_status.restype = I
         lib.gdr2_sync_status.argtypes = [P]
         _lib = lib

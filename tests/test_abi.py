@@ -82,7 +82,7 @@ def test_backward_workspace_query_and_checks(lib):
     BH, NC, SS = 32, 64, 128 * 128 * 4
     assert n >= BH * NC * SS + BH * 65 * SS
     assert n % 256 == 0
-    p = [ctypes.c_void_p(0x10000)] * 17
+    p = [ctypes.c_void_p(0x10000)] * 18  # 17 tensors + the workspace
     st = lib.gdr2_backward(2, 64, 16, 128, 128, 1, *p, ctypes.c_size_t(16), ctypes.c_void_p(0))
     assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
     assert lib.gdr2_backward_workspace_bytes(-1, 1, 1, 64, 64, 1) == 0
