@@ -6,8 +6,10 @@ tensors. ``inputs`` draws the seeded synthetic workloads. Importing the
 package does not load the CUDA library; the first call does, and fails loudly
 if it is missing.
 """
-from .binding import (GDR2Error, gdr2_abi_version, gdr2_backward, gdr2_backward_workspace_bytes,  # noqa: F401
-                      gdr2_decode_step, gdr2_forward, gdr2_last_error, gdr2_sync_status, load_library)
+from .binding import (GDR2Error, gdr2_abi_version, gdr2_backward, gdr2_backward_noalloc,  # noqa: F401
+                      gdr2_backward_workspace_bytes, gdr2_decode_step, gdr2_forward, gdr2_last_error,
+                      gdr2_sync_status, load_library)
 
-__all__ = ["GDR2Error", "gdr2_abi_version", "gdr2_backward", "gdr2_backward_workspace_bytes",
+__all__ = ["GDR2Error", "gdr2_abi_version", "gdr2_backward", "gdr2_backward_noalloc",
+           "gdr2_backward_workspace_bytes",
            "gdr2_decode_step", "gdr2_forward", "gdr2_last_error", "gdr2_sync_status", "load_library"]

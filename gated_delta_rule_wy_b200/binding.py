@@ -24,7 +24,9 @@ _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIM
 
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
 EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward", "gdr2_decode_step",
-                    "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_sync_status")
+                    "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
+                    "gdr2_sync_status")
+NOALLOC_SCRATCH_BYTES = 64 << 20  # GDR2_NOALLOC_SCRATCH_BYTES
 
 
 class GDR2Error(RuntimeError):
@@ -61,6 +63,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.gdr2_backward.restype = I
         lib.gdr2_backward.argtypes = [I, I, I, I, I, I] + [P] * 18 + [Z, P]
+        lib.gdr2_backward_noalloc.restype = I
+        lib.gdr2_backward_noalloc.argtypes = [I, I, I, I, I, I] + [P] * 18
         lib.gdr2_sync_status.restype = I
         lib.gdr2_sync_status.argtypes = [P]
         _lib = lib
@@ -194,5 +198,37 @@ def gdr2_backward(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, saved_states
                            _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(saved_states), _ptr(g["dq"]),
                            _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["db"]), _ptr(g["dw"]),
                            _ptr(g["dS0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _raise(lib, st)
+    return g
+
+
+def gdr2_backward_noalloc(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, saved_states=None, *,
+                          want_dS0=True, stream=None):
+    """gdr2_backward through the entry point that allocates nothing on the device.
+
+    The library uses its own fixed scratch array (NOALLOC_SCRATCH_BYTES per
+    device) instead of a workspace; the gradient tensors returned here are
+    ordinary torch allocations made by this binding, not by the library.
+    """
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("b", b, (B, T, H, dk)),
+                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H, dv)), ("dO", dO, (B, T, H, dv))):
+        _check(t, name, shp, dt)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32)
+    _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    _check(dS_T, "dS_T", (B, H, dk, dv), torch.float32)
+    nc = (T + CHUNK - 1) // CHUNK
+    _check(saved_states, "saved_states", (B, H, nc, dk, dv), torch.float32)
+    dev = q.device
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+         "dlog_alpha": torch.empty_like(log_alpha), "db": torch.empty_like(b), "dw": torch.empty_like(w),
+         "dS0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dS0 else None}
+    st = lib.gdr2_backward_noalloc(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                   _ptr(b), _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(saved_states),
+                                   _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
+                                   _ptr(g["db"]), _ptr(g["dw"]), _ptr(g["dS0"]), _stream(stream))
     _raise(lib, st)
     return g

@@ -22,6 +22,9 @@
 // reductions (over key channels) use a shuffle transpose-reduce inside a
 // warp, then shared memory across warps.
 
+#include <mutex>
+
+#include "../../include/gdr2.h"
 #include "gdr2_common.cuh"
 #include "gdr2_launch.h"
 
@@ -282,6 +285,51 @@ cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s)
 {
     if (a.B * a.H == 0) return cudaSuccess;
     return a.bf16 ? launch_dt<__nv_bfloat16>(a, s) : launch_dt<float>(a, s);
+}
+
+}  // namespace gdr2
+
+// ---------------------------------------------------------------------------
+// Variant for callers that may not allocate device memory: the workspace is a
+// file-scope device array of GDR2_NOALLOC_SCRATCH_BYTES. Host code must not
+// use the array's name as a device address (it is a host-side stand-in): the
+// address is looked up once per device with cudaGetSymbolAddress, with that
+// device current, and passed to the same kernel. The kernel writes every
+// scratch word before reading it, so stale contents from the previous call
+// do no harm; concurrent calls on one device share the array and race.
+namespace gdr2 {
+namespace {
+
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[GDR2_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxNoAllocDevices = 64;
+void *g_noalloc_ptr[kMaxNoAllocDevices];
+cudaError_t g_noalloc_err[kMaxNoAllocDevices];
+std::once_flag g_noalloc_once[kMaxNoAllocDevices];
+
+}  // namespace
+
+size_t backward_noalloc_scratch_needed(int B, int T, int H, int dk, int dv, bool have_saved_states)
+{
+    return bwd_layout(B, T, H, dk, dv, !have_saved_states).total;
+}
+
+cudaError_t launch_backward_noalloc(const BwdArgs &a_in, cudaStream_t s)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxNoAllocDevices) return cudaErrorInvalidDevice;
+    std::call_once(g_noalloc_once[dev], [dev] {
+        void *ptr = nullptr;
+        g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch);
+        g_noalloc_ptr[dev] = ptr;
+    });
+    if (g_noalloc_err[dev] != cudaSuccess) return g_noalloc_err[dev];
+    BwdArgs a = a_in;
+    a.workspace = g_noalloc_ptr[dev];
+    a.workspace_bytes = GDR2_NOALLOC_SCRATCH_BYTES;
+    return launch_backward(a, s);
 }
 
 }  // namespace gdr2

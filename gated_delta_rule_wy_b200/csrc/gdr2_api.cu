@@ -200,6 +200,45 @@ gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, co
     return launched(gdr2::launch_backward(a, s), "gdr2_backward");
 }
 
+gdr2_status gdr2_backward_noalloc(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                                  const void *v, const float *log_alpha, const void *b, const void *w,
+                                  const float *S0, const void *dO, const float *dS_T, const float *saved_states,
+                                  void *dq, void *dk_, void *dv_, float *dlog_alpha, void *db, void *dw, float *dS0,
+                                  void *stream)
+{
+    GDR2_TRY(check_dims(B, T, H, dk, dv));
+    GDR2_TRY(check_dtype(dt));
+    const bool has_tokens = (long long)B * T * H > 0;
+    const char *names[] = {"q", "k", "v", "log_alpha", "b", "w", "dO", "dq", "dk", "dv", "dlog_alpha", "db", "dw"};
+    const void *ptrs[] = {q, k, v, log_alpha, b, w, dO, dq, dk_, dv_, dlog_alpha, db, dw};
+    for (int i = 0; i < 13; ++i) GDR2_TRY(check_ptr(ptrs[i], names[i], !has_tokens));
+    GDR2_TRY(check_ptr(S0, "S0", true));
+    GDR2_TRY(check_ptr(dS_T, "dS_T", true));
+    GDR2_TRY(check_ptr(saved_states, "saved_states", true));
+    GDR2_TRY(check_ptr(dS0, "dS0", true));
+    if ((long long)B * H == 0) return GDR2_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (dS0) {
+            const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+            cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, bytes, cudaMemcpyDeviceToDevice, s)
+                                 : cudaMemsetAsync(dS0, 0, bytes, s);
+            return launched(e, "gdr2_backward_noalloc (T = 0)");
+        }
+        return GDR2_OK;
+    }
+    const size_t need = gdr2::backward_noalloc_scratch_needed(B, T, H, dk, dv, saved_states != nullptr);
+    if (need > GDR2_NOALLOC_SCRATCH_BYTES)
+        return fail(GDR2_ERR_UNSUPPORTED,
+                    "gdr2_backward_noalloc: this problem needs %zu bytes of scratch but the built-in array holds "
+                    "%zu (GDR2_NOALLOC_SCRATCH_BYTES); pass saved_states, split the batch, or use gdr2_backward",
+                    need, (size_t)GDR2_NOALLOC_SCRATCH_BYTES);
+    gdr2::BwdArgs a{B, T, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S0, dO, dS_T, saved_states,
+                    dq, dk_, dv_, dlog_alpha, db, dw, dS0, nullptr, 0, nullptr};
+    GDR2_TRY(device_status(&a.status));
+    return launched(gdr2::launch_backward_noalloc(a, s), "gdr2_backward_noalloc");
+}
+
 gdr2_status gdr2_sync_status(void *stream)
 {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -56,5 +56,7 @@ bool forward_tc_supported(const FwdArgs &a);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf16);
 cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s);
+size_t backward_noalloc_scratch_needed(int B, int T, int H, int dk, int dv, bool have_saved_states);
+cudaError_t launch_backward_noalloc(const BwdArgs &a, cudaStream_t s);
 
 }  // namespace gdr2

@@ -22,7 +22,9 @@
  *             the current device, contiguous in the layouts below, 16-byte
  *             aligned. The caller owns every buffer; the library allocates no
  *             device memory. Scratch, where an entry point needs any, is a
- *             caller buffer sized by the matching *_workspace_bytes query.
+ *             caller buffer sized by the matching *_workspace_bytes query
+ *             (gdr2_backward_noalloc instead uses a fixed array inside the
+ *             library; see there).
  * Layouts:    token tensors are token-major:
  *               q, k, log_alpha, b          [B, T, H, dk]
  *               v, w, o                     [B, T, H, dv]
@@ -142,6 +144,41 @@ gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
                           void *dq, void *dk_, void *dv_, float *dlog_alpha,
                           void *db, void *dw, float *dS0,
                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Size of the device scratch array behind gdr2_backward_noalloc (64 MiB). */
+#define GDR2_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * gdr2_backward_noalloc -- gdr2_backward without a caller workspace and
+ * without any device allocation. The paper has no counterpart: this is a
+ * deployment variant for callers that may not allocate device memory, such as
+ * a serving engine that reserves nearly all of HBM for its own pool at start-up
+ * (a fresh cudaMalloc would fail or fragment that pool, and cudaFree
+ * synchronises the device), or a host component that only receives device
+ * pointers from another runtime and has no allocator of its own.
+ * Scratch: a file-scope device array of GDR2_NOALLOC_SCRATCH_BYTES inside the
+ *      library. Every GPU on which the library's backward module is loaded
+ *      holds one such array until the process exits. The first call on a
+ *      device looks up the array's device address (once per device, with that
+ *      device current); make that first call before any stream capture.
+ * Sharing: all calls on a device share the one array and it keeps the last
+ *      call's contents (nothing in it needs to start at zero). Calls that
+ *      overlap on the GPU -- on different streams, or from different host
+ *      threads -- race on it; serialise them.
+ * Limit: a problem whose scratch (gdr2_backward's workspace minus the chunk
+ *      states when saved_states is given) exceeds GDR2_NOALLOC_SCRATCH_BYTES
+ *      returns GDR2_ERR_UNSUPPORTED before any work is enqueued. At
+ *      dk = dv = 128 with saved_states that is about 4.2 MiB per (batch, head).
+ * Arguments, layouts and results are those of gdr2_backward. The call itself
+ * makes no cudaMalloc, cudaFree or other allocating call.
+ */
+gdr2_status gdr2_backward_noalloc(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
+                                  const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const void *b, const void *w,
+                                  const float *S0, const void *dO, const float *dS_T,
+                                  const float *saved_states,
+                                  void *dq, void *dk_, void *dv_, float *dlog_alpha,
+                                  void *db, void *dw, float *dS0, void *stream);
 
 /*
  * gdr2_sync_status -- wait for `stream`, then report and clear the device

@@ -94,3 +94,12 @@ def test_binding_validates_before_calling():
     q = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         g.gdr2_forward(q, q, q, q, q, q)
+
+
+def test_noalloc_backward_rejects_oversized_problems_on_the_host(lib):
+    """Too large for the built-in scratch array: UNSUPPORTED, nothing launched."""
+    p = [ctypes.c_void_p(0x10000)] * 17 + [None]
+    # 64 heads of d = 128 with saved states need ~270 MiB of scratch (> 64 MiB)
+    st = lib.gdr2_backward_noalloc(4, 4096, 16, 128, 128, 1, *p)
+    assert st == binding.GDR2_ERR_UNSUPPORTED
+    assert b"GDR2_NOALLOC_SCRATCH_BYTES" in lib.gdr2_last_error()
