@@ -1,11 +1,716 @@
-// fwd_tc.cu -- tcgen05/TMEM chunkwise forward for bf16 inputs (sm_100a).
+// fwd_tc.cu -- chunkwise GDR-2 forward on the sm_100a tensor cores (bf16
+// inputs, fp32 state), dk = dv = 128.
+//
+// Algorithm: the chunkwise WY form of the Gated DeltaNet-2 note, sec. 3
+// (chunkwise training paragraph): within a chunk of C = 64 tokens the decay
+// is absorbed into the gated keys (decay-normalised state S_r =
+// Diag(gamma_r) S^_r), which leaves an asymmetric delta recurrence whose
+// token products collapse into a unit-lower-triangular solve (UT form) and a
+// chain of matmuls; the state crosses chunk boundaries in fp32.
+//
+//   A_ti = sum_c e_t[c] k_i[c] exp(G_t[c] - G_i[c])   i < t      (e = b (.) k)
+//   P_ti = sum_c q_t[c] k_i[c] exp(G_t[c] - G_i[c])   i <= t
+//   T = (I + A)^{-1};  W = T (E (.) exp G);  U = T Z - W S      (z = w (.) v)
+//   O = (Q (.) exp G) S + P U
+//   S <- Diag(exp G_C) S + (K (.) exp(G_C - G))^T U
+//
+// Decay range. exp(G_t - G_i) is formed as a product of two factors around a
+// per-channel reference g_I, the cumulative decay at the midpoint of the
+// 32-token half-chunk I that holds t:
+//   L_t = x_t exp(G_t - g_I),   R_i = k_i exp(g_I - G_i).
+// Each factor stays within exp(+-80) unless a half-chunk's decay spans more
+// than 160 nepers; a factor that underflows only loses terms whose true value
+// is itself below fp32 range. When the guard trips (alpha near 0 over a whole
+// half-chunk, e.g. a reset) the chunk takes an exact path: A and P with one
+// exponential per (t, i, c), and the decay-weighted operands from exp(G)
+// directly. Every other chunk keeps the factorised, tensor-core path.
+//
+// Mapping to tcgen05 (M = 128 everywhere; T = token, c = key channel,
+// j = value channel; every accumulator is fp32 in TMEM):
+//   [A;P] : D(128 x 32|64) = [L^e_0; L^q_0; L^e_1; L^q_1] R_I^T   (K = c)
+//   W^T_I : D(c x t) = (L^e_I)^T T[:, I]^T,  W = sum_I exp(g_I) W_I (K = s in I)
+//   U^T   : D(j x t) = Z^T T^T - S^T W^T        (A negated in the second MMA)
+//   O^T   : D(j x t) = S^T Q^T + U^T P^T
+//   S     : D(c x j) = Diag(exp G_C) S + K~^T U (row scale applied in TMEM)
+// Operands are staged by TMA (no multicast) and written by the threads into
+// 128-byte-swizzled UMMA layouts; one thread issues every MMA and commit.
+//
+// Threads: 128, thread i <-> TMEM lane i. One CTA per (batch, head); the
+// chunk loop is sequential. Every mbarrier wait is bounded; on a timeout the
+// CTA records kStatusTimeout, frees its TMEM and exits.
+
+#include <cuda.h>
+#include <mutex>
+
 #include "gdr2_common.cuh"
 #include "gdr2_launch.h"
+#include "sm100_ptx.cuh"
 
 namespace gdr2 {
+namespace {
 
-bool forward_tc_supported(const FwdArgs &) { return false; }
+using namespace sm100;
 
-cudaError_t launch_forward_tc(const FwdArgs &, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int C = 64;
+constexpr int DK = 128;
+constexpr int DV = 128;
+constexpr int NT = 128;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr float kFactorLimit = 80.f;              // |exponent| of one decay factor
+
+// ---- shared-memory map (bytes from a 1024-aligned base) ----
+constexpr uint32_t OFF_STG_Q = 0;            // q  [64][128] bf16; later T (bf16, swizzled)
+constexpr uint32_t OFF_STG_K = 16384;        // k
+constexpr uint32_t OFF_STG_B = 32768;        // b
+constexpr uint32_t OFF_STG_V = 49152;        // v; later A (fp32 [64][68]) over V and W
+constexpr uint32_t OFF_STG_W = 65536;        // w
+constexpr uint32_t OFF_STG_LA = 81920;       // log_alpha [64][128] fp32; exact path: G
+constexpr uint32_t OFF_STACK = 114688;       // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128; later S^T
+constexpr uint32_t OFF_R0 = 147456;          // R_0 32 x 128
+constexpr uint32_t OFF_R1 = 155648;          // R_1 64 x 128; U (128 x 64) over R0..R1
+constexpr uint32_t OFF_Z = 172032;           // Z 64 x 128 (value side); later W^T
+constexpr uint32_t OFF_QH = 188416;          // Q (.) exp G, 64 x 128
+constexpr uint32_t OFF_KT = 204800;          // K (.) exp(G_C - G), 64 x 128
+constexpr uint32_t OFF_P = 221184;           // P 64 x 64
+constexpr uint32_t OFF_MISC = 229376;        // barriers, per-channel vectors
+constexpr uint32_t MISC_BYTES = 1664;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+constexpr int A_LD = 68;                     // fp32 row stride of the A scratch
+constexpr uint32_t TX_BYTES = 5 * 16384 + 32768;
+
+// TMEM columns
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_W0 = 256, TM_W1 = 320, TM_AP0 = 384, TM_AP1 = 416;
+constexpr uint32_t TM_COLS = 512;
+
+struct Misc {
+    uint64_t bar_tma;
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int flag;
+    int abort;
+    int pad;
+    float gC[DK];    // exp(G_C)
+    float eg0[DK];   // W combine factor of half-chunk 0
+    float eg1[DK];   // ... of half-chunk 1
+};
+static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
+
+// Byte offset of element (row, col) in a 128-byte-swizzled tile whose rows
+// are 64 bf16 wide; tiles of 128 columns are two such blocks of `rows` rows.
+__device__ __forceinline__ uint32_t sw_off(int row, int col, int rows)
+{
+    const int blk = col >> 6, cc = col & 63;
+    return (uint32_t)(blk * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + ((cc & 7) << 1));
+}
+
+// Offset of the 16-byte chunk holding columns [8*o8, 8*o8 + 8) of `row`.
+__device__ __forceinline__ uint32_t sw_chunk(int row, int o8, int rows)
+{
+    const int blk = o8 >> 3, ch = o8 & 7;
+    return (uint32_t)(blk * rows * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8])
+{
+    uint4 u;
+    __nv_bfloat162 h;
+    h = __floats2bfloat162_rn(f[0], f[1]); u.x = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(f[2], f[3]); u.y = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(f[4], f[5]); u.z = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(f[6], f[7]); u.w = *reinterpret_cast<uint32_t *>(&h);
+    return u;
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float (&f)[8])
+{
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+struct TcParams {
+    int B, T, H;
+    const float *S0;
+    __nv_bfloat16 *o;
+    float *S_T;
+    float *saved_states;
+    unsigned *status;
+};
+
+__global__ void __launch_bounds__(NT, 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la, TcParams p)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Misc &ms = *reinterpret_cast<Misc *>(sm + OFF_MISC);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.x;
+    const int bb = bh / p.H, h = bh % p.H;
+    const int T = p.T, H = p.H;
+    const int NC = (T + C - 1) / C;
+
+    if (tid == 0) {
+        mbar_init(&ms.bar_tma, 1);
+        mbar_init(&ms.bar_mma, 1);
+        fence_mbar_init();
+        ms.abort = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(&ms.tmem_base, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tm = ms.tmem_base;
+    const uint32_t tm_lane = tm + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+
+    auto issue_loads = [&](int n) {
+        const int row = bb * T + n * C;
+        mbar_arrive_expect_tx(&ms.bar_tma, TX_BYTES);
+        tma_load_3d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, h, row);
+        tma_load_3d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, h, row);
+        tma_load_3d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, h, row);
+        tma_load_3d(sm + OFF_STG_V, &tm_v, &ms.bar_tma, 0, h, row);
+        tma_load_3d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, h, row);
+        tma_load_3d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, h, row);
+    };
+    if (tid == 0 && NC > 0) issue_loads(0);
+
+    // ---- initial state into TMEM (thread c owns row c) ----
+    {
+        const int c = tid;
+        float v[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = p.S0 ? p.S0[((size_t)bh * DK + c) * DV + q4 * 32 + i] : 0.f;
+            tmem_st32(tm_lane + TM_S + q4 * 32, v);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+
+    uint32_t ph_tma = 0, ph_mma = 0;
+    bool timed_out = false;
+    // every thread waits; any timeout aborts the CTA consistently
+    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
+        const bool ok = mbar_wait_bounded(bar, ph, kWaitLimitNs);
+        ph ^= 1u;
+        return __syncthreads_or(!ok) == 0;
+    };
+    auto mma_sync_point = [&]() {  // operands written by threads -> visible to the tensor core
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
+    };
+
+    // prep mapping: channel octet o8 (channels 8*o8 .. +7), token group tg (tokens 8*tg .. +7)
+    const int o8 = warp * 4 + (lane >> 3);
+    const int tg = lane & 7;
+    const int HI = tg >> 2;  // half-chunk of this thread's tokens
+
+    for (int n = 0; n < NC && !timed_out; ++n) {
+        const int t0 = n * C;
+        const int Cn = min(C, T - t0);
+        if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
+
+        // ================= prep: cumulative decay and decay-weighted operands =================
+        float G[8][8];  // G[token m][channel x], cumulative within the chunk
+        {
+            const float *la_s = reinterpret_cast<const float *>(sm + OFF_STG_LA);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int t = tg * 8 + m;
+                const float4 a0 = *reinterpret_cast<const float4 *>(la_s + t * DK + o8 * 8);
+                const float4 a1 = *reinterpret_cast<const float4 *>(la_s + t * DK + o8 * 8 + 4);
+                const float la[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float l = (t < Cn) ? clamp_log_alpha(la[x]) : 0.f;
+                    G[m][x] = (m == 0 ? 0.f : G[m - 1][x]) + l;
+                }
+            }
+            // exclusive prefix over the 8 token groups (8 consecutive lanes)
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const float tot = G[7][x];
+                float inc = tot;
+#pragma unroll
+                for (int d = 1; d < 8; d <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, inc, d, 8);
+                    if (tg >= d) inc += y;
+                }
+                const float ex = inc - tot;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) G[m][x] += ex;
+            }
+        }
+        float g0[8], g1[8], gC[8];
+        const int grp = lane & ~7;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            g0[x] = __shfl_sync(0xffffffffu, G[7][x], grp | 1);  // token 15
+            g1[x] = __shfl_sync(0xffffffffu, G[7][x], grp | 5);  // token 47
+            gC[x] = __shfl_sync(0xffffffffu, G[7][x], grp | 7);  // token 63
+        }
+        bool risky = false;
+        {
+            const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_Q);
+            const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
+            const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
+            const __nv_bfloat16 *vs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_V);
+            const __nv_bfloat16 *ws = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_W);
+            float egI[8], kcf[8], r10[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const float gr = HI ? g1[x] : g0[x];
+                egI[x] = __expf(gr);           // exp(g_I)
+                kcf[x] = __expf(gC[x] - gr);   // exp(G_C - g_I)
+                r10[x] = __expf(g1[x] - g0[x]);
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int t = tg * 8 + m;
+                float qv[8], kv[8], bv[8], vv[8], wv[8];
+                unpack8(*reinterpret_cast<const uint4 *>(qs + t * DK + o8 * 8), qv);
+                unpack8(*reinterpret_cast<const uint4 *>(ks + t * DK + o8 * 8), kv);
+                unpack8(*reinterpret_cast<const uint4 *>(bs + t * DK + o8 * 8), bv);
+                unpack8(*reinterpret_cast<const uint4 *>(vs + t * DV + o8 * 8), vv);
+                unpack8(*reinterpret_cast<const uint4 *>(ws + t * DV + o8 * 8), wv);
+                const bool live = t < Cn;
+                float le[8], lq[8], r[8], kt[8], qh[8], z[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float gr = HI ? g1[x] : g0[x];
+                    const float d = G[m][x] - gr;
+                    risky |= fabsf(d) > kFactorLimit;
+                    const float xl = __expf(d), yr = __expf(-d);
+                    const float kk = live ? kv[x] : 0.f;
+                    const float qq = live ? qv[x] : 0.f;
+                    const float ee = live ? bv[x] * kv[x] : 0.f;
+                    le[x] = ee * xl;
+                    lq[x] = qq * xl;
+                    r[x] = kk * yr;
+                    kt[x] = r[x] * kcf[x];
+                    qh[x] = lq[x] * egI[x];
+                    z[x] = live ? wv[x] * vv[x] : 0.f;
+                }
+                const int tl = t - 32 * HI;  // token within its half-chunk
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + 32 + tl, o8, 128)) = pack8(lq);
+                if (HI == 0) {
+                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(t, o8, 32)) = pack8(r);
+                    float r1[8];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) r1[x] = r[x] * r10[x];
+                    *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(t, o8, 64)) = pack8(r1);
+                } else {
+                    *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(t, o8, 64)) = pack8(r);
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
+                *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
+                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
+            }
+            if (tg == 0) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    ms.gC[o8 * 8 + x] = __expf(gC[x]);
+                    ms.eg0[o8 * 8 + x] = __expf(g0[x]);
+                    ms.eg1[o8 * 8 + x] = __expf(g1[x]);
+                }
+            }
+        }
+        const bool exact = __syncthreads_or(risky) != 0;
+        float *A32 = reinterpret_cast<float *>(sm + OFF_STG_V);
+        if (exact) {
+            // ---- exact path: G to shared memory, pairwise exponentials ----
+            float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) Gs[(tg * 8 + m) * DK + o8 * 8 + x] = G[m][x];
+            __syncthreads();
+            const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_Q);
+            const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
+            const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
+            // operands with one exponential of a non-positive argument each
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int t = tg * 8 + m;
+                const bool live = t < Cn;
+                float qv[8], kv[8], bv[8], le[8], kt[8], qh[8];
+                unpack8(*reinterpret_cast<const uint4 *>(qs + t * DK + o8 * 8), qv);
+                unpack8(*reinterpret_cast<const uint4 *>(ks + t * DK + o8 * 8), kv);
+                unpack8(*reinterpret_cast<const uint4 *>(bs + t * DK + o8 * 8), bv);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float eg = __expf(G[m][x]);
+                    le[x] = live ? bv[x] * kv[x] * eg : 0.f;
+                    qh[x] = live ? qv[x] * eg : 0.f;
+                    kt[x] = live ? kv[x] * __expf(gC[x] - G[m][x]) : 0.f;
+                }
+                const int tl = t - 32 * HI;
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
+                *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
+                *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
+            }
+            if (tg == 0) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) ms.eg0[o8 * 8 + x] = ms.eg1[o8 * 8 + x] = 1.f;
+            }
+            // A and P rows: thread -> row t = tid / 2, columns half*32 .. +31
+            {
+                const int t = tid >> 1, i0 = (tid & 1) * 32;
+                float accA[32], accP[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) accA[u] = accP[u] = 0.f;
+                if (i0 <= t && t < Cn) {
+                    for (int c = 0; c < DK; ++c) {
+                        const float gt = Gs[t * DK + c];
+                        const float kt_ = __bfloat162float(ks[t * DK + c]);
+                        const float et = __bfloat162float(bs[t * DK + c]) * kt_;
+                        const float qt = __bfloat162float(qs[t * DK + c]);
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const int i = i0 + u;
+                            if (i <= t) {
+                                const float f = __bfloat162float(ks[i * DK + c]) * __expf(gt - Gs[i * DK + c]);
+                                accA[u] = fmaf(et, f, accA[u]);
+                                accP[u] = fmaf(qt, f, accP[u]);
+                            }
+                        }
+                    }
+                }
+                float pr[8];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int i = i0 + u;
+                    A32[t * A_LD + i] = (i < t) ? accA[u] : 0.f;
+                }
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) {
+                        const int i = i0 + k8 * 8 + x;
+                        pr[x] = (i <= t) ? accP[k8 * 8 + x] : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, (i0 >> 3) + k8, 64)) = pack8(pr);
+                }
+            }
+            __syncthreads();
+        } else {
+            // ---- tensor-core path: [A;P] = STACK R_I^T ----
+            mma_sync_point();
+            if (tid == 0) {
+                const uint32_t id0 = idesc_bf16(128, 32, false, false);
+                const uint32_t id1 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks & 3) * 32;
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + (ks >> 2) * 16384 + koff, 16, 1024);
+                    const uint64_t b0 = sdesc_sw128(sbase + OFF_R0 + (ks >> 2) * 4096 + koff, 16, 1024);
+                    const uint64_t b1 = sdesc_sw128(sbase + OFF_R1 + (ks >> 2) * 8192 + koff, 16, 1024);
+                    mma_bf16(tm + TM_AP0, ad, b0, id0, ks > 0);
+                    mma_bf16(tm + TM_AP1, ad, b1, id1, ks > 0);
+                }
+                mma_commit(&ms.bar_mma);
+            }
+            if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
+            tc_fence_after_sync();
+            // rows: warp 0 -> A rows 0..31, warp 1 -> P rows 0..31 (32 cols of AP0),
+            //       warp 2 -> A rows 32..63, warp 3 -> P rows 32..63 (64 cols of AP1)
+            const bool isP = (warp & 1) != 0;
+            const int t = (warp >= 2 ? 32 : 0) + lane;
+            const int ncol = warp >= 2 ? 64 : 32;
+            float row[64];
+            {
+                float v[32];
+                tmem_ld32(tm_lane + (warp >= 2 ? TM_AP1 : TM_AP0), v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) row[i] = v[i];
+                if (warp >= 2) {
+                    tmem_ld32(tm_lane + TM_AP1 + 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) row[32 + i] = v[i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) row[32 + i] = 0.f;
+                }
+            }
+            (void)ncol;
+            if (!isP) {
+#pragma unroll
+                for (int i = 0; i < 64; i += 4) {
+                    float4 a;
+                    a.x = (i + 0 < t) ? row[i + 0] : 0.f;
+                    a.y = (i + 1 < t) ? row[i + 1] : 0.f;
+                    a.z = (i + 2 < t) ? row[i + 2] : 0.f;
+                    a.w = (i + 3 < t) ? row[i + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(A32 + t * A_LD + i) = a;
+                }
+            } else {
+#pragma unroll
+                for (int k8 = 0; k8 < 8; ++k8) {
+                    float pr[8];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) pr[x] = (k8 * 8 + x <= t) ? row[k8 * 8 + x] : 0.f;
+                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = pack8(pr);
+                }
+            }
+            tc_fence_before_sync();
+            __syncthreads();
+        }
+
+        // ================= UT solve: T = (I + A)^{-1}, column s by two threads =================
+        {
+            const int s = tid >> 1, par = tid & 1;
+            float half[32];  // T[2m + par][s]
+#pragma unroll
+            for (int m = 0; m < 32; ++m) half[m] = 0.f;
+#pragma unroll
+            for (int t = 0; t < C; ++t) {
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                for (int m = 0; 2 * m < t; ++m) {
+                    const int i = 2 * m + par;
+                    const float av = (i < t) ? A32[t * A_LD + i] : 0.f;
+                    if ((m & 3) == 0) a0 = fmaf(av, half[m], a0);
+                    else if ((m & 3) == 1) a1 = fmaf(av, half[m], a1);
+                    else if ((m & 3) == 2) a2 = fmaf(av, half[m], a2);
+                    else a3 = fmaf(av, half[m], a3);
+                }
+                float acc = (a0 + a1) + (a2 + a3);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                const float val = (t < s) ? 0.f : (t == s ? 1.f : -acc);
+                if ((t & 1) == par) half[t >> 1] = val;
+            }
+            // T -> bf16, K-major [t][s] (64 wide), over the q staging buffer
+            __nv_bfloat16 *Tb = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_STG_Q);
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const int t = 2 * m + par;
+                *reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<unsigned char *>(Tb) + sw_off(t, s, 64)) =
+                    __float2bfloat16_rn(half[m]);
+            }
+        }
+        mma_sync_point();
+        // ================= W^T_I = (L^e_I)^T T[:,I]^T ;  U^T = Z^T T^T =================
+        if (tid == 0) {
+            const uint32_t idW = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int I = 0; I < 2; ++I)
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + (64 * I + 16 * ks) * 128, 16384, 1024);
+                    const uint64_t bd = sdesc_sw128(sbase + OFF_STG_Q + (32 * I + 16 * ks) * 2, 16, 1024);
+                    mma_bf16(tm + (I ? TM_W1 : TM_W0), ad, bd, idW, ks > 0);
+                }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = sdesc_sw128(sbase + OFF_Z + ks * 2048, 8192, 1024);
+                const uint64_t bd = sdesc_sw128(sbase + OFF_STG_Q + ks * 32, 16, 1024);
+                mma_bf16(tm + TM_U, ad, bd, idW, ks > 0);
+            }
+            mma_commit(&ms.bar_mma);
+        }
+        if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
+        tc_fence_after_sync();
+        // staging is free: prefetch the next chunk's inputs
+        if (tid == 0 && n + 1 < NC) issue_loads(n + 1);
+
+        // ================= W epilogue, S copy and state decay =================
+        {
+            const int c = tid;
+            const float e0 = ms.eg0[c], e1 = ms.eg1[c];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float w0[32], w1[32];
+                tmem_ld32(tm_lane + TM_W0 + hf * 32, w0);
+                tmem_ld32(tm_lane + TM_W1 + hf * 32, w1);
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    float f[8];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) f[x] = e0 * w0[k8 * 8 + x] + e1 * w1[k8 * 8 + x];
+                    // W^T stored MN-major: row c, 64 t-columns
+                    *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, hf * 4 + k8, 128)) = pack8(f);
+                }
+            }
+            const float gc = ms.gC[c];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float sv[32];
+                tmem_ld32(tm_lane + TM_S + q4 * 32, sv);
+                if (p.saved_states) {
+                    float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c) * DV + q4 * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(dst + i) = make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3]);
+                }
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    float f[8];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) f[x] = sv[k8 * 8 + x];
+                    // S^T stored MN-major (j contiguous): [j-block][c rows][64 j]
+                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(c, q4 * 4 + k8, 128)) = pack8(f);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] *= gc;
+                tmem_st32(tm_lane + TM_S + q4 * 32, sv);
+            }
+        }
+        mma_sync_point();
+        // ================= U^T -= S^T W^T ;  O^T = S^T Q^T =================
+        if (tid == 0) {
+            const uint32_t idU = idesc_bf16(128, 64, true, true, true);
+            const uint32_t idO = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + ks * 2048, 16384, 1024);
+                const uint64_t bw = sdesc_sw128(sbase + OFF_Z + ks * 2048, 8192, 1024);
+                const uint64_t bq = sdesc_sw128(sbase + OFF_QH + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                mma_bf16(tm + TM_U, ad, bw, idU, 1);
+                mma_bf16(tm + TM_O, ad, bq, idO, ks > 0);
+            }
+            mma_commit(&ms.bar_mma);
+        }
+        if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
+        tc_fence_after_sync();
+        // ================= U epilogue: U^T rows -> bf16 [j][64 t] =================
+        {
+            const int j = tid;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float u[32];
+                tmem_ld32(tm_lane + TM_U + hf * 32, u);
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    float f[8];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
+                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(j, hf * 4 + k8, 128)) = pack8(f);
+                }
+            }
+        }
+        mma_sync_point();
+        // ================= O^T += U^T P^T ;  S += K~^T U =================
+        if (tid == 0) {
+            const uint32_t idO = idesc_bf16(128, 64, false, false);
+            const uint32_t idS = idesc_bf16(128, 128, true, false);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t au = sdesc_sw128(sbase + OFF_R0 + ks * 32, 16, 1024);
+                const uint64_t bp = sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024);
+                mma_bf16(tm + TM_O, au, bp, idO, 1);
+                const uint64_t ak = sdesc_sw128(sbase + OFF_KT + ks * 2048, 8192, 1024);
+                mma_bf16(tm + TM_S, ak, au, idS, 1);
+            }
+            mma_commit(&ms.bar_mma);
+        }
+        if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
+        tc_fence_after_sync();
+        // ================= O epilogue =================
+        {
+            const int j = tid;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float ov[32];
+                tmem_ld32(tm_lane + TM_O + hf * 32, ov);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int t = hf * 32 + i;
+                    if (t < Cn) p.o[(((size_t)bb * T + t0 + t) * H + h) * DV + j] = __float2bfloat16_rn(ov[i]);
+                }
+            }
+        }
+        tc_fence_before_sync();
+        __syncthreads();
+    }
+
+    if (!timed_out && p.S_T) {
+        const int c = tid;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float sv[32];
+            tmem_ld32(tm_lane + TM_S + q4 * 32, sv);
+            float *dst = p.S_T + ((size_t)bh * DK + c) * DV + q4 * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4 *>(dst + i) = make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3]);
+        }
+    }
+    if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, TM_COLS);
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [B*T, H, D] token-major tensor; box = 64 tokens x 1 head x D.
+bool make_map(CUtensorMap *m, const void *base, bool f32, int B, int T, int H, int D)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t esz = f32 ? 4 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)H * D * esz};
+    cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool forward_tc_supported(const FwdArgs &a)
+{
+    return a.bf16 && a.dk == DK && a.dv == DV && a.T > 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
+{
+    CUtensorMap mq, mk, mb, mv, mw, mla;
+    if (!make_map(&mq, a.q, false, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, false, a.B, a.T, a.H, DK) ||
+        !make_map(&mb, a.b, false, a.B, a.T, a.H, DK) || !make_map(&mv, a.v, false, a.B, a.T, a.H, DV) ||
+        !make_map(&mw, a.w, false, a.B, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    TcParams p{a.B, a.T, a.H, a.S0, static_cast<__nv_bfloat16 *>(a.o), a.S_T, a.saved_states, a.status};
+    fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, p);
+    return cudaGetLastError();
+}
 
 }  // namespace gdr2
