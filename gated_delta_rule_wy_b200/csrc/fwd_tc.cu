@@ -54,28 +54,31 @@ using namespace sm100;
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
-constexpr int NT = 128;
+constexpr int NT = 256;                           // 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kFactorLimit = 80.f;              // |exponent| of one decay factor
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ----
-constexpr uint32_t OFF_STG_Q = 0;            // q  [64][128] bf16; later T (bf16, swizzled)
-constexpr uint32_t OFF_STG_K = 16384;        // k
-constexpr uint32_t OFF_STG_B = 32768;        // b
-constexpr uint32_t OFF_STG_V = 49152;        // v; later A (fp32 [64][68]) over V and W
-constexpr uint32_t OFF_STG_W = 65536;        // w
-constexpr uint32_t OFF_STG_LA = 81920;       // log_alpha [64][128] fp32; exact path: G
-constexpr uint32_t OFF_STACK = 114688;       // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128; later S^T
-constexpr uint32_t OFF_R0 = 147456;          // R_0 32 x 128
-constexpr uint32_t OFF_R1 = 155648;          // R_1 64 x 128; U (128 x 64) over R0..R1
-constexpr uint32_t OFF_Z = 172032;           // Z 64 x 128 (value side); later W^T
-constexpr uint32_t OFF_QH = 188416;          // Q (.) exp G, 64 x 128
-constexpr uint32_t OFF_KT = 204800;          // K (.) exp(G_C - G), 64 x 128
-constexpr uint32_t OFF_P = 221184;           // P 64 x 64
-constexpr uint32_t OFF_MISC = 229376;        // barriers, per-channel vectors
+constexpr uint32_t OFF_STG_Q = 0;       // q  [64][128] bf16; later T (bf16 [64][64], swizzled)
+constexpr uint32_t OFF_STG_K = 16384;   // k; later T (fp32 [64][68]) over K and B
+constexpr uint32_t OFF_STG_B = 32768;   // b; later (from +2048) the block-product scratch
+constexpr uint32_t OFF_STG_V = 49152;   // v; later A (fp32 [64][68]) over V and W
+constexpr uint32_t OFF_STG_W = 65536;   // w
+constexpr uint32_t OFF_STG_LA = 81920;  // log_alpha [64][128] fp32; then per-channel references; exact path: G
+constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128; later S^T
+constexpr uint32_t OFF_R0 = 147456;     // R_0 32 x 128
+constexpr uint32_t OFF_R1 = 155648;     // R_1 64 x 128; U (128 x 64) over R0..R1, then the O tile
+constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later W^T
+constexpr uint32_t OFF_QH = 188416;     // Q (.) exp G, 64 x 128
+constexpr uint32_t OFF_KT = 204800;     // K (.) exp(G_C - G), 64 x 128
+constexpr uint32_t OFF_P = 221184;      // prefix-scan scratch during prep; then P 64 x 64
+constexpr uint32_t OFF_MISC = 229376;   // barriers, per-channel vectors
 constexpr uint32_t MISC_BYTES = 1664;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-constexpr int A_LD = 68;                     // fp32 row stride of the A scratch
+constexpr int F_LD = 68;                // fp32 row stride of the A and T scratch
+constexpr uint32_t OFF_T32 = OFF_STG_K;
+constexpr uint32_t OFF_Y = OFF_STG_B + 2048;  // 16 x (3*16 + 4) fp32
+constexpr int Y_LD = 52;
 constexpr uint32_t TX_BYTES = 5 * 16384 + 32768;
 
 // TMEM columns
@@ -86,12 +89,10 @@ struct Misc {
     uint64_t bar_tma;
     uint64_t bar_mma;
     uint32_t tmem_base;
-    int flag;
-    int abort;
-    int pad;
+    int pad[3];
     float gC[DK];    // exp(G_C)
-    float eg0[DK];   // W combine factor of half-chunk 0
-    float eg1[DK];   // ... of half-chunk 1
+    float eg0[DK];   // W combine factor of half-chunk 0: exp(g_0)
+    float eg1[DK];   // ... of half-chunk 1: exp(g_1)
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 
@@ -132,10 +133,22 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8])
     }
 }
 
+__device__ __forceinline__ void load8f(const float *p, float (&f)[8])
+{
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ void store8f(float *p, const float (&f)[8])
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+}
+
 struct TcParams {
     int B, T, H;
     const float *S0;
-    __nv_bfloat16 *o;
     float *S_T;
     float *saved_states;
     unsigned *status;
@@ -144,23 +157,25 @@ struct TcParams {
 __global__ void __launch_bounds__(NT, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
-              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la, TcParams p)
+              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
+              const __grid_constant__ CUtensorMap tm_o, TcParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Misc &ms = *reinterpret_cast<Misc *>(sm + OFF_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quarter = warp & 3, colhalf = warp >> 2;
     const int bh = blockIdx.x;
     const int bb = bh / p.H, h = bh % p.H;
-    const int T = p.T, H = p.H;
+    const int T = p.T;
     const int NC = (T + C - 1) / C;
 
     if (tid == 0) {
         mbar_init(&ms.bar_tma, 1);
         mbar_init(&ms.bar_mma, 1);
         fence_mbar_init();
-        ms.abort = 0;
     }
     if (warp == 0) {
         tmem_alloc(&ms.tmem_base, TM_COLS);
@@ -170,30 +185,30 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tm = ms.tmem_base;
-    const uint32_t tm_lane = tm + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+    const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);  // this warp's TMEM lanes
+    const int row = quarter * 32 + lane;                              // this thread's TMEM lane
 
     auto issue_loads = [&](int n) {
-        const int row = bb * T + n * C;
+        const int t0 = n * C;
         mbar_arrive_expect_tx(&ms.bar_tma, TX_BYTES);
-        tma_load_3d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, h, row);
-        tma_load_3d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, h, row);
-        tma_load_3d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, h, row);
-        tma_load_3d(sm + OFF_STG_V, &tm_v, &ms.bar_tma, 0, h, row);
-        tma_load_3d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, h, row);
-        tma_load_3d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, h, row);
+        tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, h, t0, bb);
+        tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, h, t0, bb);
+        tma_load_4d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, h, t0, bb);
+        tma_load_4d(sm + OFF_STG_V, &tm_v, &ms.bar_tma, 0, h, t0, bb);
+        tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, h, t0, bb);
+        tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, h, t0, bb);
     };
     if (tid == 0 && NC > 0) issue_loads(0);
 
-    // ---- initial state into TMEM (thread c owns row c) ----
+    // ---- initial state into TMEM: lane c, columns j (half per warp) ----
     {
-        const int c = tid;
         float v[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int j0 = colhalf * 64 + q2 * 32;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                v[i] = p.S0 ? p.S0[((size_t)bh * DK + c) * DV + q4 * 32 + i] : 0.f;
-            tmem_st32(tm_lane + TM_S + q4 * 32, v);
+            for (int i = 0; i < 32; ++i) v[i] = p.S0 ? p.S0[((size_t)bh * DK + row) * DV + j0 + i] : 0.f;
+            tmem_st32(tm_lane + TM_S + j0, v);
         }
     }
     tc_fence_before_sync();
@@ -214,96 +229,105 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_after_sync();
     };
 
-    // prep mapping: channel octet o8 (channels 8*o8 .. +7), token group tg (tokens 8*tg .. +7)
-    const int o8 = warp * 4 + (lane >> 3);
-    const int tg = lane & 7;
-    const int HI = tg >> 2;  // half-chunk of this thread's tokens
+    // prep mapping: channel octet o8 (channels 8*o8 .. +7), token group tg (tokens 4*tg .. +3)
+    const int o8 = tid & 15;
+    const int tg = tid >> 4;
+    const int HI = tg >> 3;  // half-chunk of this thread's tokens
+    float *A32 = reinterpret_cast<float *>(sm + OFF_STG_V);
+    float *T32 = reinterpret_cast<float *>(sm + OFF_T32);
+    float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
     for (int n = 0; n < NC && !timed_out; ++n) {
         const int t0 = n * C;
         const int Cn = min(C, T - t0);
+        if (tid == 0) bulk_wait_group_read0();  // the previous O tile has left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
-        float G[8][8];  // G[token m][channel x], cumulative within the chunk
+        // Rows beyond T are zero-filled by TMA (per-batch extent), so padded tokens are inert.
+        float G[4][8];
+        float *scan = reinterpret_cast<float *>(sm + OFF_P);         // [16 groups][128]
+        float *refs = reinterpret_cast<float *>(sm + OFF_STG_LA);    // g0, g1, gC after the scan
         {
             const float *la_s = reinterpret_cast<const float *>(sm + OFF_STG_LA);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int t = tg * 8 + m;
-                const float4 a0 = *reinterpret_cast<const float4 *>(la_s + t * DK + o8 * 8);
-                const float4 a1 = *reinterpret_cast<const float4 *>(la_s + t * DK + o8 * 8 + 4);
-                const float la[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            for (int m = 0; m < 4; ++m) {
+                float la[8];
+                load8f(la_s + (tg * 4 + m) * DK + o8 * 8, la);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const float l = (t < Cn) ? clamp_log_alpha(la[x]) : 0.f;
-                    G[m][x] = (m == 0 ? 0.f : G[m - 1][x]) + l;
-                }
+                for (int x = 0; x < 8; ++x) G[m][x] = (m == 0 ? 0.f : G[m - 1][x]) + clamp_log_alpha(la[x]);
             }
-            // exclusive prefix over the 8 token groups (8 consecutive lanes)
+            store8f(scan + tg * DK + o8 * 8, G[3]);
+        }
+        __syncthreads();
+        if (tid < DK) {
+            // exclusive prefix over the 16 token groups of channel c
+            const int c = tid;
+            float run = 0.f, g0 = 0.f, g1 = 0.f;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const float tot = G[7][x];
-                float inc = tot;
-#pragma unroll
-                for (int d = 1; d < 8; d <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, inc, d, 8);
-                    if (tg >= d) inc += y;
-                }
-                const float ex = inc - tot;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) G[m][x] += ex;
+            for (int g = 0; g < 16; ++g) {
+                if (g == 4) g0 = run;   // G at token 15
+                if (g == 12) g1 = run;  // G at token 47
+                const float v = scan[g * DK + c];
+                scan[g * DK + c] = run;
+                run += v;
             }
+            refs[c] = g0;
+            refs[DK + c] = g1;
+            refs[2 * DK + c] = run;  // G_C
+            ms.gC[c] = __expf(run);
+            ms.eg0[c] = __expf(g0);
+            ms.eg1[c] = __expf(g1);
         }
-        float g0[8], g1[8], gC[8];
-        const int grp = lane & ~7;
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-            g0[x] = __shfl_sync(0xffffffffu, G[7][x], grp | 1);  // token 15
-            g1[x] = __shfl_sync(0xffffffffu, G[7][x], grp | 5);  // token 47
-            gC[x] = __shfl_sync(0xffffffffu, G[7][x], grp | 7);  // token 63
-        }
+        __syncthreads();
         bool risky = false;
+        float g0[8], g1[8], gC[8];
+        load8f(refs + o8 * 8, g0);
+        load8f(refs + DK + o8 * 8, g1);
+        load8f(refs + 2 * DK + o8 * 8, gC);
+        {
+            float ex[8];
+            load8f(scan + tg * DK + o8 * 8, ex);
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) G[m][x] += ex[x];
+        }
         {
             const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_Q);
             const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             const __nv_bfloat16 *vs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_V);
             const __nv_bfloat16 *ws = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_W);
-            float egI[8], kcf[8], r10[8];
+            float egI[8], kcf[8], r10[8], gr[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
-                const float gr = HI ? g1[x] : g0[x];
-                egI[x] = __expf(gr);           // exp(g_I)
-                kcf[x] = __expf(gC[x] - gr);   // exp(G_C - g_I)
-                r10[x] = __expf(g1[x] - g0[x]);
+                gr[x] = HI ? g1[x] : g0[x];
+                egI[x] = __expf(gr[x]);          // exp(g_I)
+                kcf[x] = __expf(gC[x] - gr[x]);  // exp(G_C - g_I)
+                r10[x] = __expf(g1[x] - g0[x]);  // exp(g_1 - g_0)
             }
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int t = tg * 8 + m;
+            for (int m = 0; m < 4; ++m) {
+                const int t = tg * 4 + m;
                 float qv[8], kv[8], bv[8], vv[8], wv[8];
                 unpack8(*reinterpret_cast<const uint4 *>(qs + t * DK + o8 * 8), qv);
                 unpack8(*reinterpret_cast<const uint4 *>(ks + t * DK + o8 * 8), kv);
                 unpack8(*reinterpret_cast<const uint4 *>(bs + t * DK + o8 * 8), bv);
                 unpack8(*reinterpret_cast<const uint4 *>(vs + t * DV + o8 * 8), vv);
                 unpack8(*reinterpret_cast<const uint4 *>(ws + t * DV + o8 * 8), wv);
-                const bool live = t < Cn;
                 float le[8], lq[8], r[8], kt[8], qh[8], z[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
-                    const float gr = HI ? g1[x] : g0[x];
-                    const float d = G[m][x] - gr;
+                    const float d = G[m][x] - gr[x];
                     risky |= fabsf(d) > kFactorLimit;
                     const float xl = __expf(d), yr = __expf(-d);
-                    const float kk = live ? kv[x] : 0.f;
-                    const float qq = live ? qv[x] : 0.f;
-                    const float ee = live ? bv[x] * kv[x] : 0.f;
-                    le[x] = ee * xl;
-                    lq[x] = qq * xl;
-                    r[x] = kk * yr;
+                    le[x] = bv[x] * kv[x] * xl;
+                    lq[x] = qv[x] * xl;
+                    r[x] = kv[x] * yr;
                     kt[x] = r[x] * kcf[x];
                     qh[x] = lq[x] * egI[x];
-                    z[x] = live ? wv[x] * vv[x] : 0.f;
+                    z[x] = wv[x] * vv[x];
                 }
                 const int tl = t - 32 * HI;  // token within its half-chunk
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
@@ -321,33 +345,21 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
                 *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
             }
-            if (tg == 0) {
-#pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    ms.gC[o8 * 8 + x] = __expf(gC[x]);
-                    ms.eg0[o8 * 8 + x] = __expf(g0[x]);
-                    ms.eg1[o8 * 8 + x] = __expf(g1[x]);
-                }
-            }
         }
         const bool exact = __syncthreads_or(risky) != 0;
-        float *A32 = reinterpret_cast<float *>(sm + OFF_STG_V);
         if (exact) {
             // ---- exact path: G to shared memory, pairwise exponentials ----
             float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
 #pragma unroll
-            for (int m = 0; m < 8; ++m)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) Gs[(tg * 8 + m) * DK + o8 * 8 + x] = G[m][x];
+            for (int m = 0; m < 4; ++m) store8f(Gs + (tg * 4 + m) * DK + o8 * 8, G[m]);
             __syncthreads();
             const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_Q);
             const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             // operands with one exponential of a non-positive argument each
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int t = tg * 8 + m;
-                const bool live = t < Cn;
+            for (int m = 0; m < 4; ++m) {
+                const int t = tg * 4 + m;
                 float qv[8], kv[8], bv[8], le[8], kt[8], qh[8];
                 unpack8(*reinterpret_cast<const uint4 *>(qs + t * DK + o8 * 8), qv);
                 unpack8(*reinterpret_cast<const uint4 *>(ks + t * DK + o8 * 8), kv);
@@ -355,25 +367,22 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
                     const float eg = __expf(G[m][x]);
-                    le[x] = live ? bv[x] * kv[x] * eg : 0.f;
-                    qh[x] = live ? qv[x] * eg : 0.f;
-                    kt[x] = live ? kv[x] * __expf(gC[x] - G[m][x]) : 0.f;
+                    le[x] = bv[x] * kv[x] * eg;
+                    qh[x] = qv[x] * eg;
+                    kt[x] = kv[x] * __expf(gC[x] - G[m][x]);
                 }
                 const int tl = t - 32 * HI;
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
                 *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
                 *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
             }
-            if (tg == 0) {
-#pragma unroll
-                for (int x = 0; x < 8; ++x) ms.eg0[o8 * 8 + x] = ms.eg1[o8 * 8 + x] = 1.f;
-            }
-            // A and P rows: thread -> row t = tid / 2, columns half*32 .. +31
+            if (tid < DK) ms.eg0[tid] = ms.eg1[tid] = 1.f;
+            // A and P rows: thread -> row t = tid / 4, columns 16*(tid % 4) .. +15
             {
-                const int t = tid >> 1, i0 = (tid & 1) * 32;
-                float accA[32], accP[32];
+                const int t = tid >> 2, i0 = (tid & 3) * 16;
+                float accA[16], accP[16];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) accA[u] = accP[u] = 0.f;
+                for (int u = 0; u < 16; ++u) accA[u] = accP[u] = 0.f;
                 if (i0 <= t && t < Cn) {
                     for (int c = 0; c < DK; ++c) {
                         const float gt = Gs[t * DK + c];
@@ -381,7 +390,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         const float et = __bfloat162float(bs[t * DK + c]) * kt_;
                         const float qt = __bfloat162float(qs[t * DK + c]);
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) {
+                        for (int u = 0; u < 16; ++u) {
                             const int i = i0 + u;
                             if (i <= t) {
                                 const float f = __bfloat162float(ks[i * DK + c]) * __expf(gt - Gs[i * DK + c]);
@@ -391,14 +400,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         }
                     }
                 }
-                float pr[8];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int i = i0 + u;
-                    A32[t * A_LD + i] = (i < t) ? accA[u] : 0.f;
+                    A32[t * F_LD + i] = (i < t) ? accA[u] : 0.f;
                 }
 #pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
+                for (int k8 = 0; k8 < 2; ++k8) {
+                    float pr[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) {
                         const int i = i0 + k8 * 8 + x;
@@ -427,80 +436,129 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
             tc_fence_after_sync();
-            // rows: warp 0 -> A rows 0..31, warp 1 -> P rows 0..31 (32 cols of AP0),
-            //       warp 2 -> A rows 32..63, warp 3 -> P rows 32..63 (64 cols of AP1)
-            const bool isP = (warp & 1) != 0;
-            const int t = (warp >= 2 ? 32 : 0) + lane;
-            const int ncol = warp >= 2 ? 64 : 32;
-            float row[64];
-            {
-                float v[32];
-                tmem_ld32(tm_lane + (warp >= 2 ? TM_AP1 : TM_AP0), v);
+            // quarter 0: A rows 0..31, 1: P rows 0..31 (32 columns of AP0),
+            // quarter 2: A rows 32..63, 3: P rows 32..63 (64 columns of AP1); colhalf splits columns
+            const bool isP = (quarter & 1) != 0;
+            const int t = (quarter >= 2 ? 32 : 0) + lane;
+            if (quarter < 2) {
+                if (colhalf == 0) {
+                    float v[32];
+                    tmem_ld32(tm_lane + TM_AP0, v);
+                    if (!isP) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) row[i] = v[i];
-                if (warp >= 2) {
-                    tmem_ld32(tm_lane + TM_AP1 + 32, v);
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(A32 + t * F_LD + i) =
+                                make_float4(i < t ? v[i] : 0.f, i + 1 < t ? v[i + 1] : 0.f,
+                                            i + 2 < t ? v[i + 2] : 0.f, i + 3 < t ? v[i + 3] : 0.f);
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) row[32 + i] = v[i];
+                        for (int k8 = 0; k8 < 4; ++k8) {
+                            float pr[8];
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) pr[x] = (k8 * 8 + x <= t) ? v[k8 * 8 + x] : 0.f;
+                            *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = pack8(pr);
+                        }
+                    }
                 } else {
+                    // columns 32..63 of rows 0..31 are zero
+                    if (!isP) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) row[32 + i] = 0.f;
-                }
-            }
-            (void)ncol;
-            if (!isP) {
+                        for (int i = 32; i < 64; i += 4)
+                            *reinterpret_cast<float4 *>(A32 + t * F_LD + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    } else {
+                        const float zz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < 64; i += 4) {
-                    float4 a;
-                    a.x = (i + 0 < t) ? row[i + 0] : 0.f;
-                    a.y = (i + 1 < t) ? row[i + 1] : 0.f;
-                    a.z = (i + 2 < t) ? row[i + 2] : 0.f;
-                    a.w = (i + 3 < t) ? row[i + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(A32 + t * A_LD + i) = a;
+                        for (int k8 = 4; k8 < 8; ++k8)
+                            *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = pack8(zz);
+                    }
                 }
             } else {
+                float v[32];
+                tmem_ld32(tm_lane + TM_AP1 + colhalf * 32, v);
+                const int ib = colhalf * 32;
+                if (!isP) {
 #pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8) {
-                    float pr[8];
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(A32 + t * F_LD + ib + i) =
+                            make_float4(ib + i < t ? v[i] : 0.f, ib + i + 1 < t ? v[i + 1] : 0.f,
+                                        ib + i + 2 < t ? v[i + 2] : 0.f, ib + i + 3 < t ? v[i + 3] : 0.f);
+                } else {
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) pr[x] = (k8 * 8 + x <= t) ? row[k8 * 8 + x] : 0.f;
-                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = pack8(pr);
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        float pr[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) pr[x] = (ib + k8 * 8 + x <= t) ? v[k8 * 8 + x] : 0.f;
+                        *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, colhalf * 4 + k8, 64)) = pack8(pr);
+                    }
                 }
             }
             tc_fence_before_sync();
             __syncthreads();
         }
 
-        // ================= UT solve: T = (I + A)^{-1}, column s by two threads =================
-        {
-            const int s = tid >> 1, par = tid & 1;
-            float half[32];  // T[2m + par][s]
+        // ================= UT solve: T = (I + A)^{-1} by 16 x 16 blocks =================
+        // Diagonal blocks D_I = (I + A_II)^{-1} by forward substitution (one column per
+        // thread), then block rows I = 1..3: T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ.
+        if (tid < 64) {
+            const int I = tid >> 4, sl = tid & 15;
+            const float *Ab = A32 + (16 * I) * F_LD + 16 * I;
+            float col[16];
 #pragma unroll
-            for (int m = 0; m < 32; ++m) half[m] = 0.f;
+            for (int tl = 0; tl < 16; ++tl) {
+                float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int t = 0; t < C; ++t) {
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                for (int m = 0; 2 * m < t; ++m) {
-                    const int i = 2 * m + par;
-                    const float av = (i < t) ? A32[t * A_LD + i] : 0.f;
-                    if ((m & 3) == 0) a0 = fmaf(av, half[m], a0);
-                    else if ((m & 3) == 1) a1 = fmaf(av, half[m], a1);
-                    else if ((m & 3) == 2) a2 = fmaf(av, half[m], a2);
-                    else a3 = fmaf(av, half[m], a3);
+                for (int il = 0; il < tl; ++il) {
+                    if (il & 1) a1 = fmaf(Ab[tl * F_LD + il], col[il], a1);
+                    else a0 = fmaf(Ab[tl * F_LD + il], col[il], a0);
                 }
-                float acc = (a0 + a1) + (a2 + a3);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                const float val = (t < s) ? 0.f : (t == s ? 1.f : -acc);
-                if ((t & 1) == par) half[t >> 1] = val;
+                col[tl] = (tl < sl) ? 0.f : (tl == sl ? 1.f : -(a0 + a1));
             }
-            // T -> bf16, K-major [t][s] (64 wide), over the q staging buffer
-            __nv_bfloat16 *Tb = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_STG_Q);
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const int t = 2 * m + par;
-                *reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<unsigned char *>(Tb) + sw_off(t, s, 64)) =
-                    __float2bfloat16_rn(half[m]);
+            for (int tl = 0; tl < 16; ++tl) T32[(16 * I + tl) * F_LD + 16 * I + sl] = col[tl];
+        } else {
+            // zero the blocks above the diagonal (and seed the rest)
+            for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
+                const int r = idx >> 6, cc = idx & 63;
+                if ((cc >> 4) != (r >> 4)) T32[r * F_LD + cc] = 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int I = 1; I < 4; ++I) {
+            // Y_J = sum_{K=J}^{I-1} A_IK T_KJ  (16 x 16 each, J < I)
+            for (int idx = tid; idx < I * 256; idx += NT) {
+                const int J = idx >> 8, r = (idx >> 4) & 15, s = idx & 15;
+                const float *Ar = A32 + (16 * I + r) * F_LD;
+                float acc0 = 0.f, acc1 = 0.f;
+                for (int u = 16 * J; u < 16 * I; u += 2) {
+                    acc0 = fmaf(Ar[u], T32[u * F_LD + 16 * J + s], acc0);
+                    acc1 = fmaf(Ar[u + 1], T32[(u + 1) * F_LD + 16 * J + s], acc1);
+                }
+                Ys[r * Y_LD + 16 * J + s] = acc0 + acc1;
+            }
+            __syncthreads();
+            // T_IJ = -D_I Y_J
+            for (int idx = tid; idx < I * 256; idx += NT) {
+                const int J = idx >> 8, r = (idx >> 4) & 15, s = idx & 15;
+                const float *Dr = T32 + (16 * I + r) * F_LD + 16 * I;
+                float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int u = 0; u < 16; u += 2) {
+                    acc0 = fmaf(Dr[u], Ys[u * Y_LD + 16 * J + s], acc0);
+                    acc1 = fmaf(Dr[u + 1], Ys[(u + 1) * Y_LD + 16 * J + s], acc1);
+                }
+                T32[(16 * I + r) * F_LD + 16 * J + s] = -(acc0 + acc1);
+            }
+            __syncthreads();
+        }
+        // T -> bf16, K-major [t][s] (64 wide), over the q staging buffer
+        {
+            const int t = tid >> 2, k0 = (tid & 3) * 2;
+#pragma unroll
+            for (int k8 = k0; k8 < k0 + 2; ++k8) {
+                float f[8];
+                load8f(T32 + t * F_LD + k8 * 8, f);
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_Q + sw_chunk(t, k8, 64)) = pack8(f);
             }
         }
         mma_sync_point();
@@ -530,29 +588,29 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
         // ================= W epilogue, S copy and state decay =================
         {
-            const int c = tid;
+            const int c = row;
             const float e0 = ms.eg0[c], e1 = ms.eg1[c];
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            {
                 float w0[32], w1[32];
-                tmem_ld32(tm_lane + TM_W0 + hf * 32, w0);
-                tmem_ld32(tm_lane + TM_W1 + hf * 32, w1);
+                tmem_ld32(tm_lane + TM_W0 + colhalf * 32, w0);
+                tmem_ld32(tm_lane + TM_W1 + colhalf * 32, w1);
 #pragma unroll
                 for (int k8 = 0; k8 < 4; ++k8) {
                     float f[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) f[x] = e0 * w0[k8 * 8 + x] + e1 * w1[k8 * 8 + x];
                     // W^T stored MN-major: row c, 64 t-columns
-                    *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, hf * 4 + k8, 128)) = pack8(f);
+                    *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
                 }
             }
             const float gc = ms.gC[c];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int j0 = colhalf * 64 + q2 * 32;
                 float sv[32];
-                tmem_ld32(tm_lane + TM_S + q4 * 32, sv);
+                tmem_ld32(tm_lane + TM_S + j0, sv);
                 if (p.saved_states) {
-                    float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c) * DV + q4 * 32;
+                    float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c) * DV + j0;
 #pragma unroll
                     for (int i = 0; i < 32; i += 4)
                         *reinterpret_cast<float4 *>(dst + i) = make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3]);
@@ -563,11 +621,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int x = 0; x < 8; ++x) f[x] = sv[k8 * 8 + x];
                     // S^T stored MN-major (j contiguous): [j-block][c rows][64 j]
-                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(c, q4 * 4 + k8, 128)) = pack8(f);
+                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(c, (j0 >> 3) + k8, 128)) = pack8(f);
                 }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) sv[i] *= gc;
-                tmem_st32(tm_lane + TM_S + q4 * 32, sv);
+                tmem_st32(tm_lane + TM_S + j0, sv);
             }
         }
         mma_sync_point();
@@ -589,18 +647,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_after_sync();
         // ================= U epilogue: U^T rows -> bf16 [j][64 t] =================
         {
-            const int j = tid;
+            float u[32];
+            tmem_ld32(tm_lane + TM_U + colhalf * 32, u);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float u[32];
-                tmem_ld32(tm_lane + TM_U + hf * 32, u);
+            for (int k8 = 0; k8 < 4; ++k8) {
+                float f[8];
 #pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    float f[8];
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
-                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(j, hf * 4 + k8, 128)) = pack8(f);
-                }
+                for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
+                *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
             }
         }
         mma_sync_point();
@@ -620,36 +674,37 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // ================= O epilogue =================
+        // ================= O epilogue: O^T rows -> bf16 tile [t][j] -> one TMA store =================
         {
-            const int j = tid;
+            float ov[32];
+            tmem_ld32(tm_lane + TM_O + colhalf * 32, ov);
+            __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_R0);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float ov[32];
-                tmem_ld32(tm_lane + TM_O + hf * 32, ov);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int t = hf * 32 + i;
-                    if (t < Cn) p.o[(((size_t)bb * T + t0 + t) * H + h) * DV + j] = __float2bfloat16_rn(ov[i]);
-                }
-            }
+            for (int i = 0; i < 32; ++i) ot[(colhalf * 32 + i) * DV + row] = __float2bfloat16_rn(ov[i]);
         }
+        fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_o, sm + OFF_R0, 0, h, t0, bb);  // rows beyond T are clipped
+            bulk_commit_group();
+        }
+        (void)Cn;
     }
 
     if (!timed_out && p.S_T) {
-        const int c = tid;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int j0 = colhalf * 64 + q2 * 32;
             float sv[32];
-            tmem_ld32(tm_lane + TM_S + q4 * 32, sv);
-            float *dst = p.S_T + ((size_t)bh * DK + c) * DV + q4 * 32;
+            tmem_ld32(tm_lane + TM_S + j0, sv);
+            float *dst = p.S_T + ((size_t)bh * DK + row) * DV + j0;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4 *>(dst + i) = make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3]);
         }
     }
+    if (tid == 0) bulk_wait_group0();
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
@@ -675,17 +730,19 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// [B*T, H, D] token-major tensor; box = 64 tokens x 1 head x D.
+// [B, T, H, D] token-major tensor as a 4-D map {D, H, T, B}; box = D x 1 head x 64
+// tokens x 1 sequence. The per-sequence extent T makes loads past the end of a
+// sequence read zeros and stores past it drop.
 bool make_map(CUtensorMap *m, const void *base, bool f32, int B, int T, int H, int D)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t esz = f32 ? 4 : 2;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * T};
-    cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)H * D * esz};
-    cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * esz, (cuuint64_t)H * D * esz, (cuuint64_t)T * H * D * esz};
+    cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -701,15 +758,16 @@ bool forward_tc_supported(const FwdArgs &a)
 
 cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
 {
-    CUtensorMap mq, mk, mb, mv, mw, mla;
+    CUtensorMap mq, mk, mb, mv, mw, mla, mo;
     if (!make_map(&mq, a.q, false, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, false, a.B, a.T, a.H, DK) ||
         !make_map(&mb, a.b, false, a.B, a.T, a.H, DK) || !make_map(&mv, a.v, false, a.B, a.T, a.H, DV) ||
-        !make_map(&mw, a.w, false, a.B, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK))
+        !make_map(&mw, a.w, false, a.B, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK) ||
+        !make_map(&mo, a.o, false, a.B, a.T, a.H, DV))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    TcParams p{a.B, a.T, a.H, a.S0, static_cast<__nv_bfloat16 *>(a.o), a.S_T, a.saved_states, a.status};
-    fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, p);
+    TcParams p{a.B, a.T, a.H, a.S0, a.S_T, a.saved_states, a.status};
+    fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, mo, p);
     return cudaGetLastError();
 }
 

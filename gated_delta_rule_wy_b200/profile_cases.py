@@ -1,0 +1,53 @@
+"""Run one libgdr2.so kernel on its benchmark workload, for profilers.
+
+    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd} [--launches N]
+
+fwd     gdr2_forward   B=4 H=16 T=4096 d=128 bf16 (the 1.3B-model layer)
+decode  gdr2_decode_step  256 sequences x 16 heads, d=128, fp32 state (256 MiB)
+bwd     gdr2_backward  B=2 H=16 T=4096 d=128 bf16 with saved chunk states
+
+Inputs are drawn once (seeded) and stay on the device; the kernel is then
+launched N times back to back (use ncu -s/-c to pick one launch).
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import inputs as I
+from .binding import gdr2_backward, gdr2_decode_step, gdr2_forward, gdr2_sync_status
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kernel", choices=("fwd", "decode", "bwd"))
+    ap.add_argument("--launches", type=int, default=2)
+    args = ap.parse_args()
+    torch.cuda.set_device(0)
+    if args.kernel == "fwd":
+        x = I.make_forward_inputs(**I.FWD_1P3B_BF16).to("cuda")
+        o = torch.empty_like(x.v)
+        for _ in range(args.launches):
+            gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o)
+    elif args.kernel == "decode":
+        c = I.DECODE_1P3B
+        gen = torch.Generator(device="cuda").manual_seed(c["seed"])
+        S = torch.randn((c["N"], c["H"], c["dk"], c["dv"]), device="cuda", generator=gen) * c["state_std"]
+        tok = I.make_token_inputs((c["N"], c["H"], c["dk"]), (c["N"], c["H"], c["dv"]), c["dtype"],
+                                  c["decay_shift"], gen)
+        for _ in range(args.launches):
+            gdr2_decode_step(*tok, S)
+    else:
+        c = I.BWD_1P3B_BF16
+        x = I.make_forward_inputs(**c).to("cuda")
+        dO = I.make_upstream_grad(c["B"], c["T"], c["H"], c["dv"], c["seed"], dtype=c["dtype"]).cuda()
+        _, _, saved = gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, save_states=True)
+        for _ in range(args.launches):
+            gdr2_backward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, dO, None, None, saved)
+    gdr2_sync_status()
+    print(f"profile_cases {args.kernel}: {args.launches} launches ok")
+
+
+if __name__ == "__main__":
+    main()
