@@ -31,7 +31,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -49,9 +48,7 @@ BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 2 * 256 + 256  # q,k,v bf16 + log_alpha f
 FLOP_PER_TOKEN_HEAD = 139_264  # chunk products at C=64, d=128, triangular parts counted once
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+LAUNCHES_PER_STEP = 2  # chunk kernel + scan kernel (tensor-core path)
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -119,53 +116,63 @@ def committed_traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while active."""
+    """SM clock and clock-event (throttle) reasons polled through NVML every ~2 ms
+    while the timed region runs (reading only; no setting is touched)."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = None
+
+    def _handle(self, nv):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def __enter__(self):
+        import threading
+
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    bits = int(get_reasons(h))
+                    self.reasons.update(n for b, n in self.REASONS.items() if bits & b)
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.fh.close()
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
+        if not self.samples:
             return None
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def cores() -> int:
@@ -276,7 +283,7 @@ def bench_components(dev, stream, peaks):
 
 
 def run_ours(args, world, rank, local):
-    from gated_delta_rule_wy_b200 import build, gdr2_forward, gdr2_sync_status
+    from gated_delta_rule_wy_b200 import build, gdr2_forward, gdr2_forward_workspace_bytes, gdr2_sync_status
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -291,10 +298,12 @@ def run_ours(args, world, rank, local):
     x = x_cpu.to(dev)
     B, T, H, dk, dv = cfg["B"], cfg["T"], cfg["H"], cfg["dk"], cfg["dv"]
     o = torch.empty((B, T, H, dv), dtype=cfg["dtype"], device=dev)
+    ws = torch.empty(max(1, gdr2_forward_workspace_bytes(B, T, H, dk, dv, cfg["dtype"])), dtype=torch.uint8,
+                     device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o)
+        gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -322,7 +331,7 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         for d, hsrc in zip(dbufs, pinned):
             d.copy_(hsrc, non_blocking=True)
-        oo, sT, _ = gdr2_forward(*dbufs, None, out=o)
+        oo, sT, _ = gdr2_forward(*dbufs, None, out=o, workspace=ws)
         o_host.copy_(oo, non_blocking=True)
         sT_host.copy_(sT, non_blocking=True)
 
@@ -366,7 +375,7 @@ def run_ours(args, world, rank, local):
                            "l2": "inputs larger than L2 (541 MB per step vs 126 MB)"},
                 "clocks": clk.summary(),
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps, "roofline": roofline, "tensor": tensor, "components": comps,
+                "gpu_launches": LAUNCHES_PER_STEP * args.steps, "roofline": roofline, "tensor": tensor, "components": comps,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     barrier(world)
@@ -377,7 +386,7 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     args = ap.parse_args()

@@ -23,7 +23,8 @@ CHUNK = 64
 _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
 
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
-EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward", "gdr2_decode_step",
+EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspace_bytes", "gdr2_forward",
+                    "gdr2_decode_step",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
                     "gdr2_sync_status")
 NOALLOC_SCRATCH_BYTES = 64 << 20  # GDR2_NOALLOC_SCRATCH_BYTES
@@ -55,8 +56,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_abi_version.argtypes = []
         lib.gdr2_last_error.restype = ctypes.c_char_p
         lib.gdr2_last_error.argtypes = []
+        lib.gdr2_forward_workspace_bytes.restype = Z
+        lib.gdr2_forward_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.gdr2_forward.restype = I
-        lib.gdr2_forward.argtypes = [I, I, I, I, I, I] + [P] * 11
+        lib.gdr2_forward.argtypes = [I, I, I, I, I, I] + [P] * 11 + [Z, P]
         lib.gdr2_decode_step.restype = I
         lib.gdr2_decode_step.argtypes = [I, I, I, I, I] + [P] * 9
         lib.gdr2_backward_workspace_bytes.restype = Z
@@ -120,8 +123,13 @@ def gdr2_sync_status(stream=None) -> None:
     _raise(lib, lib.gdr2_sync_status(_stream(stream)))
 
 
+def gdr2_forward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    lib = load_library()
+    return int(lib.gdr2_forward_workspace_bytes(B, T, H, dk, dv, GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
+
+
 def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_states=False,
-                 out=None, stream=None):
+                 out=None, workspace=None, stream=None):
     """Chunkwise forward. Returns (o, S_T, saved_states); S_T / saved_states may be None.
 
     q, k, b: [B, T, H, dk]; v, w: [B, T, H, dv] (fp32 or bf16, one dtype);
@@ -142,8 +150,13 @@ def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_st
     S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if final_state else None
     nc = (T + CHUNK - 1) // CHUNK
     saved = torch.empty((B, H, nc, dk, dv), dtype=torch.float32, device=dev) if save_states else None
+    need = gdr2_forward_workspace_bytes(B, T, H, dk, dv, dt)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.gdr2_forward(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
-                          _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _stream(stream))
+                          _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
+                          ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
     return o, S_T, saved
 

@@ -10,9 +10,21 @@
 //
 //   A_ti = sum_c e_t[c] k_i[c] exp(G_t[c] - G_i[c])   i < t      (e = b (.) k)
 //   P_ti = sum_c q_t[c] k_i[c] exp(G_t[c] - G_i[c])   i <= t
-//   T = (I + A)^{-1};  W = T (E (.) exp G);  U = T Z - W S      (z = w (.) v)
-//   O = (Q (.) exp G) S + P U
-//   S <- Diag(exp G_C) S + (K (.) exp(G_C - G))^T U
+//   T = (I + A)^{-1};  W = T (E (.) exp G);  U~ = T Z              (z = w (.) v)
+//   U = U~ - W S;  O = (Q (.) exp G) S + P U;  S' = Diag(gamma) S + K~^T U
+//
+// Regrouped so that the state enters one batch of products per chunk:
+//   S' = Diag(gamma) S + M S + K~^T U~,   M  = -K~^T W
+//   O  = Q' S + P U~,                     Q' = Q (.) exp G - P W
+// Everything except those two lines is independent of S, so the path is two
+// kernels:
+//   1. chunk kernel (persistent, every (batch, head, chunk) task in parallel
+//      on all SMs): decay, gated keys, [A;P], the UT solve, W, U~, M, Q';
+//      writes M, K~, U~, Q', P (bf16, already in the tensor-core operand
+//      layouts of kernel 2) and gamma = exp(G_C) to the workspace;
+//   2. scan kernel (one CTA per (batch, head), chunks in order): S stays in
+//      TMEM as fp32; per chunk one pass copies S to a bf16 operand and scales
+//      it by gamma in place, then one batch of MMAs produces S' and O^T.
 //
 // Decay range. exp(G_t - G_i) is formed as a product of two factors around a
 // per-channel reference g_I, the cumulative decay at the midpoint of the
@@ -23,21 +35,18 @@
 // is itself below fp32 range. When the guard trips (alpha near 0 over a whole
 // half-chunk, e.g. a reset) the chunk takes an exact path: A and P with one
 // exponential per (t, i, c), and the decay-weighted operands from exp(G)
-// directly. Every other chunk keeps the factorised, tensor-core path.
+// directly.
 //
-// Mapping to tcgen05 (M = 128 everywhere; T = token, c = key channel,
-// j = value channel; every accumulator is fp32 in TMEM):
-//   [A;P] : D(128 x 32|64) = [L^e_0; L^q_0; L^e_1; L^q_1] R_I^T   (K = c)
-//   W^T_I : D(c x t) = (L^e_I)^T T[:, I]^T,  W = sum_I exp(g_I) W_I (K = s in I)
-//   U^T   : D(j x t) = Z^T T^T - S^T W^T        (A negated in the second MMA)
-//   O^T   : D(j x t) = S^T Q^T + U^T P^T
-//   S     : D(c x j) = Diag(exp G_C) S + K~^T U (row scale applied in TMEM)
-// Operands are staged by TMA (no multicast) and written by the threads into
-// 128-byte-swizzled UMMA layouts; one thread issues every MMA and commit.
-//
-// Threads: 128, thread i <-> TMEM lane i. One CTA per (batch, head); the
-// chunk loop is sequential. Every mbarrier wait is bounded; on a timeout the
-// CTA records kStatusTimeout, frees its TMEM and exits.
+// Tensor-core mapping (M = 128 everywhere; t, i, s tokens, c key channel,
+// j value channel; accumulators fp32 in TMEM, operands bf16 in
+// 128-byte-swizzled shared memory written by the threads, inputs staged by
+// TMA without multicast; one thread issues every MMA):
+//   chunk kernel: [A;P] = [L^e_0; L^q_0; L^e_1; L^q_1] R_I^T (K = c)
+//                 W^T_I = (L^e_I)^T T[:, I]^T, W = sum_I exp(g_I) W_I
+//                 U~^T = Z^T T^T;  Q'^T - Q^T = -W^T P^T;  M = -K~^T W
+//   scan kernel:  S += M S_bf16 + K~^T U~;  O^T = S_bf16^T Q'^T + U~^T P^T
+// Every mbarrier wait is bounded; a CTA that gives up records kStatusTimeout,
+// frees its TMEM and exits.
 
 #include <cuda.h>
 #include <mutex>
@@ -81,9 +90,7 @@ constexpr uint32_t OFF_Y = OFF_STG_B + 2048;  // 16 x (3*16 + 4) fp32
 constexpr int Y_LD = 52;
 constexpr uint32_t TX_BYTES = 5 * 16384 + 32768;
 
-// TMEM columns
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_W0 = 256, TM_W1 = 320, TM_AP0 = 384, TM_AP1 = 416;
-constexpr uint32_t TM_COLS = 512;
+constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
 
 struct Misc {
     uint64_t bar_tma;
@@ -146,19 +153,31 @@ __device__ __forceinline__ void store8f(float *p, const float (&f)[8])
     *reinterpret_cast<float4 *>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
 }
 
-struct TcParams {
-    int B, T, H;
-    const float *S0;
-    float *S_T;
-    float *saved_states;
+// ---- workspace slot written by the chunk kernel, read by the scan kernel ----
+// (one per (batch, head, chunk); operand images in the scan kernel's layouts)
+constexpr uint32_t SLOT_M = 0;        // M = -K~^T W   [c' block][c rows][64 c'] (K-major A)
+constexpr uint32_t SLOT_KT = 32768;   // K~             [c block][t rows][64 c]   (MN-major A)
+constexpr uint32_t SLOT_U = 49152;    // U~             [j rows][64 t]            (K-major A and B)
+constexpr uint32_t SLOT_Q = 65536;    // Q'^T           [c rows][64 t]            (MN-major B)
+constexpr uint32_t SLOT_P = 81920;    // P              [t rows][64 i]            (K-major B)
+constexpr uint32_t SLOT_BYTES = 90112;
+constexpr uint32_t GAMMA_BYTES = DK * 4;  // exp(G_C), stored after all slots
+
+struct ChunkParams {
+    int B, T, H, NC;
+    int ntasks;            // B * H * NC, task = bh * NC + n
+    unsigned char *ws;     // workspace: ntasks slots, then ntasks gamma vectors
     unsigned *status;
 };
 
+// TMEM columns of the chunk kernel
+constexpr uint32_t CK_M = 0, CK_U = 128, CK_Q = 192, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384, CK_AP1 = 416;
+
 __global__ void __launch_bounds__(NT, 1)
-fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
-              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
-              const __grid_constant__ CUtensorMap tm_o, TcParams p)
+fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
+                 ChunkParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm =
@@ -167,10 +186,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quarter = warp & 3, colhalf = warp >> 2;
-    const int bh = blockIdx.x;
-    const int bb = bh / p.H, h = bh % p.H;
-    const int T = p.T;
-    const int NC = (T + C - 1) / C;
+    const int NC = p.NC;
 
     if (tid == 0) {
         mbar_init(&ms.bar_tma, 1);
@@ -188,8 +204,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);  // this warp's TMEM lanes
     const int row = quarter * 32 + lane;                              // this thread's TMEM lane
 
-    auto issue_loads = [&](int n) {
-        const int t0 = n * C;
+    auto issue_loads = [&](int task) {
+        const int bh = task / NC, n = task % NC;
+        const int bb = bh / p.H, h = bh % p.H, t0 = n * C;
         mbar_arrive_expect_tx(&ms.bar_tma, TX_BYTES);
         tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, h, t0, bb);
         tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, h, t0, bb);
@@ -198,25 +215,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, h, t0, bb);
         tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, h, t0, bb);
     };
-    if (tid == 0 && NC > 0) issue_loads(0);
-
-    // ---- initial state into TMEM: lane c, columns j (half per warp) ----
-    {
-        float v[32];
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            const int j0 = colhalf * 64 + q2 * 32;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = p.S0 ? p.S0[((size_t)bh * DK + row) * DV + j0 + i] : 0.f;
-            tmem_st32(tm_lane + TM_S + j0, v);
-        }
-    }
-    tc_fence_before_sync();
-    __syncthreads();
+    if (tid == 0 && (int)blockIdx.x < p.ntasks) issue_loads(blockIdx.x);
 
     uint32_t ph_tma = 0, ph_mma = 0;
     bool timed_out = false;
-    // every thread waits; any timeout aborts the CTA consistently
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
         const bool ok = mbar_wait_bounded(bar, ph, kWaitLimitNs);
         ph ^= 1u;
@@ -237,17 +239,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     float *T32 = reinterpret_cast<float *>(sm + OFF_T32);
     float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
-    for (int n = 0; n < NC && !timed_out; ++n) {
-        const int t0 = n * C;
-        const int Cn = min(C, T - t0);
-        if (tid == 0) bulk_wait_group_read0();  // the previous O tile has left shared memory
+    for (int task = blockIdx.x; task < p.ntasks && !timed_out; task += gridDim.x) {
+        const int n = task % NC;
+        const int Cn = min(C, p.T - n * C);
+        if (tid == 0) bulk_wait_group_read0();  // the previous task's outputs have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
-        // Rows beyond T are zero-filled by TMA (per-batch extent), so padded tokens are inert.
+        // Rows beyond T are zero-filled by TMA (per-sequence extent): padded tokens are inert.
         float G[4][8];
-        float *scan = reinterpret_cast<float *>(sm + OFF_P);         // [16 groups][128]
-        float *refs = reinterpret_cast<float *>(sm + OFF_STG_LA);    // g0, g1, gC after the scan
+        float *scan = reinterpret_cast<float *>(sm + OFF_P);       // [16 groups][128]
+        float *refs = reinterpret_cast<float *>(sm + OFF_STG_LA);  // g0, g1, gC after the scan
         {
             const float *la_s = reinterpret_cast<const float *>(sm + OFF_STG_LA);
 #pragma unroll
@@ -429,8 +431,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + (ks >> 2) * 16384 + koff, 16, 1024);
                     const uint64_t b0 = sdesc_sw128(sbase + OFF_R0 + (ks >> 2) * 4096 + koff, 16, 1024);
                     const uint64_t b1 = sdesc_sw128(sbase + OFF_R1 + (ks >> 2) * 8192 + koff, 16, 1024);
-                    mma_bf16(tm + TM_AP0, ad, b0, id0, ks > 0);
-                    mma_bf16(tm + TM_AP1, ad, b1, id1, ks > 0);
+                    mma_bf16(tm + CK_AP0, ad, b0, id0, ks > 0);
+                    mma_bf16(tm + CK_AP1, ad, b1, id1, ks > 0);
                 }
                 mma_commit(&ms.bar_mma);
             }
@@ -443,7 +445,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (quarter < 2) {
                 if (colhalf == 0) {
                     float v[32];
-                    tmem_ld32(tm_lane + TM_AP0, v);
+                    tmem_ld32(tm_lane + CK_AP0, v);
                     if (!isP) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -474,7 +476,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             } else {
                 float v[32];
-                tmem_ld32(tm_lane + TM_AP1 + colhalf * 32, v);
+                tmem_ld32(tm_lane + CK_AP1 + colhalf * 32, v);
                 const int ib = colhalf * 32;
                 if (!isP) {
 #pragma unroll
@@ -516,7 +518,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int tl = 0; tl < 16; ++tl) T32[(16 * I + tl) * F_LD + 16 * I + sl] = col[tl];
         } else {
-            // zero the blocks above the diagonal (and seed the rest)
             for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
                 const int r = idx >> 6, cc = idx & 63;
                 if ((cc >> 4) != (r >> 4)) T32[r * F_LD + cc] = 0.f;
@@ -525,7 +526,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         __syncthreads();
 #pragma unroll
         for (int I = 1; I < 4; ++I) {
-            // Y_J = sum_{K=J}^{I-1} A_IK T_KJ  (16 x 16 each, J < I)
             for (int idx = tid; idx < I * 256; idx += NT) {
                 const int J = idx >> 8, r = (idx >> 4) & 15, s = idx & 15;
                 const float *Ar = A32 + (16 * I + r) * F_LD;
@@ -537,7 +537,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 Ys[r * Y_LD + 16 * J + s] = acc0 + acc1;
             }
             __syncthreads();
-            // T_IJ = -D_I Y_J
             for (int idx = tid; idx < I * 256; idx += NT) {
                 const int J = idx >> 8, r = (idx >> 4) & 15, s = idx & 15;
                 const float *Dr = T32 + (16 * I + r) * F_LD + 16 * I;
@@ -551,7 +550,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             __syncthreads();
         }
-        // T -> bf16, K-major [t][s] (64 wide), over the q staging buffer
         {
             const int t = tid >> 2, k0 = (tid & 3) * 2;
 #pragma unroll
@@ -562,7 +560,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         mma_sync_point();
-        // ================= W^T_I = (L^e_I)^T T[:,I]^T ;  U^T = Z^T T^T =================
+        // ================= W^T_I = (L^e_I)^T T[:,I]^T ;  U~^T = Z^T T^T =================
         if (tid == 0) {
             const uint32_t idW = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -571,44 +569,218 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int ks = 0; ks < 2; ++ks) {
                     const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + (64 * I + 16 * ks) * 128, 16384, 1024);
                     const uint64_t bd = sdesc_sw128(sbase + OFF_STG_Q + (32 * I + 16 * ks) * 2, 16, 1024);
-                    mma_bf16(tm + (I ? TM_W1 : TM_W0), ad, bd, idW, ks > 0);
+                    mma_bf16(tm + (I ? CK_W1 : CK_W0), ad, bd, idW, ks > 0);
                 }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = sdesc_sw128(sbase + OFF_Z + ks * 2048, 8192, 1024);
                 const uint64_t bd = sdesc_sw128(sbase + OFF_STG_Q + ks * 32, 16, 1024);
-                mma_bf16(tm + TM_U, ad, bd, idW, ks > 0);
+                mma_bf16(tm + CK_U, ad, bd, idW, ks > 0);
             }
             mma_commit(&ms.bar_mma);
         }
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // staging is free: prefetch the next chunk's inputs
-        if (tid == 0 && n + 1 < NC) issue_loads(n + 1);
+        // staging is free: prefetch the next task's inputs
+        if (tid == 0 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
 
-        // ================= W epilogue, S copy and state decay =================
+        // ================= W -> [c][64 t] over Z;  U~ -> [j][64 t] over R0..R1 =================
+        {
+            const float e0 = ms.eg0[row], e1 = ms.eg1[row];
+            float w0[32], w1[32];
+            tmem_ld32(tm_lane + CK_W0 + colhalf * 32, w0);
+            tmem_ld32(tm_lane + CK_W1 + colhalf * 32, w1);
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+                float f[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) f[x] = e0 * w0[k8 * 8 + x] + e1 * w1[k8 * 8 + x];
+                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
+            }
+            float u[32];
+            tmem_ld32(tm_lane + CK_U + colhalf * 32, u);
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+                float f[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
+                *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
+            }
+        }
+        mma_sync_point();
+        // ================= Q'^T - Q^T = -W^T P^T ;  M = -K~^T W =================
+        if (tid == 0) {
+            const uint32_t idQ = idesc_bf16(128, 64, false, false, true);
+            const uint32_t idM = idesc_bf16(128, 128, true, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t aw = sdesc_sw128(sbase + OFF_Z + ks * 32, 16, 1024);
+                const uint64_t bp = sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024);
+                mma_bf16(tm + CK_Q, aw, bp, idQ, ks > 0);
+                const uint64_t ak = sdesc_sw128(sbase + OFF_KT + ks * 2048, 8192, 1024);
+                mma_bf16(tm + CK_M, ak, aw, idM, ks > 0);
+            }
+            mma_commit(&ms.bar_mma);
+        }
+        if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
+        tc_fence_after_sync();
+        // ================= Q' -> [c][64 t] over Z;  M -> [c' block][c][64 c'] over STACK =================
         {
             const int c = row;
-            const float e0 = ms.eg0[c], e1 = ms.eg1[c];
-            {
-                float w0[32], w1[32];
-                tmem_ld32(tm_lane + TM_W0 + colhalf * 32, w0);
-                tmem_ld32(tm_lane + TM_W1 + colhalf * 32, w1);
+            float d[32];
+            tmem_ld32(tm_lane + CK_Q + colhalf * 32, d);
+            const unsigned char *qh = sm + OFF_QH;
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+                float f[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const int t = colhalf * 32 + k8 * 8 + x;
+                    f[x] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qh + sw_off(t, c, 64))) +
+                           d[k8 * 8 + x];
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
+            }
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int c0 = colhalf * 64 + q2 * 32;
+                float mv[32];
+                tmem_ld32(tm_lane + CK_M + c0, mv);
 #pragma unroll
                 for (int k8 = 0; k8 < 4; ++k8) {
                     float f[8];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) f[x] = e0 * w0[k8 * 8 + x] + e1 * w1[k8 * 8 + x];
-                    // W^T stored MN-major: row c, 64 t-columns
-                    *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
+                    for (int x = 0; x < 8; ++x) f[x] = mv[k8 * 8 + x];
+                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(c, (c0 >> 3) + k8, 128)) = pack8(f);
                 }
             }
-            const float gc = ms.gC[c];
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
+            bulk_store(slot + SLOT_M, sm + OFF_STACK, 32768);
+            bulk_store(slot + SLOT_KT, sm + OFF_KT, 16384);
+            bulk_store(slot + SLOT_U, sm + OFF_R0, 16384);
+            bulk_store(slot + SLOT_Q, sm + OFF_Z, 16384);
+            bulk_store(slot + SLOT_P, sm + OFF_P, 8192);
+            bulk_store(p.ws + (size_t)p.ntasks * SLOT_BYTES + (size_t)task * GAMMA_BYTES, ms.gC, GAMMA_BYTES);
+            bulk_commit_group();
+        }
+    }
+    if (tid == 0) bulk_wait_group0();
+    if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, TM_COLS);
+}
+
+// ---- scan kernel ----
+constexpr uint32_t SC_SLOT0 = 0;
+constexpr uint32_t SC_SLOT1 = SLOT_BYTES;          // 90112, 1024-aligned
+constexpr uint32_t SC_SB = 2 * SLOT_BYTES;         // S^T bf16 [j block][c rows][64 j]
+constexpr uint32_t SC_O = SC_SB + 32768;           // O tile [64 t][128 j] bf16
+constexpr uint32_t SC_MISC = SC_O + 16384;
+constexpr uint32_t SC_SMEM_BYTES = SC_MISC + 1280 + 1024;
+constexpr uint32_t SC_S = 0, SC_OT = 128, SC_COLS = 256;
+
+struct ScanMisc {
+    uint64_t bar_full[2];
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int pad;
+    float gam[2][DK];
+};
+static_assert(sizeof(ScanMisc) <= 1280, "scan misc region");
+
+struct ScanParams {
+    int B, T, H, NC, ntasks;
+    const unsigned char *ws;
+    const float *S0;
+    float *S_T;
+    float *saved_states;
+    unsigned *status;
+};
+
+__global__ void __launch_bounds__(NT, 1)
+fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    ScanMisc &ms = *reinterpret_cast<ScanMisc *>(sm + SC_MISC);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quarter = warp & 3, colhalf = warp >> 2;
+    const int bh = blockIdx.x;
+    const int bb = bh / p.H, h = bh % p.H;
+    const int NC = p.NC;
+
+    if (tid == 0) {
+        mbar_init(&ms.bar_full[0], 1);
+        mbar_init(&ms.bar_full[1], 1);
+        mbar_init(&ms.bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&ms.tmem_base, SC_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tm = ms.tmem_base;
+    const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
+    const int row = quarter * 32 + lane;
+
+    auto issue_slot = [&](int n) {
+        const int sl = n & 1;
+        const size_t task = (size_t)bh * NC + n;
+        mbar_arrive_expect_tx(&ms.bar_full[sl], SLOT_BYTES + GAMMA_BYTES);
+        bulk_load(sm + (sl ? SC_SLOT1 : SC_SLOT0), p.ws + task * SLOT_BYTES, SLOT_BYTES, &ms.bar_full[sl]);
+        bulk_load(ms.gam[sl], p.ws + (size_t)p.ntasks * SLOT_BYTES + task * GAMMA_BYTES, GAMMA_BYTES,
+                  &ms.bar_full[sl]);
+    };
+    if (tid == 0) {
+        if (NC > 0) issue_slot(0);
+        if (NC > 1) issue_slot(1);
+    }
+    // initial state: lane c, columns j (half per warp)
+    {
+        float v[32];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int j0 = colhalf * 64 + q2 * 32;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = p.S0 ? p.S0[((size_t)bh * DK + row) * DV + j0 + i] : 0.f;
+            tmem_st32(tm_lane + SC_S + j0, v);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+
+    uint32_t ph_full[2] = {0, 0}, ph_mma = 0;
+    bool timed_out = false;
+    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
+        const bool ok = mbar_wait_bounded(bar, ph, kWaitLimitNs);
+        ph ^= 1u;
+        return __syncthreads_or(!ok) == 0;
+    };
+
+    for (int n = 0; n < NC; ++n) {
+        const int sl = n & 1;
+        const uint32_t slot = sbase + (sl ? SC_SLOT1 : SC_SLOT0);
+        if (!wait_bar(&ms.bar_full[sl], ph_full[sl])) { timed_out = true; break; }
+        // ---- S -> bf16 operand; S <- Diag(gamma) S in TMEM ----
+        {
+            const int c = row;
+            const float g = ms.gam[sl][c];
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int j0 = colhalf * 64 + q2 * 32;
                 float sv[32];
-                tmem_ld32(tm_lane + TM_S + j0, sv);
+                tmem_ld32(tm_lane + SC_S + j0, sv);
                 if (p.saved_states) {
                     float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c) * DV + j0;
 #pragma unroll
@@ -620,65 +792,50 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     float f[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) f[x] = sv[k8 * 8 + x];
-                    // S^T stored MN-major (j contiguous): [j-block][c rows][64 j]
-                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(c, (j0 >> 3) + k8, 128)) = pack8(f);
+                    *reinterpret_cast<uint4 *>(sm + SC_SB + sw_chunk(c, (j0 >> 3) + k8, 128)) = pack8(f);
                 }
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] *= gc;
-                tmem_st32(tm_lane + TM_S + j0, sv);
+                for (int i = 0; i < 32; ++i) sv[i] *= g;
+                tmem_st32(tm_lane + SC_S + j0, sv);
             }
         }
-        mma_sync_point();
-        // ================= U^T -= S^T W^T ;  O^T = S^T Q^T =================
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
+        // ---- S += M S_bf16 + K~^T U~ ;  O^T = S_bf16^T Q'^T + U~^T P^T ----
         if (tid == 0) {
-            const uint32_t idU = idesc_bf16(128, 64, true, true, true);
-            const uint32_t idO = idesc_bf16(128, 64, true, false);
+            const uint32_t idM = idesc_bf16(128, 128, false, true);
+            const uint32_t idK = idesc_bf16(128, 128, true, false);
+            const uint32_t idO1 = idesc_bf16(128, 64, true, true);
+            const uint32_t idO2 = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + ks * 2048, 16384, 1024);
-                const uint64_t bw = sdesc_sw128(sbase + OFF_Z + ks * 2048, 8192, 1024);
-                const uint64_t bq = sdesc_sw128(sbase + OFF_QH + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                mma_bf16(tm + TM_U, ad, bw, idU, 1);
-                mma_bf16(tm + TM_O, ad, bq, idO, ks > 0);
+                const uint64_t am = sdesc_sw128(slot + SLOT_M + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                const uint64_t bs = sdesc_sw128(sbase + SC_SB + ks * 2048, 16384, 1024);
+                mma_bf16(tm + SC_S, am, bs, idM, 1);
+                const uint64_t bq = sdesc_sw128(slot + SLOT_Q + ks * 2048, 8192, 1024);
+                mma_bf16(tm + SC_OT, bs, bq, idO1, ks > 0);
             }
-            mma_commit(&ms.bar_mma);
-        }
-        if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
-        tc_fence_after_sync();
-        // ================= U epilogue: U^T rows -> bf16 [j][64 t] =================
-        {
-            float u[32];
-            tmem_ld32(tm_lane + TM_U + colhalf * 32, u);
-#pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) {
-                float f[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
-            }
-        }
-        mma_sync_point();
-        // ================= O^T += U^T P^T ;  S += K~^T U =================
-        if (tid == 0) {
-            const uint32_t idO = idesc_bf16(128, 64, false, false);
-            const uint32_t idS = idesc_bf16(128, 128, true, false);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t au = sdesc_sw128(sbase + OFF_R0 + ks * 32, 16, 1024);
-                const uint64_t bp = sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024);
-                mma_bf16(tm + TM_O, au, bp, idO, 1);
-                const uint64_t ak = sdesc_sw128(sbase + OFF_KT + ks * 2048, 8192, 1024);
-                mma_bf16(tm + TM_S, ak, au, idS, 1);
+                const uint64_t ak = sdesc_sw128(slot + SLOT_KT + ks * 2048, 8192, 1024);
+                const uint64_t uu = sdesc_sw128(slot + SLOT_U + ks * 32, 16, 1024);
+                mma_bf16(tm + SC_S, ak, uu, idK, 1);
+                const uint64_t bp = sdesc_sw128(slot + SLOT_P + ks * 32, 16, 1024);
+                mma_bf16(tm + SC_OT, uu, bp, idO2, 1);
             }
             mma_commit(&ms.bar_mma);
         }
+        if (tid == 0) bulk_wait_group_read0();  // the previous O tile has left shared memory
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // ================= O epilogue: O^T rows -> bf16 tile [t][j] -> one TMA store =================
+        if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
+        // ---- O^T rows -> bf16 tile [t][j] -> one TMA store (rows past T are clipped) ----
         {
             float ov[32];
-            tmem_ld32(tm_lane + TM_O + colhalf * 32, ov);
-            __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_R0);
+            tmem_ld32(tm_lane + SC_OT + colhalf * 32, ov);
+            __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
 #pragma unroll
             for (int i = 0; i < 32; ++i) ot[(colhalf * 32 + i) * DV + row] = __float2bfloat16_rn(ov[i]);
         }
@@ -686,18 +843,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before_sync();
         __syncthreads();
         if (tid == 0) {
-            tma_store_4d(&tm_o, sm + OFF_R0, 0, h, t0, bb);  // rows beyond T are clipped
+            tma_store_4d(&tm_o, sm + SC_O, 0, h, n * C, bb);
             bulk_commit_group();
         }
-        (void)Cn;
     }
-
     if (!timed_out && p.S_T) {
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
             const int j0 = colhalf * 64 + q2 * 32;
             float sv[32];
-            tmem_ld32(tm_lane + TM_S + j0, sv);
+            tmem_ld32(tm_lane + SC_S + j0, sv);
             float *dst = p.S_T + ((size_t)bh * DK + row) * DV + j0;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -708,7 +863,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, TM_COLS);
+    if (warp == 0) tmem_dealloc(tm, SC_COLS);
 }
 
 // ---------------------------------------------------------------- host side
@@ -756,6 +911,12 @@ bool forward_tc_supported(const FwdArgs &a)
     return a.bf16 && a.dk == DK && a.dv == DV && a.T > 0 && encode_fn() != nullptr;
 }
 
+size_t forward_tc_workspace_bytes(int B, int T, int H)
+{
+    const size_t ntasks = (size_t)B * H * ((T + C - 1) / C);
+    return ntasks * (SLOT_BYTES + GAMMA_BYTES);
+}
+
 cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
 {
     CUtensorMap mq, mk, mb, mv, mw, mla, mo;
@@ -764,10 +925,22 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
         !make_map(&mw, a.w, false, a.B, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK) ||
         !make_map(&mo, a.o, false, a.B, a.T, a.H, DV))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    TcParams p{a.B, a.T, a.H, a.S0, a.S_T, a.saved_states, a.status};
-    fwd_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, mo, p);
+    e = cudaFuncSetAttribute(fwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int NC = (a.T + C - 1) / C;
+    const int ntasks = a.B * a.H * NC;
+    ChunkParams cp{a.B, a.T, a.H, NC, ntasks, static_cast<unsigned char *>(a.workspace), a.status};
+    fwd_chunk_kernel<<<ntasks < nsm ? ntasks : nsm, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ScanParams sp{a.B, a.T, a.H, NC, ntasks, static_cast<const unsigned char *>(a.workspace), a.S0, a.S_T,
+                  a.saved_states, a.status};
+    fwd_scan_kernel<<<a.B * a.H, NT, SC_SMEM_BYTES, s>>>(mo, sp);
     return cudaGetLastError();
 }
 

@@ -100,9 +100,17 @@ int gdr2_abi_version(void) { return GDR2_ABI_VERSION; }
 
 const char *gdr2_last_error(void) { return g_last_error; }
 
+size_t gdr2_forward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt)
+{
+    if (B < 0 || T < 0 || H < 0) return 0;
+    if (dt != GDR2_BF16 || dk != 128 || dv != 128) return 0;
+    return gdr2::forward_tc_workspace_bytes(B, T, H);
+}
+
 gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
                          const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
-                         void *o, float *S_T, float *saved_states, void *stream)
+                         void *o, float *S_T, float *saved_states, void *workspace, size_t workspace_bytes,
+                         void *stream)
 {
     GDR2_TRY(check_dims(B, T, H, dk, dv));
     GDR2_TRY(check_dtype(dt));
@@ -129,7 +137,16 @@ gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, con
         }
         return GDR2_OK;
     }
-    gdr2::FwdArgs a{B, T, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S0, o, S_T, saved_states, nullptr};
+    const size_t need = gdr2_forward_workspace_bytes(B, T, H, dk, dv, dt);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(GDR2_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes,
+                        need);
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    }
+    gdr2::FwdArgs a{B,  T,    H,  dk,  dv,           dt == GDR2_BF16, q,         k,               v,      log_alpha,
+                    b,  w,    S0, o,   S_T,          saved_states,    workspace, workspace_bytes, nullptr};
     GDR2_TRY(device_status(&a.status));
     if (gdr2::forward_tc_supported(a)) return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward (tcgen05)");
     return launched(gdr2::launch_forward_simt(a, s), "gdr2_forward (simt)");

@@ -16,7 +16,7 @@ import argparse
 import torch
 
 from . import inputs as I
-from .binding import gdr2_backward, gdr2_decode_step, gdr2_forward, gdr2_sync_status
+from .binding import gdr2_backward, gdr2_decode_step, gdr2_forward, gdr2_forward_workspace_bytes, gdr2_sync_status
 
 
 def main():
@@ -26,10 +26,13 @@ def main():
     args = ap.parse_args()
     torch.cuda.set_device(0)
     if args.kernel == "fwd":
-        x = I.make_forward_inputs(**I.FWD_1P3B_BF16).to("cuda")
+        c = I.FWD_1P3B_BF16
+        x = I.make_forward_inputs(**c).to("cuda")
         o = torch.empty_like(x.v)
+        ws = torch.empty(gdr2_forward_workspace_bytes(c["B"], c["T"], c["H"], c["dk"], c["dv"], c["dtype"]),
+                         dtype=torch.uint8, device="cuda")
         for _ in range(args.launches):
-            gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o)
+            gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o, workspace=ws)
     elif args.kernel == "decode":
         c = I.DECODE_1P3B
         gen = torch.Generator(device="cuda").manual_seed(c["seed"])

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 1
+#define GDR2_ABI_VERSION 2
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -83,6 +83,10 @@ int gdr2_abi_version(void);
  * the same thread. */
 const char *gdr2_last_error(void);
 
+/* Bytes of device scratch gdr2_forward needs for this problem (0 when the
+ * call runs on CUDA cores: fp32 inputs, or dk/dv other than 128). */
+size_t gdr2_forward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt);
+
 /*
  * gdr2_forward -- chunkwise forward over whole sequences (prefill/training).
  *   Computes o_t for every token and the final state S_T, starting from S0.
@@ -97,13 +101,17 @@ const char *gdr2_last_error(void);
  * out: o [B,T,H,dv] dt; S_T [B,H,dk,dv] fp32 or NULL (not written);
  *      saved_states [B,H,ceil(T/64),dk,dv] fp32 or NULL: the state entering
  *      each chunk (chunk 0 receives S0), for gdr2_backward.
+ * scratch: workspace of at least gdr2_forward_workspace_bytes(...) bytes,
+ *      256-byte aligned (may be NULL when that size is 0); contents on entry
+ *      do not matter. The bf16 path at d = 128 keeps each chunk's
+ *      state-independent intermediates there (88.5 KiB per (b, h, chunk)).
  * Input and output buffers must not overlap (S0 == S_T is allowed).
  */
 gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
                          const void *q, const void *k, const void *v,
                          const float *log_alpha, const void *b, const void *w,
                          const float *S0, void *o, float *S_T, float *saved_states,
-                         void *stream);
+                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * gdr2_decode_step -- one recurrent token for N*H resident states

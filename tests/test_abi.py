@@ -37,10 +37,10 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 1
+    assert lib.gdr2_abi_version() == 2
 
 
-NULL11 = [None] * 11
+NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
 
 
 @pytest.mark.parametrize("dims,dt,status", [
@@ -60,7 +60,7 @@ def test_forward_rejects_bad_arguments(lib, dims, dt, status):
 def test_forward_rejects_misaligned_pointer(lib):
     p = [ctypes.c_void_p(0x10000)] * 11
     p[2] = ctypes.c_void_p(0x10008)  # v
-    assert lib.gdr2_forward(1, 4, 1, 64, 64, 1, *p) == binding.GDR2_ERR_INVALID_ARG
+    assert lib.gdr2_forward(1, 4, 1, 64, 64, 1, *p, ctypes.c_size_t(0), None) == binding.GDR2_ERR_INVALID_ARG
     assert b"v is not 16-byte aligned" in lib.gdr2_last_error()
 
 
@@ -103,3 +103,14 @@ def test_noalloc_backward_rejects_oversized_problems_on_the_host(lib):
     st = lib.gdr2_backward_noalloc(4, 4096, 16, 128, 128, 1, *p)
     assert st == binding.GDR2_ERR_UNSUPPORTED
     assert b"GDR2_NOALLOC_SCRATCH_BYTES" in lib.gdr2_last_error()
+
+
+def test_forward_workspace_query_and_check(lib):
+    # bf16 at d = 128 runs on the tensor cores and needs the chunk workspace
+    n = lib.gdr2_forward_workspace_bytes(4, 4096, 16, 128, 128, 1)
+    assert n == 4 * 16 * 64 * (90112 + 512)
+    assert lib.gdr2_forward_workspace_bytes(4, 4096, 16, 128, 128, 0) == 0  # fp32: CUDA cores
+    assert lib.gdr2_forward_workspace_bytes(4, 4096, 16, 64, 64, 1) == 0
+    p = [ctypes.c_void_p(0x10000)] * 11  # 10 tensors + the workspace
+    st = lib.gdr2_forward(1, 100, 1, 128, 128, 1, *p, ctypes.c_size_t(1024), None)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
