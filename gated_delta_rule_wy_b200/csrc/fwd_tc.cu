@@ -78,7 +78,7 @@ constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 12
 constexpr uint32_t OFF_R0 = 147456;     // R_0 32 x 128
 constexpr uint32_t OFF_R1 = 155648;     // R_1 64 x 128; U (128 x 64) over R0..R1, then the O tile
 constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later W^T
-constexpr uint32_t OFF_QH = 188416;     // Q (.) exp G, 64 x 128
+constexpr uint32_t OFF_QH = 188416;     // Q (.) exp G, transposed [c rows][64 t] (see qt_off)
 constexpr uint32_t OFF_KT = 204800;     // K (.) exp(G_C - G), 64 x 128
 constexpr uint32_t OFF_P = 221184;      // prefix-scan scratch during prep; then P 64 x 64
 constexpr uint32_t OFF_MISC = 229376;   // barriers, per-channel vectors
@@ -103,19 +103,29 @@ struct Misc {
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 
-// Byte offset of element (row, col) in a 128-byte-swizzled tile whose rows
-// are 64 bf16 wide; tiles of 128 columns are two such blocks of `rows` rows.
-__device__ __forceinline__ uint32_t sw_off(int row, int col, int rows)
-{
-    const int blk = col >> 6, cc = col & 63;
-    return (uint32_t)(blk * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + ((cc & 7) << 1));
-}
-
 // Offset of the 16-byte chunk holding columns [8*o8, 8*o8 + 8) of `row`.
 __device__ __forceinline__ uint32_t sw_chunk(int row, int o8, int rows)
 {
     const int blk = o8 >> 3, ch = o8 & 7;
     return (uint32_t)(blk * rows * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
+}
+
+// Byte offset of (c, t) in the transposed Q (.) exp G buffer: rows of 64 t
+// (128 bytes), 16-byte chunks permuted by both c % 8 and (c / 8) % 8, so the
+// prep (8 channels apart per lane) and the epilogue (one row per lane) are both
+// free of bank conflicts.
+__device__ __forceinline__ uint32_t qt_off(int c, int t)
+{
+    return (uint32_t)(c * 128 + ((((t >> 3) ^ (c & 7) ^ ((c >> 3) & 7))) << 4) + ((t & 7) << 1));
+}
+
+__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d)
+{
+    uint2 u;
+    __nv_bfloat162 h;
+    h = __floats2bfloat162_rn(a, b); u.x = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2bfloat162_rn(c, d); u.y = *reinterpret_cast<uint32_t *>(&h);
+    return u;
 }
 
 __device__ __forceinline__ uint4 pack8(const float (&f)[8])
@@ -301,7 +311,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             const __nv_bfloat16 *vs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_V);
             const __nv_bfloat16 *ws = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_W);
-            float egI[8], kcf[8], r10[8], gr[8];
+            float egI[8], kcf[8], r10[8], gr[8], qh4[8][4];
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
                 gr[x] = HI ? g1[x] : g0[x];
@@ -344,9 +354,14 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(t, o8, 64)) = pack8(r);
                 }
                 *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
-                *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
                 *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
             }
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+                *reinterpret_cast<uint2 *>(sm + OFF_QH + qt_off(o8 * 8 + x, tg * 4)) =
+                    pack4(qh4[x][0], qh4[x][1], qh4[x][2], qh4[x][3]);
         }
         const bool exact = __syncthreads_or(risky) != 0;
         if (exact) {
@@ -359,6 +374,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             // operands with one exponential of a non-positive argument each
+            float qh4[8][4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int t = tg * 4 + m;
@@ -376,8 +392,13 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int tl = t - 32 * HI;
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
                 *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
-                *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
             }
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+                *reinterpret_cast<uint2 *>(sm + OFF_QH + qt_off(o8 * 8 + x, tg * 4)) =
+                    pack4(qh4[x][0], qh4[x][1], qh4[x][2], qh4[x][3]);
             if (tid < DK) ms.eg0[tid] = ms.eg1[tid] = 1.f;
             // A and P rows: thread -> row t = tid / 4, columns 16*(tid % 4) .. +15
             {
@@ -500,53 +521,77 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
         // ================= UT solve: T = (I + A)^{-1} by 16 x 16 blocks =================
         // Diagonal blocks D_I = (I + A_II)^{-1} by forward substitution (one column per
-        // thread), then block rows I = 1..3: T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ.
+        // thread), then block rows I = 1..3: T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ, each
+        // thread producing one row x 4 columns from 16-byte operand loads.
         if (tid < 64) {
             const int I = tid >> 4, sl = tid & 15;
             const float *Ab = A32 + (16 * I) * F_LD + 16 * I;
             float col[16];
 #pragma unroll
             for (int tl = 0; tl < 16; ++tl) {
+                float arow[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (4 * q < tl) {
+                        const float4 v = *reinterpret_cast<const float4 *>(Ab + tl * F_LD + 4 * q);
+                        arow[4 * q] = v.x; arow[4 * q + 1] = v.y; arow[4 * q + 2] = v.z; arow[4 * q + 3] = v.w;
+                    }
+                }
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                 for (int il = 0; il < tl; ++il) {
-                    if (il & 1) a1 = fmaf(Ab[tl * F_LD + il], col[il], a1);
-                    else a0 = fmaf(Ab[tl * F_LD + il], col[il], a0);
+                    if (il & 1) a1 = fmaf(arow[il], col[il], a1);
+                    else a0 = fmaf(arow[il], col[il], a0);
                 }
                 col[tl] = (tl < sl) ? 0.f : (tl == sl ? 1.f : -(a0 + a1));
             }
 #pragma unroll
             for (int tl = 0; tl < 16; ++tl) T32[(16 * I + tl) * F_LD + 16 * I + sl] = col[tl];
         } else {
-            for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
-                const int r = idx >> 6, cc = idx & 63;
-                if ((cc >> 4) != (r >> 4)) T32[r * F_LD + cc] = 0.f;
+            // zero the blocks above the diagonal: 6 blocks x 16 rows x 4 quads
+            for (int idx = tid - 64; idx < 6 * 64; idx += NT - 64) {
+                const int blk = idx >> 6, r = (idx >> 2) & 15, q = idx & 3;
+                const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                *reinterpret_cast<float4 *>(T32 + (16 * I + r) * F_LD + 16 * J + 4 * q) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         __syncthreads();
 #pragma unroll
         for (int I = 1; I < 4; ++I) {
-            for (int idx = tid; idx < I * 256; idx += NT) {
-                const int J = idx >> 8, r = (idx >> 4) & 15, s = idx & 15;
+            const int J = tid >> 6, r = (tid >> 2) & 15, cs = 16 * J + 4 * (tid & 3);
+            if (tid < 64 * I) {  // Y_J = sum_{u in [16J, 16I)} A[16I + r][u] T[u][cs .. cs+3]
                 const float *Ar = A32 + (16 * I + r) * F_LD;
-                float acc0 = 0.f, acc1 = 0.f;
-                for (int u = 16 * J; u < 16 * I; u += 2) {
-                    acc0 = fmaf(Ar[u], T32[u * F_LD + 16 * J + s], acc0);
-                    acc1 = fmaf(Ar[u + 1], T32[(u + 1) * F_LD + 16 * J + s], acc1);
+                float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll 4
+                for (int u = 16 * J; u < 16 * I; u += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
+                    const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float4 tv = *reinterpret_cast<const float4 *>(T32 + (u + k) * F_LD + cs);
+                        y0 = fmaf(av[k], tv.x, y0); y1 = fmaf(av[k], tv.y, y1);
+                        y2 = fmaf(av[k], tv.z, y2); y3 = fmaf(av[k], tv.w, y3);
+                    }
                 }
-                Ys[r * Y_LD + 16 * J + s] = acc0 + acc1;
+                *reinterpret_cast<float4 *>(Ys + r * Y_LD + cs) = make_float4(y0, y1, y2, y3);
             }
             __syncthreads();
-            for (int idx = tid; idx < I * 256; idx += NT) {
-                const int J = idx >> 8, r = (idx >> 4) & 15, s = idx & 15;
+            if (tid < 64 * I) {  // T_IJ = -D_I Y_J
                 const float *Dr = T32 + (16 * I + r) * F_LD + 16 * I;
-                float acc0 = 0.f, acc1 = 0.f;
+                float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
 #pragma unroll
-                for (int u = 0; u < 16; u += 2) {
-                    acc0 = fmaf(Dr[u], Ys[u * Y_LD + 16 * J + s], acc0);
-                    acc1 = fmaf(Dr[u + 1], Ys[(u + 1) * Y_LD + 16 * J + s], acc1);
+                for (int u = 0; u < 16; u += 4) {
+                    const float4 d = *reinterpret_cast<const float4 *>(Dr + u);
+                    const float dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float4 yv = *reinterpret_cast<const float4 *>(Ys + (u + k) * Y_LD + cs);
+                        y0 = fmaf(dv[k], yv.x, y0); y1 = fmaf(dv[k], yv.y, y1);
+                        y2 = fmaf(dv[k], yv.z, y2); y3 = fmaf(dv[k], yv.w, y3);
+                    }
                 }
-                T32[(16 * I + r) * F_LD + 16 * J + s] = -(acc0 + acc1);
+                *reinterpret_cast<float4 *>(T32 + (16 * I + r) * F_LD + cs) = make_float4(-y0, -y1, -y2, -y3);
             }
             __syncthreads();
         }
@@ -629,16 +674,12 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int c = row;
             float d[32];
             tmem_ld32(tm_lane + CK_Q + colhalf * 32, d);
-            const unsigned char *qh = sm + OFF_QH;
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
                 float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QH + qt_off(c, colhalf * 32 + k8 * 8)), f);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const int t = colhalf * 32 + k8 * 8 + x;
-                    f[x] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qh + sw_off(t, c, 64))) +
-                           d[k8 * 8 + x];
-                }
+                for (int x = 0; x < 8; ++x) f[x] += d[k8 * 8 + x];
                 *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
             }
 #pragma unroll
@@ -683,7 +724,7 @@ constexpr uint32_t SC_SB = 2 * SLOT_BYTES;         // S^T bf16 [j block][c rows]
 constexpr uint32_t SC_O = SC_SB + 32768;           // O tile [64 t][128 j] bf16
 constexpr uint32_t SC_MISC = SC_O + 16384;
 constexpr uint32_t SC_SMEM_BYTES = SC_MISC + 1280 + 1024;
-constexpr uint32_t SC_S = 0, SC_OT = 128, SC_COLS = 256;
+constexpr uint32_t SC_S = 0, SC_OT = 128, SC_COLS = 256;  // O^T double-buffered: SC_OT + 64 * (n & 1)
 
 struct ScanMisc {
     uint64_t bar_full[2];
@@ -768,6 +809,24 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         return __syncthreads_or(!ok) == 0;
     };
 
+    // O^T of chunk m -> bf16 tile [t][j] -> one TMA store (rows past T are clipped)
+    auto store_o = [&](int m) {
+        if (tid == 0) bulk_wait_group_read0();  // the previous tile has left shared memory
+        __syncthreads();
+        float ov[32];
+        tmem_ld32(tm_lane + SC_OT + 64 * (m & 1) + colhalf * 32, ov);
+        __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ot[(colhalf * 32 + i) * DV + row] = __float2bfloat16_rn(ov[i]);
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_o, sm + SC_O, 0, h, m * C, bb);
+            bulk_commit_group();
+        }
+    };
+
     for (int n = 0; n < NC; ++n) {
         const int sl = n & 1;
         const uint32_t slot = sbase + (sl ? SC_SLOT1 : SC_SLOT0);
@@ -809,13 +868,14 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
             const uint32_t idK = idesc_bf16(128, 128, true, false);
             const uint32_t idO1 = idesc_bf16(128, 64, true, true);
             const uint32_t idO2 = idesc_bf16(128, 64, false, false);
+            const uint32_t d_o = tm + SC_OT + 64 * sl;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t am = sdesc_sw128(slot + SLOT_M + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                 const uint64_t bs = sdesc_sw128(sbase + SC_SB + ks * 2048, 16384, 1024);
                 mma_bf16(tm + SC_S, am, bs, idM, 1);
                 const uint64_t bq = sdesc_sw128(slot + SLOT_Q + ks * 2048, 8192, 1024);
-                mma_bf16(tm + SC_OT, bs, bq, idO1, ks > 0);
+                mma_bf16(d_o, bs, bq, idO1, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
@@ -823,30 +883,16 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
                 const uint64_t uu = sdesc_sw128(slot + SLOT_U + ks * 32, 16, 1024);
                 mma_bf16(tm + SC_S, ak, uu, idK, 1);
                 const uint64_t bp = sdesc_sw128(slot + SLOT_P + ks * 32, 16, 1024);
-                mma_bf16(tm + SC_OT, uu, bp, idO2, 1);
+                mma_bf16(d_o, uu, bp, idO2, 1);
             }
             mma_commit(&ms.bar_mma);
         }
-        if (tid == 0) bulk_wait_group_read0();  // the previous O tile has left shared memory
+        if (n > 0) store_o(n - 1);  // overlaps this chunk's MMAs (other TMEM columns)
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
         if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
-        // ---- O^T rows -> bf16 tile [t][j] -> one TMA store (rows past T are clipped) ----
-        {
-            float ov[32];
-            tmem_ld32(tm_lane + SC_OT + colhalf * 32, ov);
-            __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ot[(colhalf * 32 + i) * DV + row] = __float2bfloat16_rn(ov[i]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_4d(&tm_o, sm + SC_O, 0, h, n * C, bb);
-            bulk_commit_group();
-        }
     }
+    if (!timed_out && NC > 0) store_o(NC - 1);
     if (!timed_out && p.S_T) {
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
