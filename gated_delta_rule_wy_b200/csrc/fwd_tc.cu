@@ -68,26 +68,28 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kFactorLimit = 80.f;              // |exponent| of one decay factor
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ----
-constexpr uint32_t OFF_STG_Q = 0;       // q  [64][128] bf16; later T (bf16 [64][64], swizzled)
-constexpr uint32_t OFF_STG_K = 16384;   // k; later T (fp32 [64][68]) over K and B
-constexpr uint32_t OFF_STG_B = 32768;   // b; later (from +2048) the block-product scratch
-constexpr uint32_t OFF_STG_V = 49152;   // v; later A (fp32 [64][68]) over V and W
+constexpr uint32_t OFF_STG_Q = 0;       // q  [64][128] bf16
+constexpr uint32_t OFF_STG_K = 16384;   // k
+constexpr uint32_t OFF_STG_B = 32768;   // b
+constexpr uint32_t OFF_STG_V = 49152;   // v; exact path: A (fp32 [64][68]) over V and W
 constexpr uint32_t OFF_STG_W = 65536;   // w
 constexpr uint32_t OFF_STG_LA = 81920;  // log_alpha [64][128] fp32; then per-channel references; exact path: G
-constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128; later S^T
+constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128
 constexpr uint32_t OFF_R0 = 147456;     // R_0 32 x 128
-constexpr uint32_t OFF_R1 = 155648;     // R_1 64 x 128; U (128 x 64) over R0..R1, then the O tile
-constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later W^T
+constexpr uint32_t OFF_R1 = 155648;     // R_1 64 x 128; then over R0..R1: A and T (fp32 [64][68]) with the
+                                        // block-product scratch, then T (bf16 [64][64])
+constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later W as [c][64 t]
 constexpr uint32_t OFF_QH = 188416;     // Q (.) exp G, transposed [c rows][64 t] (see qt_off)
 constexpr uint32_t OFF_KT = 204800;     // K (.) exp(G_C - G), 64 x 128
 constexpr uint32_t OFF_P = 221184;      // prefix-scan scratch during prep; then P 64 x 64
 constexpr uint32_t OFF_MISC = 229376;   // barriers, per-channel vectors
 constexpr uint32_t MISC_BYTES = 1664;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-constexpr int F_LD = 68;                // fp32 row stride of the A and T scratch
-constexpr uint32_t OFF_T32 = OFF_STG_K;
-constexpr uint32_t OFF_Y = OFF_STG_B + 2048;  // 16 x (3*16 + 4) fp32
-constexpr int Y_LD = 52;
+constexpr int F_LD = 68;                // fp32 row stride of the A / T scratch
+constexpr uint32_t OFF_A32 = OFF_R0;     // A, solved in place into T
+constexpr uint32_t OFF_Y = OFF_R0 + 64 * F_LD * 4;  // block-product scratch, 32 x 36 fp32
+constexpr int Y_LD = 36;
+constexpr uint32_t OFF_TB = OFF_R0;      // T in bf16, K-major [t][64 s]
 constexpr uint32_t TX_BYTES = 5 * 16384 + 32768;
 
 constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
@@ -245,14 +247,14 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int o8 = tid & 15;
     const int tg = tid >> 4;
     const int HI = tg >> 3;  // half-chunk of this thread's tokens
-    float *A32 = reinterpret_cast<float *>(sm + OFF_STG_V);
-    float *T32 = reinterpret_cast<float *>(sm + OFF_T32);
+    float *A32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
     for (int task = blockIdx.x; task < p.ntasks && !timed_out; task += gridDim.x) {
         const int n = task % NC;
         const int Cn = min(C, p.T - n * C);
-        if (tid == 0) bulk_wait_group_read0();  // the previous task's outputs have left shared memory
+        // this task's workspace slot: the threads store their parts of it directly
+        unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
@@ -353,7 +355,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 } else {
                     *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(t, o8, 64)) = pack8(r);
                 }
-                *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
+                {
+                    const uint4 v = pack8(kt);
+                    *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = v;
+                    *reinterpret_cast<uint4 *>(slot + SLOT_KT + sw_chunk(t, o8, 64)) = v;
+                }
                 *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
@@ -364,6 +370,8 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     pack4(qh4[x][0], qh4[x][1], qh4[x][2], qh4[x][3]);
         }
         const bool exact = __syncthreads_or(risky) != 0;
+        // the staging buffers are free once the operands are built: prefetch the next task
+        if (!exact && tid == 0 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
         if (exact) {
             // ---- exact path: G to shared memory, pairwise exponentials ----
             float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
@@ -391,7 +399,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 const int tl = t - 32 * HI;
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
-                *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
+                {
+                    const uint4 v = pack8(kt);
+                    *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = v;
+                    *reinterpret_cast<uint4 *>(slot + SLOT_KT + sw_chunk(t, o8, 64)) = v;
+                }
 #pragma unroll
                 for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
             }
@@ -436,10 +448,15 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const int i = i0 + k8 * 8 + x;
                         pr[x] = (i <= t) ? accP[k8 * 8 + x] : 0.f;
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, (i0 >> 3) + k8, 64)) = pack8(pr);
+                    {
+                        const uint4 v = pack8(pr);
+                        *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, (i0 >> 3) + k8, 64)) = v;
+                        *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, (i0 >> 3) + k8, 64)) = v;
+                    }
                 }
             }
             __syncthreads();
+            if (tid == 0 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
         } else {
             // ---- tensor-core path: [A;P] = STACK R_I^T ----
             mma_sync_point();
@@ -479,7 +496,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             float pr[8];
 #pragma unroll
                             for (int x = 0; x < 8; ++x) pr[x] = (k8 * 8 + x <= t) ? v[k8 * 8 + x] : 0.f;
-                            *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = pack8(pr);
+                            {
+                                const uint4 v = pack8(pr);
+                                *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = v;
+                                *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, k8, 64)) = v;
+                            }
                         }
                     }
                 } else {
@@ -492,7 +513,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const float zz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int k8 = 4; k8 < 8; ++k8)
-                            *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = pack8(zz);
+                            {
+                                const uint4 v = pack8(zz);
+                                *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = v;
+                                *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, k8, 64)) = v;
+                            }
                     }
                 }
             } else {
@@ -511,7 +536,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         float pr[8];
 #pragma unroll
                         for (int x = 0; x < 8; ++x) pr[x] = (ib + k8 * 8 + x <= t) ? v[k8 * 8 + x] : 0.f;
-                        *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, colhalf * 4 + k8, 64)) = pack8(pr);
+                        {
+                            const uint4 v = pack8(pr);
+                            *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, colhalf * 4 + k8, 64)) = v;
+                            *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, colhalf * 4 + k8, 64)) = v;
+                        }
                     }
                 }
             }
@@ -519,90 +548,126 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncthreads();
         }
 
-        // ================= UT solve: T = (I + A)^{-1} by 16 x 16 blocks =================
-        // Diagonal blocks D_I = (I + A_II)^{-1} by forward substitution (one column per
-        // thread), then block rows I = 1..3: T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ, each
-        // thread producing one row x 4 columns from 16-byte operand loads.
-        if (tid < 64) {
-            const int I = tid >> 4, sl = tid & 15;
-            const float *Ab = A32 + (16 * I) * F_LD + 16 * I;
+        // ================= UT solve: T = (I + A)^{-1}, in place =================
+        // D_I = (I + A_II)^{-1} for the four 16 x 16 diagonal blocks (forward substitution,
+        // one column per thread); then two doubling levels, each of the form
+        //   [[X, 0], [Y, Z]]^{-1} = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
+        // at 32 and at 64 rows. Every thread produces one row x four columns from
+        // 16-byte operand loads. A holds zeros on and above the diagonal, so the
+        // finished array is T with its zero upper triangle.
+        {
             float col[16];
+            const int I = (tid >> 4) & 3, sl = tid & 15;
+            float *Ab = A32 + (16 * I) * F_LD + 16 * I;
+            if (tid < 64) {
 #pragma unroll
-            for (int tl = 0; tl < 16; ++tl) {
-                float arow[16];
+                for (int tl = 0; tl < 16; ++tl) {
+                    float arow[16];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (4 * q < tl) {
-                        const float4 v = *reinterpret_cast<const float4 *>(Ab + tl * F_LD + 4 * q);
-                        arow[4 * q] = v.x; arow[4 * q + 1] = v.y; arow[4 * q + 2] = v.z; arow[4 * q + 3] = v.w;
+                    for (int q = 0; q < 4; ++q) {
+                        if (4 * q < tl) {
+                            const float4 v = *reinterpret_cast<const float4 *>(Ab + tl * F_LD + 4 * q);
+                            arow[4 * q] = v.x; arow[4 * q + 1] = v.y; arow[4 * q + 2] = v.z; arow[4 * q + 3] = v.w;
+                        }
                     }
-                }
-                float a0 = 0.f, a1 = 0.f;
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                for (int il = 0; il < tl; ++il) {
-                    if (il & 1) a1 = fmaf(arow[il], col[il], a1);
-                    else a0 = fmaf(arow[il], col[il], a0);
+                    for (int il = 0; il < tl; ++il) {
+                        if ((il & 3) == 0) a0 = fmaf(arow[il], col[il], a0);
+                        else if ((il & 3) == 1) a1 = fmaf(arow[il], col[il], a1);
+                        else if ((il & 3) == 2) a2 = fmaf(arow[il], col[il], a2);
+                        else a3 = fmaf(arow[il], col[il], a3);
+                    }
+                    col[tl] = (tl < sl) ? 0.f : (tl == sl ? 1.f : -((a0 + a1) + (a2 + a3)));
                 }
-                col[tl] = (tl < sl) ? 0.f : (tl == sl ? 1.f : -(a0 + a1));
             }
+            __syncthreads();
+            if (tid < 64) {
 #pragma unroll
-            for (int tl = 0; tl < 16; ++tl) T32[(16 * I + tl) * F_LD + 16 * I + sl] = col[tl];
-        } else {
-            // zero the blocks above the diagonal: 6 blocks x 16 rows x 4 quads
-            for (int idx = tid - 64; idx < 6 * 64; idx += NT - 64) {
-                const int blk = idx >> 6, r = (idx >> 2) & 15, q = idx & 3;
-                const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                const int J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                *reinterpret_cast<float4 *>(T32 + (16 * I + r) * F_LD + 16 * J + 4 * q) = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int tl = 0; tl < 16; ++tl) Ab[tl * F_LD + sl] = col[tl];
             }
+            __syncthreads();
         }
-        __syncthreads();
-#pragma unroll
-        for (int I = 1; I < 4; ++I) {
-            const int J = tid >> 6, r = (tid >> 2) & 15, cs = 16 * J + 4 * (tid & 3);
-            if (tid < 64 * I) {  // Y_J = sum_{u in [16J, 16I)} A[16I + r][u] T[u][cs .. cs+3]
-                const float *Ar = A32 + (16 * I + r) * F_LD;
-                float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        // one row x four columns of  Y = A[r0+r][c0 .. c0+n) . A[c0 .. c0+n)[k0+cs .. +3]
+        auto row_times_block = [&](int arow, int acol, int brow, int bcol, int n, float (&y)[4]) {
+            const float *Ar = A32 + arow * F_LD + acol;
+            y[0] = y[1] = y[2] = y[3] = 0.f;
 #pragma unroll 4
-                for (int u = 16 * J; u < 16 * I; u += 4) {
+            for (int u = 0; u < n; u += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
+                const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 tv = *reinterpret_cast<const float4 *>(A32 + (brow + u + k) * F_LD + bcol);
+                    y[0] = fmaf(av[k], tv.x, y[0]); y[1] = fmaf(av[k], tv.y, y[1]);
+                    y[2] = fmaf(av[k], tv.z, y[2]); y[3] = fmaf(av[k], tv.w, y[3]);
+                }
+            }
+        };
+        auto neg_row_times_y = [&](int arow, int acol, int n, int ycol, float (&y)[4]) {
+            const float *Ar = A32 + arow * F_LD + acol;
+            y[0] = y[1] = y[2] = y[3] = 0.f;
+#pragma unroll 4
+            for (int u = 0; u < n; u += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
+                const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 yv = *reinterpret_cast<const float4 *>(Ys + (u + k) * Y_LD + ycol);
+                    y[0] = fmaf(av[k], yv.x, y[0]); y[1] = fmaf(av[k], yv.y, y[1]);
+                    y[2] = fmaf(av[k], yv.z, y[2]); y[3] = fmaf(av[k], yv.w, y[3]);
+                }
+            }
+            y[0] = -y[0]; y[1] = -y[1]; y[2] = -y[2]; y[3] = -y[3];
+        };
+        // level 32: blocks b = 0, 1 (rows 32b .. 32b+31):  A[32b+16.., 32b..] <- -D_hi (A_lohi D_lo)
+        {
+            const int b = tid >> 6, r = (tid >> 2) & 15, cs = 4 * (tid & 3);
+            float y[4];
+            if (tid < 128) {
+                row_times_block(32 * b + 16 + r, 32 * b, 32 * b, 32 * b + cs, 16, y);
+                *reinterpret_cast<float4 *>(Ys + (16 * b + r) * Y_LD + cs) = make_float4(y[0], y[1], y[2], y[3]);
+            }
+            __syncthreads();
+            if (tid < 128) {
+                const float *Ar = A32 + (32 * b + 16 + r) * F_LD + 32 * b + 16;  // D_hi row
+                y[0] = y[1] = y[2] = y[3] = 0.f;
+#pragma unroll
+                for (int u = 0; u < 16; u += 4) {
                     const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
                     const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float4 tv = *reinterpret_cast<const float4 *>(T32 + (u + k) * F_LD + cs);
-                        y0 = fmaf(av[k], tv.x, y0); y1 = fmaf(av[k], tv.y, y1);
-                        y2 = fmaf(av[k], tv.z, y2); y3 = fmaf(av[k], tv.w, y3);
+                        const float4 yv = *reinterpret_cast<const float4 *>(Ys + (16 * b + u + k) * Y_LD + cs);
+                        y[0] = fmaf(av[k], yv.x, y[0]); y[1] = fmaf(av[k], yv.y, y[1]);
+                        y[2] = fmaf(av[k], yv.z, y[2]); y[3] = fmaf(av[k], yv.w, y[3]);
                     }
                 }
-                *reinterpret_cast<float4 *>(Ys + r * Y_LD + cs) = make_float4(y0, y1, y2, y3);
-            }
-            __syncthreads();
-            if (tid < 64 * I) {  // T_IJ = -D_I Y_J
-                const float *Dr = T32 + (16 * I + r) * F_LD + 16 * I;
-                float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-#pragma unroll
-                for (int u = 0; u < 16; u += 4) {
-                    const float4 d = *reinterpret_cast<const float4 *>(Dr + u);
-                    const float dv[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float4 yv = *reinterpret_cast<const float4 *>(Ys + (u + k) * Y_LD + cs);
-                        y0 = fmaf(dv[k], yv.x, y0); y1 = fmaf(dv[k], yv.y, y1);
-                        y2 = fmaf(dv[k], yv.z, y2); y3 = fmaf(dv[k], yv.w, y3);
-                    }
-                }
-                *reinterpret_cast<float4 *>(T32 + (16 * I + r) * F_LD + cs) = make_float4(-y0, -y1, -y2, -y3);
+                *reinterpret_cast<float4 *>(A32 + (32 * b + 16 + r) * F_LD + 32 * b + cs) =
+                    make_float4(-y[0], -y[1], -y[2], -y[3]);
             }
             __syncthreads();
         }
+        // level 64:  A[32.., 0..31] <- -T_1 (A_10 T_0)
+        {
+            const int r = tid >> 3, cs = 4 * (tid & 7);
+            float y[4];
+            row_times_block(32 + r, 0, 0, cs, 32, y);
+            *reinterpret_cast<float4 *>(Ys + r * Y_LD + cs) = make_float4(y[0], y[1], y[2], y[3]);
+            __syncthreads();
+            neg_row_times_y(32 + r, 32, 32, cs, y);
+            *reinterpret_cast<float4 *>(A32 + (32 + r) * F_LD + cs) = make_float4(y[0], y[1], y[2], y[3]);
+            __syncthreads();
+        }
+        // T -> bf16, K-major [t][64 s], over the front of the same region
         {
             const int t = tid >> 2, k0 = (tid & 3) * 2;
-#pragma unroll
-            for (int k8 = k0; k8 < k0 + 2; ++k8) {
-                float f[8];
-                load8f(T32 + t * F_LD + k8 * 8, f);
-                *reinterpret_cast<uint4 *>(sm + OFF_STG_Q + sw_chunk(t, k8, 64)) = pack8(f);
-            }
+            float f0[8], f1[8];
+            load8f(A32 + t * F_LD + k0 * 8, f0);
+            load8f(A32 + t * F_LD + (k0 + 1) * 8, f1);
+            __syncthreads();
+            *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(t, k0, 64)) = pack8(f0);
+            *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(t, k0 + 1, 64)) = pack8(f1);
         }
         mma_sync_point();
         // ================= W^T_I = (L^e_I)^T T[:,I]^T ;  U~^T = Z^T T^T =================
@@ -613,28 +678,25 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
                     const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + (64 * I + 16 * ks) * 128, 16384, 1024);
-                    const uint64_t bd = sdesc_sw128(sbase + OFF_STG_Q + (32 * I + 16 * ks) * 2, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sbase + OFF_TB + (32 * I + 16 * ks) * 2, 16, 1024);
                     mma_bf16(tm + (I ? CK_W1 : CK_W0), ad, bd, idW, ks > 0);
                 }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = sdesc_sw128(sbase + OFF_Z + ks * 2048, 8192, 1024);
-                const uint64_t bd = sdesc_sw128(sbase + OFF_STG_Q + ks * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024);
                 mma_bf16(tm + CK_U, ad, bd, idW, ks > 0);
             }
             mma_commit(&ms.bar_mma);
         }
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // staging is free: prefetch the next task's inputs
-        if (tid == 0 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
 
-        // ================= W -> [c][64 t] over Z;  U~ -> [j][64 t] over R0..R1 =================
+        // ================= W -> [c][64 t] over Z;  U~ -> [j][64 t] straight to the slot =================
         {
             const float e0 = ms.eg0[row], e1 = ms.eg1[row];
             float w0[32], w1[32];
-            tmem_ld32(tm_lane + CK_W0 + colhalf * 32, w0);
-            tmem_ld32(tm_lane + CK_W1 + colhalf * 32, w1);
+            tmem_ld32x2(tm_lane + CK_W0 + colhalf * 32, tm_lane + CK_W1 + colhalf * 32, w0, w1);
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
                 float f[8];
@@ -649,7 +711,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float f[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
+                *reinterpret_cast<uint4 *>(slot + SLOT_U + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
             }
         }
         mma_sync_point();
@@ -669,46 +731,42 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // ================= Q' -> [c][64 t] over Z;  M -> [c' block][c][64 c'] over STACK =================
+        // ================= Q' -> [c][64 t] and M -> [c' block][c][64 c'], straight to the slot =================
         {
             const int c = row;
-            float d[32];
-            tmem_ld32(tm_lane + CK_Q + colhalf * 32, d);
+            float d[32], m0[32];
+            tmem_ld32x2(tm_lane + CK_Q + colhalf * 32, tm_lane + CK_M + colhalf * 64, d, m0);
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
                 float f[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QH + qt_off(c, colhalf * 32 + k8 * 8)), f);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) f[x] += d[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
+                *reinterpret_cast<uint4 *>(slot + SLOT_Q + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
             }
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int c0 = colhalf * 64 + q2 * 32;
                 float mv[32];
-                tmem_ld32(tm_lane + CK_M + c0, mv);
+                if (q2 == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mv[i] = m0[i];
+                } else {
+                    tmem_ld32(tm_lane + CK_M + c0, mv);
+                }
 #pragma unroll
                 for (int k8 = 0; k8 < 4; ++k8) {
                     float f[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) f[x] = mv[k8 * 8 + x];
-                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(c, (c0 >> 3) + k8, 128)) = pack8(f);
+                    *reinterpret_cast<uint4 *>(slot + SLOT_M + sw_chunk(c, (c0 >> 3) + k8, 128)) = pack8(f);
                 }
             }
         }
-        fence_proxy_async_smem();
+        if (tid < DK) reinterpret_cast<float *>(p.ws + (size_t)p.ntasks * SLOT_BYTES + (size_t)task * GAMMA_BYTES)[tid] =
+            ms.gC[tid];
         tc_fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
-            bulk_store(slot + SLOT_M, sm + OFF_STACK, 32768);
-            bulk_store(slot + SLOT_KT, sm + OFF_KT, 16384);
-            bulk_store(slot + SLOT_U, sm + OFF_R0, 16384);
-            bulk_store(slot + SLOT_Q, sm + OFF_Z, 16384);
-            bulk_store(slot + SLOT_P, sm + OFF_P, 8192);
-            bulk_store(p.ws + (size_t)p.ntasks * SLOT_BYTES + (size_t)task * GAMMA_BYTES, ms.gC, GAMMA_BYTES);
-            bulk_commit_group();
-        }
+        __syncthreads();  // every TMEM read of this task is done before the next task's MMAs
     }
     if (tid == 0) bulk_wait_group0();
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
@@ -809,18 +867,23 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         return __syncthreads_or(!ok) == 0;
     };
 
-    // O^T of chunk m -> bf16 tile [t][j] -> one TMA store (rows past T are clipped)
+    // O^T of chunk m -> bf16 tile [t][j] -> one TMA store (rows past T are clipped).
+    // Warps 0-3 only (thread = TMEM lane, all 64 columns), under named barrier 1, so
+    // they run while the MMA issuer in warp 4 is busy with the next chunk.
     auto store_o = [&](int m) {
         if (tid == 0) bulk_wait_group_read0();  // the previous tile has left shared memory
-        __syncthreads();
-        float ov[32];
-        tmem_ld32(tm_lane + SC_OT + 64 * (m & 1) + colhalf * 32, ov);
+        named_barrier(1, 128);
+        float o0[32], o1[32];
+        tmem_ld32x2(tm_lane + SC_OT + 64 * (m & 1), tm_lane + SC_OT + 64 * (m & 1) + 32, o0, o1);
         __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ot[(colhalf * 32 + i) * DV + row] = __float2bfloat16_rn(ov[i]);
+        for (int i = 0; i < 32; ++i) {
+            ot[i * DV + row] = __float2bfloat16_rn(o0[i]);
+            ot[(32 + i) * DV + row] = __float2bfloat16_rn(o1[i]);
+        }
         fence_proxy_async_smem();
         tc_fence_before_sync();
-        __syncthreads();
+        named_barrier(1, 128);
         if (tid == 0) {
             tma_store_4d(&tm_o, sm + SC_O, 0, h, m * C, bb);
             bulk_commit_group();
@@ -835,11 +898,12 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         {
             const int c = row;
             const float g = ms.gam[sl][c];
+            float s2[2][32];
+            tmem_ld32x2(tm_lane + SC_S + colhalf * 64, tm_lane + SC_S + colhalf * 64 + 32, s2[0], s2[1]);
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int j0 = colhalf * 64 + q2 * 32;
-                float sv[32];
-                tmem_ld32(tm_lane + SC_S + j0, sv);
+                float (&sv)[32] = s2[q2];
                 if (p.saved_states) {
                     float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c) * DV + j0;
 #pragma unroll
@@ -863,7 +927,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         __syncthreads();
         tc_fence_after_sync();
         // ---- S += M S_bf16 + K~^T U~ ;  O^T = S_bf16^T Q'^T + U~^T P^T ----
-        if (tid == 0) {
+        if (tid == 128) {
             const uint32_t idM = idesc_bf16(128, 128, false, true);
             const uint32_t idK = idesc_bf16(128, 128, true, false);
             const uint32_t idO1 = idesc_bf16(128, 64, true, true);
@@ -887,12 +951,12 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
             }
             mma_commit(&ms.bar_mma);
         }
-        if (n > 0) store_o(n - 1);  // overlaps this chunk's MMAs (other TMEM columns)
+        if (n > 0 && warp < 4) store_o(n - 1);  // overlaps this chunk's MMAs (other TMEM columns)
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
         if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
     }
-    if (!timed_out && NC > 0) store_o(NC - 1);
+    if (!timed_out && NC > 0 && warp < 4) store_o(NC - 1);
     if (!timed_out && p.S_T) {
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
