@@ -84,6 +84,15 @@ def shard_seed(base: int, rank: int) -> int:
     return base + 7 * rank
 
 
+def job_throughput(local_total_ms: float, steps: int, units_per_rank: int, world: int, device):
+    """Whole-job units/s: every rank's units over the slowest rank's time.
+
+    Returns (units per second, ms per step of the slowest rank)."""
+    total_ms = max_over_ranks(local_total_ms, world, device)
+    ms_per_step = total_ms / steps
+    return units_per_rank * world / (ms_per_step * 1e-3), ms_per_step
+
+
 # ----------------------------------------------------------------------------- measurement helpers
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -315,10 +324,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     gdr2_sync_status()
-    total_ms = max_over_ranks(sum(ms), world, dev)
-    ms_per_step = total_ms / args.steps
-    tokens = B * T * world
-    value = tokens / (ms_per_step * 1e-3)
+    tokens = B * T  # per rank
+    value, ms_per_step = job_throughput(sum(ms), args.steps, tokens, world, dev)
 
     # ---- end to end through the C ABI with host buffers ----
     pinned = [t.pin_memory() for t in (x_cpu.q, x_cpu.k, x_cpu.v, x_cpu.log_alpha, x_cpu.b, x_cpu.w)]
@@ -340,8 +347,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_steps = max(3, min(args.steps, 10))
     barrier(world)
-    e2e_ms = max_over_ranks(sum(time_steps(e2e_step, e2e_steps, stream)), world, dev) / e2e_steps
-    e2e_value = tokens / (e2e_ms * 1e-3)
+    e2e_value, _ = job_throughput(sum(time_steps(e2e_step, e2e_steps, stream)), e2e_steps, tokens, world, dev)
 
     # ---- roofline of the forward kernel (one launch per step) ----
     alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD + B * H * dk * dv * 4
@@ -351,7 +357,8 @@ def run_ours(args, world, rank, local):
     traffic = committed_traffic("fwd")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
-                "algorithmic_bytes_per_launch": alg_bytes}
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "kernel": "one gdr2_forward call: fwd_chunk_kernel (71% of its device time) + fwd_scan_kernel"}
     tflops = alg_flop / t_launch / 1e12
     tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
               "frac": tflops / peaks["bf16_tflops"], "algorithmic_flop_per_launch": alg_flop,

@@ -1,13 +1,15 @@
 """Run one libgdr2.so kernel on its benchmark workload, for profilers.
 
-    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd} [--launches N]
+    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd} [--launches N] [--batch B]
 
 fwd     gdr2_forward   B=4 H=16 T=4096 d=128 bf16 (the 1.3B-model layer)
 decode  gdr2_decode_step  256 sequences x 16 heads, d=128, fp32 state (256 MiB)
 bwd     gdr2_backward  B=2 H=16 T=4096 d=128 bf16 with saved chunk states
 
 Inputs are drawn once (seeded) and stay on the device; the kernel is then
-launched N times back to back (use ncu -s/-c to pick one launch).
+launched N times back to back (use ncu -s/-c to pick one launch). --batch
+overrides B of the forward and backward cases (a smaller capture whose inputs
+still exceed the 126 MB L2 at B >= 2).
 """
 from __future__ import annotations
 
@@ -23,10 +25,13 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=("fwd", "decode", "bwd"))
     ap.add_argument("--launches", type=int, default=2)
+    ap.add_argument("--batch", type=int, default=None)
     args = ap.parse_args()
     torch.cuda.set_device(0)
     if args.kernel == "fwd":
-        c = I.FWD_1P3B_BF16
+        c = dict(I.FWD_1P3B_BF16)
+        if args.batch:
+            c["B"] = args.batch
         x = I.make_forward_inputs(**c).to("cuda")
         o = torch.empty_like(x.v)
         ws = torch.empty(gdr2_forward_workspace_bytes(c["B"], c["T"], c["H"], c["dk"], c["dv"], c["dtype"]),
@@ -42,7 +47,9 @@ def main():
         for _ in range(args.launches):
             gdr2_decode_step(*tok, S)
     else:
-        c = I.BWD_1P3B_BF16
+        c = dict(I.BWD_1P3B_BF16)
+        if args.batch:
+            c["B"] = args.batch
         x = I.make_forward_inputs(**c).to("cuda")
         dO = I.make_upstream_grad(c["B"], c["T"], c["H"], c["dv"], c["seed"], dtype=c["dtype"]).cuda()
         _, _, saved = gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, save_states=True)
