@@ -75,9 +75,10 @@ constexpr uint32_t OFF_STG_V = 49152;   // v; exact path: A (fp32 [64][68]) over
 constexpr uint32_t OFF_STG_W = 65536;   // w
 constexpr uint32_t OFF_STG_LA = 81920;  // log_alpha [64][128] fp32; then per-channel references; exact path: G
 constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128
-constexpr uint32_t OFF_R0 = 147456;     // R_0 32 x 128
-constexpr uint32_t OFF_R1 = 155648;     // R_1 64 x 128; then over R0..R1: A and T (fp32 [64][68]) with the
-                                        // block-product scratch, then T (bf16 [64][64])
+constexpr uint32_t OFF_R0 = 147456;     // [R_0; R_1] (32 + 64 rows) x 128 as one B operand (24 KB); then
+                                        // A and T (fp32 [64][68]) with the block-product scratch, then
+                                        // T (bf16 [64][64]); last, M for the slot over R_1 and Z
+constexpr uint32_t OFF_R1 = 155648;     // second 16 KB of that region (M's first block)
 constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later W as [c][64 t]
 constexpr uint32_t OFF_QH = 188416;     // Q (.) exp G, transposed [c rows][64 t] (see qt_off)
 constexpr uint32_t OFF_KT = 204800;     // K (.) exp(G_C - G), 64 x 128
@@ -91,6 +92,8 @@ constexpr uint32_t OFF_Y = OFF_R0 + 64 * F_LD * 4;  // block-product scratch, 32
 constexpr int Y_LD = 36;
 constexpr uint32_t OFF_TB = OFF_R0;      // T in bf16, K-major [t][64 s]
 constexpr uint32_t TX_BYTES = 5 * 16384 + 32768;
+constexpr int R_ROWS = 96;               // rows of the stacked [R_0; R_1] operand
+static_assert(OFF_Z == OFF_R1 + 16384, "M (32 KB) is staged over R_1 and Z");
 
 constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
 
@@ -253,8 +256,9 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int task = blockIdx.x; task < p.ntasks && !timed_out; task += gridDim.x) {
         const int n = task % NC;
         const int Cn = min(C, p.T - n * C);
-        // this task's workspace slot: the threads store their parts of it directly
+        // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
+        if (tid == 0) bulk_wait_group_read0();  // the previous task's slot images have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
@@ -347,19 +351,15 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + 32 + tl, o8, 128)) = pack8(lq);
                 if (HI == 0) {
-                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(t, o8, 32)) = pack8(r);
+                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(t, o8, R_ROWS)) = pack8(r);
                     float r1[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) r1[x] = r[x] * r10[x];
-                    *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(t, o8, 64)) = pack8(r1);
+                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(32 + t, o8, R_ROWS)) = pack8(r1);
                 } else {
-                    *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(t, o8, 64)) = pack8(r);
+                    *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(32 + t, o8, R_ROWS)) = pack8(r);
                 }
-                {
-                    const uint4 v = pack8(kt);
-                    *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = v;
-                    *reinterpret_cast<uint4 *>(slot + SLOT_KT + sw_chunk(t, o8, 64)) = v;
-                }
+                *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
                 *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
@@ -371,7 +371,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         const bool exact = __syncthreads_or(risky) != 0;
         // the staging buffers are free once the operands are built: prefetch the next task
-        if (!exact && tid == 0 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
+        if (!exact && tid == 32 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
         if (exact) {
             // ---- exact path: G to shared memory, pairwise exponentials ----
             float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
@@ -399,11 +399,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 const int tl = t - 32 * HI;
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
-                {
-                    const uint4 v = pack8(kt);
-                    *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = v;
-                    *reinterpret_cast<uint4 *>(slot + SLOT_KT + sw_chunk(t, o8, 64)) = v;
-                }
+                *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
             }
@@ -451,26 +447,25 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     {
                         const uint4 v = pack8(pr);
                         *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, (i0 >> 3) + k8, 64)) = v;
-                        *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, (i0 >> 3) + k8, 64)) = v;
                     }
                 }
             }
+            fence_proxy_async_smem();  // P and K~ -> the bulk stores below
             __syncthreads();
-            if (tid == 0 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
+            if (tid == 32 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
         } else {
             // ---- tensor-core path: [A;P] = STACK R_I^T ----
             mma_sync_point();
             if (tid == 0) {
-                const uint32_t id0 = idesc_bf16(128, 32, false, false);
-                const uint32_t id1 = idesc_bf16(128, 64, false, false);
+                // one N = 96 product: columns [0, 32) against R_0, [32, 96) against R_1
+                static_assert(CK_AP1 == CK_AP0 + 32, "AP0 and AP1 are one accumulator");
+                const uint32_t idR = idesc_bf16(128, R_ROWS, false, false);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t koff = (ks & 3) * 32;
                     const uint64_t ad = sdesc_sw128(sbase + OFF_STACK + (ks >> 2) * 16384 + koff, 16, 1024);
-                    const uint64_t b0 = sdesc_sw128(sbase + OFF_R0 + (ks >> 2) * 4096 + koff, 16, 1024);
-                    const uint64_t b1 = sdesc_sw128(sbase + OFF_R1 + (ks >> 2) * 8192 + koff, 16, 1024);
-                    mma_bf16(tm + CK_AP0, ad, b0, id0, ks > 0);
-                    mma_bf16(tm + CK_AP1, ad, b1, id1, ks > 0);
+                    const uint64_t br = sdesc_sw128(sbase + OFF_R0 + (ks >> 2) * (R_ROWS * 128) + koff, 16, 1024);
+                    mma_bf16(tm + CK_AP0, ad, br, idR, ks > 0);
                 }
                 mma_commit(&ms.bar_mma);
             }
@@ -499,7 +494,6 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             {
                                 const uint4 v = pack8(pr);
                                 *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = v;
-                                *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, k8, 64)) = v;
                             }
                         }
                     }
@@ -516,7 +510,6 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             {
                                 const uint4 v = pack8(zz);
                                 *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, k8, 64)) = v;
-                                *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, k8, 64)) = v;
                             }
                     }
                 }
@@ -539,13 +532,19 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         {
                             const uint4 v = pack8(pr);
                             *reinterpret_cast<uint4 *>(sm + OFF_P + sw_chunk(t, colhalf * 4 + k8, 64)) = v;
-                            *reinterpret_cast<uint4 *>(slot + SLOT_P + sw_chunk(t, colhalf * 4 + k8, 64)) = v;
                         }
                     }
                 }
             }
+            fence_proxy_async_smem();  // P -> the bulk store below
             tc_fence_before_sync();
             __syncthreads();
+        }
+        // K~ and P are final: copy them to the slot in the background
+        if (tid == 0) {
+            bulk_store(slot + SLOT_KT, sm + OFF_KT, 16384);
+            bulk_store(slot + SLOT_P, sm + OFF_P, 8192);
+            bulk_commit_group();
         }
 
         // ================= UT solve: T = (I + A)^{-1}, in place =================
@@ -692,7 +691,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
 
-        // ================= W -> [c][64 t] over Z;  U~ -> [j][64 t] straight to the slot =================
+        // ================= W -> [c][64 t] over Z;  U~ -> [j][64 t] over STACK (for the slot) =================
         {
             const float e0 = ms.eg0[row], e1 = ms.eg1[row];
             float w0[32], w1[32];
@@ -711,12 +710,14 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float f[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(slot + SLOT_U + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
             }
         }
         mma_sync_point();
         // ================= Q'^T - Q^T = -W^T P^T ;  M = -K~^T W =================
         if (tid == 0) {
+            bulk_store(slot + SLOT_U, sm + OFF_STACK, 16384);  // U~, staged over the free STACK
+            bulk_commit_group();
             const uint32_t idQ = idesc_bf16(128, 64, false, false, true);
             const uint32_t idM = idesc_bf16(128, 128, true, false, true);
 #pragma unroll
@@ -731,7 +732,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // ================= Q' -> [c][64 t] and M -> [c' block][c][64 c'], straight to the slot =================
+        // ================= Q' -> [c][64 t] over STACK and M -> [c' block][c][64 c'] over R_1, Z (for the slot) ====
         {
             const int c = row;
             float d[32], m0[32];
@@ -742,7 +743,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QH + qt_off(c, colhalf * 32 + k8 * 8)), f);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) f[x] += d[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(slot + SLOT_Q + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + 16384 + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
             }
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
@@ -759,14 +760,20 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float f[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) f[x] = mv[k8 * 8 + x];
-                    *reinterpret_cast<uint4 *>(slot + SLOT_M + sw_chunk(c, (c0 >> 3) + k8, 128)) = pack8(f);
+                    *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(c, (c0 >> 3) + k8, 128)) = pack8(f);
                 }
             }
         }
         if (tid < DK) reinterpret_cast<float *>(p.ws + (size_t)p.ntasks * SLOT_BYTES + (size_t)task * GAMMA_BYTES)[tid] =
             ms.gC[tid];
+        fence_proxy_async_smem();  // Q' and M -> the bulk stores below
         tc_fence_before_sync();
         __syncthreads();  // every TMEM read of this task is done before the next task's MMAs
+        if (tid == 0) {
+            bulk_store(slot + SLOT_Q, sm + OFF_STACK + 16384, 16384);
+            bulk_store(slot + SLOT_M, sm + OFF_R1, 32768);
+            bulk_commit_group();
+        }
     }
     if (tid == 0) bulk_wait_group0();
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
