@@ -547,126 +547,203 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bulk_commit_group();
         }
 
-        // ================= UT solve: T = (I + A)^{-1}, in place =================
-        // D_I = (I + A_II)^{-1} for the four 16 x 16 diagonal blocks (forward substitution,
-        // one column per thread); then two doubling levels, each of the form
-        //   [[X, 0], [Y, Z]]^{-1} = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
-        // at 32 and at 64 rows. Every thread produces one row x four columns from
-        // 16-byte operand loads. A holds zeros on and above the diagonal, so the
-        // finished array is T with its zero upper triangle.
+        // ================= UT solve: T = (I + A)^{-1} =================
+        // Doubling from the sixteen 4 x 4 diagonal blocks: a unit lower-triangular block
+        // [[X, 0], [Y, Z]] has the inverse [[X^-1, 0], [-Z^-1 (Y X^-1), Z^-1]], so each level
+        // forms its lower-left blocks as two small products with the inverses of the level
+        // below. A holds zeros on and above the diagonal; levels 4..32 overwrite it in place
+        // (warps 0-1), level 64 (warps 0-3) writes T straight into its bf16 K-major copy
+        // while warps 4-7 convert the parts of T that are already final.
         {
-            float col[16];
-            const int I = (tid >> 4) & 3, sl = tid & 15;
-            float *Ab = A32 + (16 * I) * F_LD + 16 * I;
-            if (tid < 64) {
-#pragma unroll
-                for (int tl = 0; tl < 16; ++tl) {
-                    float arow[16];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (4 * q < tl) {
-                            const float4 v = *reinterpret_cast<const float4 *>(Ab + tl * F_LD + 4 * q);
-                            arow[4 * q] = v.x; arow[4 * q + 1] = v.y; arow[4 * q + 2] = v.z; arow[4 * q + 3] = v.w;
-                        }
-                    }
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                    for (int il = 0; il < tl; ++il) {
-                        if ((il & 3) == 0) a0 = fmaf(arow[il], col[il], a0);
-                        else if ((il & 3) == 1) a1 = fmaf(arow[il], col[il], a1);
-                        else if ((il & 3) == 2) a2 = fmaf(arow[il], col[il], a2);
-                        else a3 = fmaf(arow[il], col[il], a3);
-                    }
-                    col[tl] = (tl < sl) ? 0.f : (tl == sl ? 1.f : -((a0 + a1) + (a2 + a3)));
-                }
+            // level 4: one thread per diagonal block, by substitution
+            if (tid < 16) {
+                float *B0 = A32 + (4 * tid) * F_LD + 4 * tid;
+                const float4 r1 = *reinterpret_cast<const float4 *>(B0 + F_LD);
+                const float4 r2 = *reinterpret_cast<const float4 *>(B0 + 2 * F_LD);
+                const float4 r3 = *reinterpret_cast<const float4 *>(B0 + 3 * F_LD);
+                const float t10 = -r1.x;
+                const float t21 = -r2.y, t20 = -fmaf(r2.y, t10, r2.x);
+                const float t32 = -r3.z, t31 = -fmaf(r3.z, t21, r3.y);
+                const float t30 = -fmaf(r3.z, t20, fmaf(r3.y, t10, r3.x));
+                *reinterpret_cast<float4 *>(B0) = make_float4(1.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(B0 + F_LD) = make_float4(t10, 1.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(B0 + 2 * F_LD) = make_float4(t20, t21, 1.f, 0.f);
+                *reinterpret_cast<float4 *>(B0 + 3 * F_LD) = make_float4(t30, t31, t32, 1.f);
             }
-            __syncthreads();
-            if (tid < 64) {
-#pragma unroll
-                for (int tl = 0; tl < 16; ++tl) Ab[tl * F_LD + sl] = col[tl];
-            }
-            __syncthreads();
-        }
-        // one row x four columns of  Y = A[r0+r][c0 .. c0+n) . A[c0 .. c0+n)[k0+cs .. +3]
-        auto row_times_block = [&](int arow, int acol, int brow, int bcol, int n, float (&y)[4]) {
-            const float *Ar = A32 + arow * F_LD + acol;
-            y[0] = y[1] = y[2] = y[3] = 0.f;
-#pragma unroll 4
-            for (int u = 0; u < n; u += 4) {
-                const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
+            __syncwarp();
+            // level 8: warp 0, lane = (block h, row r of the lower half); Y rows through shuffles
+            if (tid < 32) {
+                const int h = tid >> 2, r = tid & 3;
+                float *Ar = A32 + (8 * h + 4 + r) * F_LD + 8 * h;  // A_10 row r, then T_1 row r at +4
+                const float *T0 = A32 + (8 * h) * F_LD + 8 * h;
+                const float4 a = *reinterpret_cast<const float4 *>(Ar);
                 const float av[4] = {a.x, a.y, a.z, a.w};
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const float4 tv = *reinterpret_cast<const float4 *>(A32 + (brow + u + k) * F_LD + bcol);
+                    const float4 tv = *reinterpret_cast<const float4 *>(T0 + k * F_LD);
                     y[0] = fmaf(av[k], tv.x, y[0]); y[1] = fmaf(av[k], tv.y, y[1]);
                     y[2] = fmaf(av[k], tv.z, y[2]); y[3] = fmaf(av[k], tv.w, y[3]);
                 }
-            }
-        };
-        auto neg_row_times_y = [&](int arow, int acol, int n, int ycol, float (&y)[4]) {
-            const float *Ar = A32 + arow * F_LD + acol;
-            y[0] = y[1] = y[2] = y[3] = 0.f;
-#pragma unroll 4
-            for (int u = 0; u < n; u += 4) {
-                const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
-                const float av[4] = {a.x, a.y, a.z, a.w};
+                const float4 t1 = *reinterpret_cast<const float4 *>(Ar + 4);
+                const float tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+                float o[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 yv = *reinterpret_cast<const float4 *>(Ys + (u + k) * Y_LD + ycol);
-                    y[0] = fmaf(av[k], yv.x, y[0]); y[1] = fmaf(av[k], yv.y, y[1]);
-                    y[2] = fmaf(av[k], yv.z, y[2]); y[3] = fmaf(av[k], yv.w, y[3]);
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) o[c] = fmaf(tv1[u], __shfl_sync(0xffffffffu, y[c], (tid & ~3) | u), o[c]);
+                *reinterpret_cast<float4 *>(Ar) = make_float4(-o[0], -o[1], -o[2], -o[3]);
+            }
+            if (tid < 64) {
+                named_barrier(1, 64);  // level 8 (warp 0) -> warp 1
+                // level 16: block I = tid / 16, row r of the lower half, column half ch
+                {
+                    const int I = tid >> 4, r = (tid >> 1) & 7, ch = tid & 1, base = 16 * I;
+                    float *Ar = A32 + (base + 8 + r) * F_LD + base;  // A_10 row r (8 wide), T_1 row r at +8
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const float4 a = *reinterpret_cast<const float4 *>(Ar + 4 * kk);
+                        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float4 tv =
+                                *reinterpret_cast<const float4 *>(A32 + (base + 4 * kk + k) * F_LD + base + 4 * ch);
+                            y[0] = fmaf(av[k], tv.x, y[0]); y[1] = fmaf(av[k], tv.y, y[1]);
+                            y[2] = fmaf(av[k], tv.z, y[2]); y[3] = fmaf(av[k], tv.w, y[3]);
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(Ys + (8 * I + r) * Y_LD + 4 * ch) = make_float4(y[0], y[1], y[2], y[3]);
+                    __syncwarp();
+                    float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int uu = 0; uu < 2; ++uu) {
+                        const float4 t = *reinterpret_cast<const float4 *>(Ar + 8 + 4 * uu);
+                        const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float4 yv = *reinterpret_cast<const float4 *>(Ys + (8 * I + 4 * uu + u) * Y_LD + 4 * ch);
+                            o[0] = fmaf(tv[u], yv.x, o[0]); o[1] = fmaf(tv[u], yv.y, o[1]);
+                            o[2] = fmaf(tv[u], yv.z, o[2]); o[3] = fmaf(tv[u], yv.w, o[3]);
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(Ar + 4 * ch) = make_float4(-o[0], -o[1], -o[2], -o[3]);
+                }
+                __syncwarp();
+                // level 32: block b = warp (its two 16-blocks came from this warp), two rows x four columns
+                {
+                    const int b = tid >> 5, rp = lane >> 2, cg = lane & 3, base = 32 * b;
+                    float *A0 = A32 + (base + 16 + 2 * rp) * F_LD + base;  // A_10 rows 2rp, 2rp+1; T_1 at +16
+                    float *A1 = A0 + F_LD;
+                    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const float4 a0 = *reinterpret_cast<const float4 *>(A0 + 4 * kk);
+                        const float4 a1 = *reinterpret_cast<const float4 *>(A1 + 4 * kk);
+                        const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float4 tv =
+                                *reinterpret_cast<const float4 *>(A32 + (base + 4 * kk + k) * F_LD + base + 4 * cg);
+                            y0[0] = fmaf(av0[k], tv.x, y0[0]); y0[1] = fmaf(av0[k], tv.y, y0[1]);
+                            y0[2] = fmaf(av0[k], tv.z, y0[2]); y0[3] = fmaf(av0[k], tv.w, y0[3]);
+                            y1[0] = fmaf(av1[k], tv.x, y1[0]); y1[1] = fmaf(av1[k], tv.y, y1[1]);
+                            y1[2] = fmaf(av1[k], tv.z, y1[2]); y1[3] = fmaf(av1[k], tv.w, y1[3]);
+                        }
+                    }
+                    float *Yb = Ys + (16 * b) * Y_LD;
+                    *reinterpret_cast<float4 *>(Yb + (2 * rp) * Y_LD + 4 * cg) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+                    *reinterpret_cast<float4 *>(Yb + (2 * rp + 1) * Y_LD + 4 * cg) =
+                        make_float4(y1[0], y1[1], y1[2], y1[3]);
+                    __syncwarp();
+                    float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        const float4 t0 = *reinterpret_cast<const float4 *>(A0 + 16 + 4 * uu);
+                        const float4 t1 = *reinterpret_cast<const float4 *>(A1 + 16 + 4 * uu);
+                        const float tv0[4] = {t0.x, t0.y, t0.z, t0.w}, tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float4 yv = *reinterpret_cast<const float4 *>(Yb + (4 * uu + u) * Y_LD + 4 * cg);
+                            o0[0] = fmaf(tv0[u], yv.x, o0[0]); o0[1] = fmaf(tv0[u], yv.y, o0[1]);
+                            o0[2] = fmaf(tv0[u], yv.z, o0[2]); o0[3] = fmaf(tv0[u], yv.w, o0[3]);
+                            o1[0] = fmaf(tv1[u], yv.x, o1[0]); o1[1] = fmaf(tv1[u], yv.y, o1[1]);
+                            o1[2] = fmaf(tv1[u], yv.z, o1[2]); o1[3] = fmaf(tv1[u], yv.w, o1[3]);
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(A0 + 4 * cg) = make_float4(-o0[0], -o0[1], -o0[2], -o0[3]);
+                    *reinterpret_cast<float4 *>(A1 + 4 * cg) = make_float4(-o1[0], -o1[1], -o1[2], -o1[3]);
                 }
             }
-            y[0] = -y[0]; y[1] = -y[1]; y[2] = -y[2]; y[3] = -y[3];
-        };
-        // level 32: blocks b = 0, 1 (rows 32b .. 32b+31):  A[32b+16.., 32b..] <- -D_hi (A_lohi D_lo)
-        {
-            const int b = tid >> 6, r = (tid >> 2) & 15, cs = 4 * (tid & 3);
-            float y[4];
-            if (tid < 128) {
-                row_times_block(32 * b + 16 + r, 32 * b, 32 * b, 32 * b + cs, 16, y);
-                *reinterpret_cast<float4 *>(Ys + (16 * b + r) * Y_LD + cs) = make_float4(y[0], y[1], y[2], y[3]);
-            }
             __syncthreads();
+            // level 64: rows 32 + 2rp, +1 and columns 4cg .. 4cg+3 of T_10 = -T_1 (A_10 T_0)
+            const int rp = tid >> 3, cg = tid & 7;
+            const float *A0 = A32 + (32 + 2 * rp) * F_LD;  // A_10 row (32 wide), T_1 row at +32
+            const float *A1 = A0 + F_LD;
             if (tid < 128) {
-                const float *Ar = A32 + (32 * b + 16 + r) * F_LD + 32 * b + 16;  // D_hi row
-                y[0] = y[1] = y[2] = y[3] = 0.f;
-#pragma unroll
-                for (int u = 0; u < 16; u += 4) {
-                    const float4 a = *reinterpret_cast<const float4 *>(Ar + u);
-                    const float av[4] = {a.x, a.y, a.z, a.w};
+                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+                for (int kk = 0; kk < 8; ++kk) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(A0 + 4 * kk);
+                    const float4 a1 = *reinterpret_cast<const float4 *>(A1 + 4 * kk);
+                    const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float4 yv = *reinterpret_cast<const float4 *>(Ys + (16 * b + u + k) * Y_LD + cs);
-                        y[0] = fmaf(av[k], yv.x, y[0]); y[1] = fmaf(av[k], yv.y, y[1]);
-                        y[2] = fmaf(av[k], yv.z, y[2]); y[3] = fmaf(av[k], yv.w, y[3]);
+                        const float4 tv = *reinterpret_cast<const float4 *>(A32 + (4 * kk + k) * F_LD + 4 * cg);
+                        y0[0] = fmaf(av0[k], tv.x, y0[0]); y0[1] = fmaf(av0[k], tv.y, y0[1]);
+                        y0[2] = fmaf(av0[k], tv.z, y0[2]); y0[3] = fmaf(av0[k], tv.w, y0[3]);
+                        y1[0] = fmaf(av1[k], tv.x, y1[0]); y1[1] = fmaf(av1[k], tv.y, y1[1]);
+                        y1[2] = fmaf(av1[k], tv.z, y1[2]); y1[3] = fmaf(av1[k], tv.w, y1[3]);
                     }
                 }
-                *reinterpret_cast<float4 *>(A32 + (32 * b + 16 + r) * F_LD + 32 * b + cs) =
-                    make_float4(-y[0], -y[1], -y[2], -y[3]);
+                *reinterpret_cast<float4 *>(Ys + (2 * rp) * Y_LD + 4 * cg) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+                *reinterpret_cast<float4 *>(Ys + (2 * rp + 1) * Y_LD + 4 * cg) = make_float4(y1[0], y1[1], y1[2], y1[3]);
             }
             __syncthreads();
-        }
-        // level 64:  A[32.., 0..31] <- -T_1 (A_10 T_0)
-        {
-            const int r = tid >> 3, cs = 4 * (tid & 7);
-            float y[4];
-            row_times_block(32 + r, 0, 0, cs, 32, y);
-            *reinterpret_cast<float4 *>(Ys + r * Y_LD + cs) = make_float4(y[0], y[1], y[2], y[3]);
+            // T in bf16, K-major [t][64 s] over the front of the fp32 array: every read of
+            // the array below precedes the barrier, every write follows it
+            float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+            float lo[8], hi[8];
+            const int ct = (tid - 128) >> 2, c8 = tid & 3;  // converter: row, 8-column chunk
+            if (tid < 128) {
+#pragma unroll 2
+                for (int uu = 0; uu < 8; ++uu) {
+                    const float4 t0 = *reinterpret_cast<const float4 *>(A0 + 32 + 4 * uu);
+                    const float4 t1 = *reinterpret_cast<const float4 *>(A1 + 32 + 4 * uu);
+                    const float tv0[4] = {t0.x, t0.y, t0.z, t0.w}, tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 yv = *reinterpret_cast<const float4 *>(Ys + (4 * uu + u) * Y_LD + 4 * cg);
+                        o0[0] = fmaf(tv0[u], yv.x, o0[0]); o0[1] = fmaf(tv0[u], yv.y, o0[1]);
+                        o0[2] = fmaf(tv0[u], yv.z, o0[2]); o0[3] = fmaf(tv0[u], yv.w, o0[3]);
+                        o1[0] = fmaf(tv1[u], yv.x, o1[0]); o1[1] = fmaf(tv1[u], yv.y, o1[1]);
+                        o1[2] = fmaf(tv1[u], yv.z, o1[2]); o1[3] = fmaf(tv1[u], yv.w, o1[3]);
+                    }
+                }
+            } else {
+                // T rows 0..31 (columns 0..31; 32..63 are zero) and T_1 (rows and columns 32..63)
+                load8f(A32 + ct * F_LD + 8 * c8, lo);
+                load8f(A32 + (32 + ct) * F_LD + 32 + 8 * c8, hi);
+            }
             __syncthreads();
-            neg_row_times_y(32 + r, 32, 32, cs, y);
-            *reinterpret_cast<float4 *>(A32 + (32 + r) * F_LD + cs) = make_float4(y[0], y[1], y[2], y[3]);
-            __syncthreads();
-        }
-        // T -> bf16, K-major [t][64 s], over the front of the same region
-        {
-            const int t = tid >> 2, k0 = (tid & 3) * 2;
-            float f0[8], f1[8];
-            load8f(A32 + t * F_LD + k0 * 8, f0);
-            load8f(A32 + t * F_LD + (k0 + 1) * 8, f1);
-            __syncthreads();
-            *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(t, k0, 64)) = pack8(f0);
-            *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(t, k0 + 1, 64)) = pack8(f1);
+            if (tid < 128) {
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(-o0[0], -o0[1]), h1 = __floats2bfloat162_rn(-o0[2], -o0[3]);
+                uint2 u0;
+                u0.x = *reinterpret_cast<uint32_t *>(&h0);
+                u0.y = *reinterpret_cast<uint32_t *>(&h1);
+                h0 = __floats2bfloat162_rn(-o1[0], -o1[1]);
+                h1 = __floats2bfloat162_rn(-o1[2], -o1[3]);
+                uint2 u1;
+                u1.x = *reinterpret_cast<uint32_t *>(&h0);
+                u1.y = *reinterpret_cast<uint32_t *>(&h1);
+                *reinterpret_cast<uint2 *>(sm + OFF_TB + sw_chunk(32 + 2 * rp, cg >> 1, 64) + (cg & 1) * 8) = u0;
+                *reinterpret_cast<uint2 *>(sm + OFF_TB + sw_chunk(32 + 2 * rp + 1, cg >> 1, 64) + (cg & 1) * 8) = u1;
+            } else {
+                const float zz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(ct, c8, 64)) = pack8(lo);
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(ct, 4 + c8, 64)) = pack8(zz);
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw_chunk(32 + ct, 4 + c8, 64)) = pack8(hi);
+            }
         }
         mma_sync_point();
         // ================= W^T_I = (L^e_I)^T T[:,I]^T ;  U~^T = Z^T T^T =================
