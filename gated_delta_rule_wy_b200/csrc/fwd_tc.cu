@@ -20,11 +20,11 @@
 // kernels:
 //   1. chunk kernel (persistent, every (batch, head, chunk) task in parallel
 //      on all SMs): decay, gated keys, [A;P], the UT solve, W, U~, M, Q';
-//      writes M, K~, U~, Q', P (bf16, already in the tensor-core operand
+//      writes [Q'; M], K~, U~, P (bf16, already in the tensor-core operand
 //      layouts of kernel 2) and gamma = exp(G_C) to the workspace;
-//   2. scan kernel (one CTA per (batch, head), chunks in order): S stays in
-//      TMEM as fp32; per chunk one pass copies S to a bf16 operand and scales
-//      it by gamma in place, then one batch of MMAs produces S' and O^T.
+//   2. scan kernel (one CTA per (batch, head), chunks in order): S^T stays in
+//      TMEM as fp32; per chunk one pass copies it to a bf16 TMEM operand and
+//      scales it by gamma, then one batch of MMAs produces S'^T and O^T.
 //
 // Decay range. exp(G_t - G_i) is formed as a product of two factors around a
 // per-channel reference g_I, the cumulative decay at the midpoint of the
@@ -41,10 +41,11 @@
 // j value channel; accumulators fp32 in TMEM, operands bf16 in
 // 128-byte-swizzled shared memory written by the threads, inputs staged by
 // TMA without multicast; one thread issues every MMA):
-//   chunk kernel: [A;P] = [L^e_0; L^q_0; L^e_1; L^q_1] R_I^T (K = c)
+//   chunk kernel: [A;P] = [L^e_0; L^q_0; L^e_1; L^q_1] [R_0; R_1]^T (K = c)
 //                 W^T_I = (L^e_I)^T T[:, I]^T, W = sum_I exp(g_I) W_I
-//                 U~^T = Z^T T^T;  Q'^T - Q^T = -W^T P^T;  M = -K~^T W
-//   scan kernel:  S += M S_bf16 + K~^T U~;  O^T = S_bf16^T Q'^T + U~^T P^T
+//                 U~^T = Z^T T^T;  Q' - Q^ = -P W (M = 64);  M = -K~^T W
+//   scan kernel:  [O^T | S^T] += S_bf16^T [Q'; M]^T   (A from TMEM, N = 192)
+//                 S^T += U~^T K~;  O^T += U~^T P^T
 // Every mbarrier wait is bounded; a CTA that gives up records kStatusTimeout,
 // frees its TMEM and exits.
 
@@ -74,13 +75,13 @@ constexpr uint32_t OFF_STG_B = 32768;   // b
 constexpr uint32_t OFF_STG_V = 49152;   // v; exact path: A (fp32 [64][68]) over V and W
 constexpr uint32_t OFF_STG_W = 65536;   // w
 constexpr uint32_t OFF_STG_LA = 81920;  // log_alpha [64][128] fp32; then per-channel references; exact path: G
-constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128
+constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128; later W as [c][64 t]
 constexpr uint32_t OFF_R0 = 147456;     // [R_0; R_1] (32 + 64 rows) x 128 as one B operand (24 KB); then
                                         // A and T (fp32 [64][68]) with the block-product scratch, then
-                                        // T (bf16 [64][64]); last, M for the slot over R_1 and Z
-constexpr uint32_t OFF_R1 = 155648;     // second 16 KB of that region (M's first block)
-constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later W as [c][64 t]
-constexpr uint32_t OFF_QH = 188416;     // Q (.) exp G, transposed [c rows][64 t] (see qt_off)
+                                        // T (bf16 [64][64]); last, the tail of [Q'; M] (staged from STACK on)
+
+constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later U~^T as [j][64 t] for the slot
+constexpr uint32_t OFF_QH = 188416;     // Q^ = Q (.) exp G, [t rows][128 c] (K-major chunks)
 constexpr uint32_t OFF_KT = 204800;     // K (.) exp(G_C - G), 64 x 128
 constexpr uint32_t OFF_P = 221184;      // prefix-scan scratch during prep; then P 64 x 64
 constexpr uint32_t OFF_MISC = 229376;   // barriers, per-channel vectors
@@ -93,7 +94,7 @@ constexpr int Y_LD = 36;
 constexpr uint32_t OFF_TB = OFF_R0;      // T in bf16, K-major [t][64 s]
 constexpr uint32_t TX_BYTES = 5 * 16384 + 32768;
 constexpr int R_ROWS = 96;               // rows of the stacked [R_0; R_1] operand
-static_assert(OFF_Z == OFF_R1 + 16384, "M (32 KB) is staged over R_1 and Z");
+static_assert(OFF_STACK + 2 * 192 * 128 <= OFF_Z, "[Q'; M] (48 KB) is staged over STACK and R, clear of Z");
 
 constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
 
@@ -113,24 +114,6 @@ __device__ __forceinline__ uint32_t sw_chunk(int row, int o8, int rows)
 {
     const int blk = o8 >> 3, ch = o8 & 7;
     return (uint32_t)(blk * rows * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
-}
-
-// Byte offset of (c, t) in the transposed Q (.) exp G buffer: rows of 64 t
-// (128 bytes), 16-byte chunks permuted by both c % 8 and (c / 8) % 8, so the
-// prep (8 channels apart per lane) and the epilogue (one row per lane) are both
-// free of bank conflicts.
-__device__ __forceinline__ uint32_t qt_off(int c, int t)
-{
-    return (uint32_t)(c * 128 + ((((t >> 3) ^ (c & 7) ^ ((c >> 3) & 7))) << 4) + ((t & 7) << 1));
-}
-
-__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d)
-{
-    uint2 u;
-    __nv_bfloat162 h;
-    h = __floats2bfloat162_rn(a, b); u.x = *reinterpret_cast<uint32_t *>(&h);
-    h = __floats2bfloat162_rn(c, d); u.y = *reinterpret_cast<uint32_t *>(&h);
-    return u;
 }
 
 __device__ __forceinline__ uint4 pack8(const float (&f)[8])
@@ -170,12 +153,12 @@ __device__ __forceinline__ void store8f(float *p, const float (&f)[8])
 
 // ---- workspace slot written by the chunk kernel, read by the scan kernel ----
 // (one per (batch, head, chunk); operand images in the scan kernel's layouts)
-constexpr uint32_t SLOT_M = 0;        // M = -K~^T W   [c' block][c rows][64 c'] (K-major A)
-constexpr uint32_t SLOT_KT = 32768;   // K~             [c block][t rows][64 c]   (MN-major A)
-constexpr uint32_t SLOT_U = 49152;    // U~             [j rows][64 t]            (K-major A and B)
-constexpr uint32_t SLOT_Q = 65536;    // Q'^T           [c rows][64 t]            (MN-major B)
-constexpr uint32_t SLOT_P = 81920;    // P              [t rows][64 i]            (K-major B)
+constexpr uint32_t SLOT_B1 = 0;       // [Q'; M]  [c' block][64 t + 128 c rows][64 c'] (K-major B, N = 192)
+constexpr uint32_t SLOT_KT = 49152;   // K~       [c block][t rows][64 c]   (MN-major B)
+constexpr uint32_t SLOT_U = 65536;    // U~^T     [j rows][64 t]            (K-major A)
+constexpr uint32_t SLOT_P = 81920;    // P        [t rows][64 i]            (K-major B)
 constexpr uint32_t SLOT_BYTES = 90112;
+constexpr int B1_ROWS = 192;          // rows of [Q'; M]: t first, then c
 constexpr uint32_t GAMMA_BYTES = DK * 4;  // exp(G_C), stored after all slots
 
 struct ChunkParams {
@@ -186,7 +169,8 @@ struct ChunkParams {
 };
 
 // TMEM columns of the chunk kernel
-constexpr uint32_t CK_M = 0, CK_U = 128, CK_Q = 192, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384, CK_AP1 = 416;
+constexpr uint32_t CK_M = 0, CK_U = 128, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384, CK_AP1 = 416;
+constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W_0, W_1 once those are read
 
 __global__ void __launch_bounds__(NT, 1)
 fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -258,7 +242,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int Cn = min(C, p.T - n * C);
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
-        if (tid == 0) bulk_wait_group_read0();  // the previous task's slot images have left shared memory
+        if (tid == 0) bulk_wait_group_read1();  // K~ and P of the previous task have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
@@ -297,6 +281,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ms.eg0[c] = __expf(g0);
             ms.eg1[c] = __expf(g1);
         }
+        if (tid == 0) bulk_wait_group_read0();  // ... and [Q'; M], U~ too, before the operands are rebuilt
         __syncthreads();
         bool risky = false;
         float g0[8], g1[8], gC[8];
@@ -317,7 +302,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             const __nv_bfloat16 *vs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_V);
             const __nv_bfloat16 *ws = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_W);
-            float egI[8], kcf[8], r10[8], gr[8], qh4[8][4];
+            float egI[8], kcf[8], r10[8], gr[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
                 gr[x] = HI ? g1[x] : g0[x];
@@ -361,13 +346,8 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
                 *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
-#pragma unroll
-                for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
+                *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
             }
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-                *reinterpret_cast<uint2 *>(sm + OFF_QH + qt_off(o8 * 8 + x, tg * 4)) =
-                    pack4(qh4[x][0], qh4[x][1], qh4[x][2], qh4[x][3]);
         }
         const bool exact = __syncthreads_or(risky) != 0;
         // the staging buffers are free once the operands are built: prefetch the next task
@@ -382,7 +362,6 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             // operands with one exponential of a non-positive argument each
-            float qh4[8][4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int t = tg * 4 + m;
@@ -400,13 +379,8 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int tl = t - 32 * HI;
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
                 *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
-#pragma unroll
-                for (int x = 0; x < 8; ++x) qh4[x][m] = qh[x];
+                *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
             }
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-                *reinterpret_cast<uint2 *>(sm + OFF_QH + qt_off(o8 * 8 + x, tg * 4)) =
-                    pack4(qh4[x][0], qh4[x][1], qh4[x][2], qh4[x][3]);
             if (tid < DK) ms.eg0[tid] = ms.eg1[tid] = 1.f;
             // A and P rows: thread -> row t = tid / 4, columns 16*(tid % 4) .. +15
             {
@@ -768,7 +742,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
 
-        // ================= W -> [c][64 t] over Z;  U~ -> [j][64 t] over STACK (for the slot) =================
+        // ================= W -> [c][64 t] over STACK;  U~^T -> [j][64 t] over Z (for the slot) =================
         {
             const float e0 = ms.eg0[row], e1 = ms.eg1[row];
             float w0[32], w1[32];
@@ -778,7 +752,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float f[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) f[x] = e0 * w0[k8 * 8 + x] + e1 * w1[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
             }
             float u[32];
             tmem_ld32(tm_lane + CK_U + colhalf * 32, u);
@@ -787,21 +761,19 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float f[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) f[x] = u[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
+                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(row, colhalf * 4 + k8, 128)) = pack8(f);
             }
         }
         mma_sync_point();
-        // ================= Q'^T - Q^T = -W^T P^T ;  M = -K~^T W =================
+        // ================= Q' - Q^ = -P W (M = 64) ;  M = -K~^T W =================
         if (tid == 0) {
-            bulk_store(slot + SLOT_U, sm + OFF_STACK, 16384);  // U~, staged over the free STACK
-            bulk_commit_group();
-            const uint32_t idQ = idesc_bf16(128, 64, false, false, true);
+            const uint32_t idQ = idesc_bf16(64, 128, false, false, true);
             const uint32_t idM = idesc_bf16(128, 128, true, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t aw = sdesc_sw128(sbase + OFF_Z + ks * 32, 16, 1024);
-                const uint64_t bp = sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024);
-                mma_bf16(tm + CK_Q, aw, bp, idQ, ks > 0);
+                const uint64_t aw = sdesc_sw128(sbase + OFF_STACK + ks * 32, 16, 1024);  // W as [c][64 s]
+                const uint64_t ap = sdesc_sw128(sbase + OFF_P + ks * 32, 16, 1024);      // P as [t][64 s]
+                mma_bf16(tm + CK_Q, ap, aw, idQ, ks > 0);
                 const uint64_t ak = sdesc_sw128(sbase + OFF_KT + ks * 2048, 8192, 1024);
                 mma_bf16(tm + CK_M, ak, aw, idM, ks > 0);
             }
@@ -809,46 +781,41 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
-        // ================= Q' -> [c][64 t] over STACK and M -> [c' block][c][64 c'] over R_1, Z (for the slot) ====
+        // ================= [Q'; M] -> [c' block][192 rows][64 c'] over STACK and R (for the slot) =================
         {
-            const int c = row;
-            float d[32], m0[32];
-            tmem_ld32x2(tm_lane + CK_Q + colhalf * 32, tm_lane + CK_M + colhalf * 64, d, m0);
+            // M: lane c, columns c' of this thread's half -> rows 64 + c
+            float m0[32], m1[32];
+            tmem_ld32x2(tm_lane + CK_M + colhalf * 64, tm_lane + CK_M + colhalf * 64 + 32, m0, m1);
 #pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) {
+            for (int k8 = 0; k8 < 8; ++k8) {
                 float f[8];
-                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QH + qt_off(c, colhalf * 32 + k8 * 8)), f);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) f[x] += d[k8 * 8 + x];
-                *reinterpret_cast<uint4 *>(sm + OFF_STACK + 16384 + sw_chunk(c, colhalf * 4 + k8, 128)) = pack8(f);
+                for (int x = 0; x < 8; ++x) f[x] = k8 < 4 ? m0[k8 * 8 + x] : m1[(k8 - 4) * 8 + x];
+                *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 + row, colhalf * 8 + k8, B1_ROWS)) = pack8(f);
             }
+            // Q': the M = 64 accumulator holds row t in lane t % 16 of warp quarter t / 16
+            float d0[32], d1[32];
+            tmem_ld32x2(tm_lane + CK_Q + colhalf * 64, tm_lane + CK_Q + colhalf * 64 + 32, d0, d1);
+            if (lane < 16) {
+                const int t = quarter * 16 + lane;
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                const int c0 = colhalf * 64 + q2 * 32;
-                float mv[32];
-                if (q2 == 0) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) mv[i] = m0[i];
-                } else {
-                    tmem_ld32(tm_lane + CK_M + c0, mv);
-                }
-#pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
+                for (int k8 = 0; k8 < 8; ++k8) {
                     float f[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QH + sw_chunk(t, colhalf * 8 + k8, 64)), f);
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) f[x] = mv[k8 * 8 + x];
-                    *reinterpret_cast<uint4 *>(sm + OFF_R1 + sw_chunk(c, (c0 >> 3) + k8, 128)) = pack8(f);
+                    for (int x = 0; x < 8; ++x) f[x] += k8 < 4 ? d0[k8 * 8 + x] : d1[(k8 - 4) * 8 + x];
+                    *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(t, colhalf * 8 + k8, B1_ROWS)) = pack8(f);
                 }
             }
         }
         if (tid < DK) reinterpret_cast<float *>(p.ws + (size_t)p.ntasks * SLOT_BYTES + (size_t)task * GAMMA_BYTES)[tid] =
             ms.gC[tid];
-        fence_proxy_async_smem();  // Q' and M -> the bulk stores below
+        fence_proxy_async_smem();  // [Q'; M] and U~^T -> the bulk stores below
         tc_fence_before_sync();
         __syncthreads();  // every TMEM read of this task is done before the next task's MMAs
         if (tid == 0) {
-            bulk_store(slot + SLOT_Q, sm + OFF_STACK + 16384, 16384);
-            bulk_store(slot + SLOT_M, sm + OFF_R1, 32768);
+            bulk_store(slot + SLOT_B1, sm + OFF_STACK, 2 * B1_ROWS * 128);
+            bulk_store(slot + SLOT_U, sm + OFF_Z, 16384);
             bulk_commit_group();
         }
     }
@@ -860,13 +827,20 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 // ---- scan kernel ----
+// One CTA per (b, h). TMEM holds S^T (lane j, column c) in fp32 in one of two
+// regions that alternate per chunk, each laid out [O^T (64 t) | S^T (128 c)] so
+// that one N = 192 product writes a chunk's output and state together; the
+// bf16 copy of S^T that those products read as their A operand sits in TMEM
+// too. O^T of chunk n is stored while chunk n + 1 runs in the other region.
 constexpr uint32_t SC_SLOT0 = 0;
 constexpr uint32_t SC_SLOT1 = SLOT_BYTES;          // 90112, 1024-aligned
-constexpr uint32_t SC_SB = 2 * SLOT_BYTES;         // S^T bf16 [j block][c rows][64 j]
-constexpr uint32_t SC_O = SC_SB + 32768;           // O tile [64 t][128 j] bf16
+constexpr uint32_t SC_O = 2 * SLOT_BYTES;          // O tile [64 t][128 j] bf16
 constexpr uint32_t SC_MISC = SC_O + 16384;
 constexpr uint32_t SC_SMEM_BYTES = SC_MISC + 1280 + 1024;
-constexpr uint32_t SC_S = 0, SC_OT = 128, SC_COLS = 256;  // O^T double-buffered: SC_OT + 64 * (n & 1)
+constexpr uint32_t SC_REG = 256;                    // region r at columns 256 r: O^T then S^T
+constexpr uint32_t SC_OT = 0, SC_ST = 64;           // offsets within a region
+constexpr uint32_t SC_SA = 448;                     // S^T in bf16, two values per column (64 columns)
+constexpr uint32_t SC_COLS = 512;
 
 struct ScanMisc {
     uint64_t bar_full[2];
@@ -899,6 +873,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     const int bh = blockIdx.x;
     const int bb = bh / p.H, h = bh % p.H;
     const int NC = p.NC;
+    const int c0 = colhalf * 64;  // this thread's 64 state columns c (S^T columns)
 
     if (tid == 0) {
         mbar_init(&ms.bar_full[0], 1);
@@ -915,7 +890,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     tc_fence_after_sync();
     const uint32_t tm = ms.tmem_base;
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
-    const int row = quarter * 32 + lane;
+    const int j = quarter * 32 + lane;  // this thread's TMEM lane = value channel
 
     auto issue_slot = [&](int n) {
         const int sl = n & 1;
@@ -929,15 +904,15 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         if (NC > 0) issue_slot(0);
         if (NC > 1) issue_slot(1);
     }
-    // initial state: lane c, columns j (half per warp)
+    // initial state S^T[j][c] = S0[c][j] into region 1 (chunk 0 reads the region of "chunk -1")
     {
         float v[32];
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
-            const int j0 = colhalf * 64 + q2 * 32;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = p.S0 ? p.S0[((size_t)bh * DK + row) * DV + j0 + i] : 0.f;
-            tmem_st32(tm_lane + SC_S + j0, v);
+            for (int i = 0; i < 32; ++i)
+                v[i] = p.S0 ? p.S0[((size_t)bh * DK + c0 + q2 * 32 + i) * DV + j] : 0.f;
+            tmem_st32(tm_lane + SC_REG + SC_ST + c0 + q2 * 32, v);
         }
     }
     tc_fence_before_sync();
@@ -958,12 +933,13 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         if (tid == 0) bulk_wait_group_read0();  // the previous tile has left shared memory
         named_barrier(1, 128);
         float o0[32], o1[32];
-        tmem_ld32x2(tm_lane + SC_OT + 64 * (m & 1), tm_lane + SC_OT + 64 * (m & 1) + 32, o0, o1);
+        const uint32_t ot_col = SC_REG * (m & 1) + SC_OT;
+        tmem_ld32x2(tm_lane + ot_col, tm_lane + ot_col + 32, o0, o1);
         __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            ot[i * DV + row] = __float2bfloat16_rn(o0[i]);
-            ot[(32 + i) * DV + row] = __float2bfloat16_rn(o1[i]);
+            ot[i * DV + j] = __float2bfloat16_rn(o0[i]);
+            ot[(32 + i) * DV + j] = __float2bfloat16_rn(o1[i]);
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
@@ -977,80 +953,76 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     for (int n = 0; n < NC; ++n) {
         const int sl = n & 1;
         const uint32_t slot = sbase + (sl ? SC_SLOT1 : SC_SLOT0);
+        const uint32_t rg = SC_REG * (uint32_t)sl, rg_prev = SC_REG * (uint32_t)(sl ^ 1);
         if (!wait_bar(&ms.bar_full[sl], ph_full[sl])) { timed_out = true; break; }
-        // ---- S -> bf16 operand; S <- Diag(gamma) S in TMEM ----
-        {
-            const int c = row;
-            const float g = ms.gam[sl][c];
-            float s2[2][32];
-            tmem_ld32x2(tm_lane + SC_S + colhalf * 64, tm_lane + SC_S + colhalf * 64 + 32, s2[0], s2[1]);
+        // ---- S^T (previous region) -> bf16 operand; gamma-scaled S^T -> this region; O^T <- 0 ----
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                const int j0 = colhalf * 64 + q2 * 32;
-                float (&sv)[32] = s2[q2];
-                if (p.saved_states) {
-                    float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c) * DV + j0;
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int cb = c0 + q2 * 32;
+            float sv[32];
+            tmem_ld32(tm_lane + rg_prev + SC_ST + cb, sv);
+            if (p.saved_states) {
+                float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + cb) * DV + j;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4 *>(dst + i) = make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3]);
-                }
-#pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    float f[8];
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) f[x] = sv[k8 * 8 + x];
-                    *reinterpret_cast<uint4 *>(sm + SC_SB + sw_chunk(c, (j0 >> 3) + k8, 128)) = pack8(f);
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] *= g;
-                tmem_st32(tm_lane + SC_S + j0, sv);
+                for (int i = 0; i < 32; ++i) dst[(size_t)i * DV] = sv[i];
             }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                __nv_bfloat162 hv = __floats2bfloat162_rn(sv[2 * i], sv[2 * i + 1]);
+                pk[i] = *reinterpret_cast<uint32_t *>(&hv);
+            }
+            tmem_st16u(tm_lane + SC_SA + (uint32_t)(cb >> 1), pk);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] *= ms.gam[sl][cb + i];
+            tmem_st32(tm_lane + rg + SC_ST + cb, sv);
         }
-        fence_proxy_async_smem();
+        {
+            float zz[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) zz[i] = 0.f;
+            tmem_st32(tm_lane + rg + SC_OT + colhalf * 32, zz);
+        }
         tc_fence_before_sync();
         __syncthreads();
         tc_fence_after_sync();
-        // ---- S += M S_bf16 + K~^T U~ ;  O^T = S_bf16^T Q'^T + U~^T P^T ----
+        // ---- [O^T | S^T] += S_bf16^T [Q'; M]^T ;  S^T += U~^T K~ ;  O^T += U~^T P^T ----
         if (tid == 128) {
-            const uint32_t idM = idesc_bf16(128, 128, false, true);
-            const uint32_t idK = idesc_bf16(128, 128, true, false);
-            const uint32_t idO1 = idesc_bf16(128, 64, true, true);
-            const uint32_t idO2 = idesc_bf16(128, 64, false, false);
-            const uint32_t d_o = tm + SC_OT + 64 * sl;
+            const uint32_t id1 = idesc_bf16(128, B1_ROWS, false, false);
+            const uint32_t idS = idesc_bf16(128, 128, false, true);
+            const uint32_t idO = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t am = sdesc_sw128(slot + SLOT_M + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                const uint64_t bs = sdesc_sw128(sbase + SC_SB + ks * 2048, 16384, 1024);
-                mma_bf16(tm + SC_S, am, bs, idM, 1);
-                const uint64_t bq = sdesc_sw128(slot + SLOT_Q + ks * 2048, 8192, 1024);
-                mma_bf16(d_o, bs, bq, idO1, ks > 0);
+                const uint64_t b1 =
+                    sdesc_sw128(slot + SLOT_B1 + (ks >> 2) * (B1_ROWS * 128) + (ks & 3) * 32, 16, 1024);
+                mma_bf16_ts(tm + rg + SC_OT, tm + SC_SA + ks * 8, b1, id1, 1);
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ak = sdesc_sw128(slot + SLOT_KT + ks * 2048, 8192, 1024);
-                const uint64_t uu = sdesc_sw128(slot + SLOT_U + ks * 32, 16, 1024);
-                mma_bf16(tm + SC_S, ak, uu, idK, 1);
+                const uint64_t au = sdesc_sw128(slot + SLOT_U + ks * 32, 16, 1024);
+                const uint64_t bk = sdesc_sw128(slot + SLOT_KT + ks * 2048, 8192, 1024);
+                mma_bf16(tm + rg + SC_ST, au, bk, idS, 1);
                 const uint64_t bp = sdesc_sw128(slot + SLOT_P + ks * 32, 16, 1024);
-                mma_bf16(d_o, uu, bp, idO2, 1);
+                mma_bf16(tm + rg + SC_OT, au, bp, idO, 1);
             }
             mma_commit(&ms.bar_mma);
         }
-        if (n > 0 && warp < 4) store_o(n - 1);  // overlaps this chunk's MMAs (other TMEM columns)
+        if (n > 0 && warp < 4) store_o(n - 1);  // overlaps this chunk's MMAs (the other region)
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
         if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
     }
     if (!timed_out && NC > 0 && warp < 4) store_o(NC - 1);
     if (!timed_out && p.S_T) {
+        const uint32_t rg_last = SC_REG * (uint32_t)((NC + 1) & 1);  // region of chunk NC - 1 (region 1 if NC = 0)
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
-            const int j0 = colhalf * 64 + q2 * 32;
+            const int cb = c0 + q2 * 32;
             float sv[32];
-            tmem_ld32(tm_lane + SC_S + j0, sv);
-            float *dst = p.S_T + ((size_t)bh * DK + row) * DV + j0;
+            tmem_ld32(tm_lane + rg_last + SC_ST + cb, sv);
+            float *dst = p.S_T + ((size_t)bh * DK + cb) * DV + j;
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(dst + i) = make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3]);
+            for (int i = 0; i < 32; ++i) dst[(size_t)i * DV] = sv[i];
         }
     }
     if (tid == 0) bulk_wait_group0();
