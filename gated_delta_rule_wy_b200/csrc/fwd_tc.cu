@@ -30,12 +30,15 @@
 // per-channel reference g_I, the cumulative decay at the midpoint of the
 // 32-token half-chunk I that holds t:
 //   L_t = x_t exp(G_t - g_I),   R_i = k_i exp(g_I - G_i).
-// Each factor stays within exp(+-80) unless a half-chunk's decay spans more
-// than 160 nepers; a factor that underflows only loses terms whose true value
-// is itself below fp32 range. When the guard trips (alpha near 0 over a whole
-// half-chunk, e.g. a reset) the chunk takes an exact path: A and P with one
-// exponential per (t, i, c), and the decay-weighted operands from exp(G)
-// directly.
+// The guard requires |G_t - g_I| <= 70 for every token against its own
+// half's reference. Keys of the first half also meet second-half rows, through
+// R1_i = k_i exp(g_1 - G_i), formed with one exponential: if it underflows
+// (g_1 - G_i < -87), every product it enters has G_t - G_i = (G_t - g_1) +
+// (g_1 - G_i) < 70 - 87, so only terms below exp(-17) are lost; the same bound
+// covers the other factors that can underflow (exp(g_I), exp(G_C - g_I)).
+// When the guard trips (alpha near 0 over much of a chunk, e.g. a reset) the
+// chunk takes an exact path: A and P with one exponential per (t, i, c), and
+// the decay-weighted operands from exp(G) directly.
 //
 // Tensor-core mapping (M = 128 everywhere; t, i, s tokens, c key channel,
 // j value channel; accumulators fp32 in TMEM, operands bf16 in
@@ -66,7 +69,7 @@ constexpr int DK = 128;
 constexpr int DV = 128;
 constexpr int NT = 256;                           // 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr float kFactorLimit = 80.f;              // |exponent| of one decay factor
+constexpr float kFactorLimit = 70.f;              // |exponent| of one decay factor
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_STG_Q = 0;       // q  [64][128] bf16
@@ -302,24 +305,33 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
             const __nv_bfloat16 *vs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_V);
             const __nv_bfloat16 *ws = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_W);
-            float egI[8], kcf[8], r10[8], gr[8];
+            float egI[8], kcf[8], gr[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
                 gr[x] = HI ? g1[x] : g0[x];
                 egI[x] = __expf(gr[x]);          // exp(g_I)
                 kcf[x] = __expf(gC[x] - gr[x]);  // exp(G_C - g_I)
-                r10[x] = __expf(g1[x] - g0[x]);  // exp(g_1 - g_0)
             }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int t = tg * 4 + m;
-                float qv[8], kv[8], bv[8], vv[8], wv[8];
+                float qv[8], kv[8], bv[8];
                 unpack8(*reinterpret_cast<const uint4 *>(qs + t * DK + o8 * 8), qv);
                 unpack8(*reinterpret_cast<const uint4 *>(ks + t * DK + o8 * 8), kv);
                 unpack8(*reinterpret_cast<const uint4 *>(bs + t * DK + o8 * 8), bv);
-                unpack8(*reinterpret_cast<const uint4 *>(vs + t * DV + o8 * 8), vv);
-                unpack8(*reinterpret_cast<const uint4 *>(ws + t * DV + o8 * 8), wv);
-                float le[8], lq[8], r[8], kt[8], qh[8], z[8];
+                // z = w (.) v in bf16 pairs: the product of two bf16 values is exact in fp32,
+                // so one rounding to bf16 gives the same value as the fp32 route
+                uint4 z;
+                {
+                    const uint4 vr = *reinterpret_cast<const uint4 *>(vs + t * DV + o8 * 8);
+                    const uint4 wr = *reinterpret_cast<const uint4 *>(ws + t * DV + o8 * 8);
+                    const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+                    const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&wr);
+                    __nv_bfloat162 *z2 = reinterpret_cast<__nv_bfloat162 *>(&z);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) z2[x] = __hmul2(w2[x], v2[x]);
+                }
+                float le[8], lq[8], r[8], kt[8], qh[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
                     const float d = G[m][x] - gr[x];
@@ -330,22 +342,23 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     r[x] = kv[x] * yr;
                     kt[x] = r[x] * kcf[x];
                     qh[x] = lq[x] * egI[x];
-                    z[x] = wv[x] * vv[x];
                 }
                 const int tl = t - 32 * HI;  // token within its half-chunk
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + tl, o8, 128)) = pack8(le);
                 *reinterpret_cast<uint4 *>(sm + OFF_STACK + sw_chunk(64 * HI + 32 + tl, o8, 128)) = pack8(lq);
                 if (HI == 0) {
                     *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(t, o8, R_ROWS)) = pack8(r);
+                    // R_1 row of a first-half key: one exponential, exp(g_1 - G_i), so that no
+                    // intermediate factor (such as exp(g_1 - g_0) alone) can underflow
                     float r1[8];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) r1[x] = r[x] * r10[x];
+                    for (int x = 0; x < 8; ++x) r1[x] = kv[x] * __expf(g1[x] - G[m][x]);
                     *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(32 + t, o8, R_ROWS)) = pack8(r1);
                 } else {
                     *reinterpret_cast<uint4 *>(sm + OFF_R0 + sw_chunk(32 + t, o8, R_ROWS)) = pack8(r);
                 }
                 *reinterpret_cast<uint4 *>(sm + OFF_KT + sw_chunk(t, o8, 64)) = pack8(kt);
-                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = pack8(z);
+                *reinterpret_cast<uint4 *>(sm + OFF_Z + sw_chunk(t, o8, 64)) = z;
                 *reinterpret_cast<uint4 *>(sm + OFF_QH + sw_chunk(t, o8, 64)) = pack8(qh);
             }
         }
@@ -914,6 +927,10 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
                 v[i] = p.S0 ? p.S0[((size_t)bh * DK + c0 + q2 * 32 + i) * DV + j] : 0.f;
             tmem_st32(tm_lane + SC_REG + SC_ST + c0 + q2 * 32, v);
         }
+        float zz[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) zz[i] = 0.f;
+        tmem_st32(tm_lane + SC_OT + colhalf * 32, zz);  // chunk 0's O^T starts at zero
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -950,38 +967,42 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         }
     };
 
-    for (int n = 0; n < NC; ++n) {
+    if (NC > 0 && !wait_bar(&ms.bar_full[0], ph_full[0])) timed_out = true;
+    for (int n = 0; n < NC && !timed_out; ++n) {
         const int sl = n & 1;
         const uint32_t slot = sbase + (sl ? SC_SLOT1 : SC_SLOT0);
         const uint32_t rg = SC_REG * (uint32_t)sl, rg_prev = SC_REG * (uint32_t)(sl ^ 1);
-        if (!wait_bar(&ms.bar_full[sl], ph_full[sl])) { timed_out = true; break; }
-        // ---- S^T (previous region) -> bf16 operand; gamma-scaled S^T -> this region; O^T <- 0 ----
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            const int cb = c0 + q2 * 32;
-            float sv[32];
-            tmem_ld32(tm_lane + rg_prev + SC_ST + cb, sv);
+        // ---- S^T (previous region) -> bf16 operand; gamma-scaled S^T -> this region ----
+        {
+            float s0[32], s1[32];
+            tmem_ld32x2(tm_lane + rg_prev + SC_ST + c0, tm_lane + rg_prev + SC_ST + c0 + 32, s0, s1);
             if (p.saved_states) {
-                float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + cb) * DV + j;
+                float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c0) * DV + j;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) dst[(size_t)i * DV] = sv[i];
+                for (int i = 0; i < 32; ++i) {
+                    dst[(size_t)i * DV] = s0[i];
+                    dst[(size_t)(32 + i) * DV] = s1[i];
+                }
             }
-            uint32_t pk[16];
+            uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                __nv_bfloat162 hv = __floats2bfloat162_rn(sv[2 * i], sv[2 * i + 1]);
-                pk[i] = *reinterpret_cast<uint32_t *>(&hv);
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(s0[2 * i], s0[2 * i + 1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(s1[2 * i], s1[2 * i + 1]);
+                pk[i] = *reinterpret_cast<uint32_t *>(&h0);
+                pk[16 + i] = *reinterpret_cast<uint32_t *>(&h1);
             }
-            tmem_st16u(tm_lane + SC_SA + (uint32_t)(cb >> 1), pk);
+            tmem_st32u_nw(tm_lane + SC_SA + (uint32_t)(c0 >> 1), pk);
+            const float4 *g4 = reinterpret_cast<const float4 *>(&ms.gam[sl][c0]);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] *= ms.gam[sl][cb + i];
-            tmem_st32(tm_lane + rg + SC_ST + cb, sv);
-        }
-        {
-            float zz[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) zz[i] = 0.f;
-            tmem_st32(tm_lane + rg + SC_OT + colhalf * 32, zz);
+            for (int i = 0; i < 8; ++i) {
+                const float4 ga = g4[i], gb = g4[8 + i];
+                s0[4 * i] *= ga.x; s0[4 * i + 1] *= ga.y; s0[4 * i + 2] *= ga.z; s0[4 * i + 3] *= ga.w;
+                s1[4 * i] *= gb.x; s1[4 * i + 1] *= gb.y; s1[4 * i + 2] *= gb.z; s1[4 * i + 3] *= gb.w;
+            }
+            tmem_st32_nw(tm_lane + rg + SC_ST + c0, s0);
+            tmem_st32_nw(tm_lane + rg + SC_ST + c0 + 32, s1);
+            tmem_wait_st();
         }
         tc_fence_before_sync();
         __syncthreads();
@@ -1007,9 +1028,30 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
             }
             mma_commit(&ms.bar_mma);
         }
-        if (n > 0 && warp < 4) store_o(n - 1);  // overlaps this chunk's MMAs (the other region)
-        if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
-        tc_fence_after_sync();
+        if (warp < 4) {
+            // overlaps this chunk's MMAs (the other region), then clears that region's O^T
+            // for chunk n + 1 (each thread rewrites only the lane it has just read)
+            if (n > 0) store_o(n - 1);
+            float zz[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) zz[i] = 0.f;
+            tmem_st32_nw(tm_lane + rg_prev + SC_OT, zz);
+            tmem_st32_nw(tm_lane + rg_prev + SC_OT + 32, zz);
+            tmem_wait_st();
+        }
+        // the next slot (issued two chunks ago) and this chunk's MMAs, one barrier for both
+        {
+            bool ok = true;
+            if (n + 1 < NC) {
+                ok = mbar_wait_bounded(&ms.bar_full[sl ^ 1], ph_full[sl ^ 1], kWaitLimitNs);
+                ph_full[sl ^ 1] ^= 1u;
+            }
+            ok = mbar_wait_bounded(&ms.bar_mma, ph_mma, kWaitLimitNs) && ok;
+            ph_mma ^= 1u;
+            tc_fence_before_sync();
+            if (__syncthreads_or(!ok)) { timed_out = true; break; }
+            tc_fence_after_sync();
+        }
         if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
     }
     if (!timed_out && NC > 0 && warp < 4) store_o(NC - 1);

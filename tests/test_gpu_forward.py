@@ -84,7 +84,7 @@ def _edit(x: I.FwdInputs, **fields) -> I.FwdInputs:
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("case", ["reset", "no_erase", "full_erase", "erase_range_2", "no_decay",
-                                  "strong_decay", "one_hot_keys", "kda_gates"])
+                                  "strong_decay", "decay_cliff", "one_hot_keys", "kda_gates"])
 def test_degenerate_cases(dtype, case):
     x = I.make_forward_inputs(B=1, H=2, T=160, dk=128, dv=128, dtype=dtype, decay_shift=1.0, seed=5, with_S0=True)
     la, b, k, w = x.log_alpha.clone(), x.b.clone(), x.k.clone(), x.w.clone()
@@ -100,6 +100,16 @@ def test_degenerate_cases(dtype, case):
         la.zero_()
     elif case == "strong_decay":  # alpha ~ 1e-13 per token: exercises the decay-range handling
         la = la - 30.0
+    elif case == "decay_cliff":
+        # per 64-token chunk: no decay to token 15, -30 nepers over tokens 16..31, none over
+        # 32..39, -69.5 over 40..47, none after. Every token is within 70 nepers of its own
+        # half-chunk's midpoint, the two midpoints are ~100 nepers apart (a factor
+        # exp(g_1 - g_0) alone underflows), and the products exp(G_t - G_i), t in 32..39,
+        # i near 31, are O(1).
+        prof = torch.zeros(64)
+        prof[16:32] = -30.0 / 16
+        prof[40:48] = -69.5 / 8
+        la = prof.repeat(3)[:la.shape[1]][None, :, None, None].expand_as(la).contiguous()
     elif case == "one_hot_keys":
         k = torch.nn.functional.one_hot(torch.randint(0, 128, k.shape[:-1], generator=torch.Generator().manual_seed(0)),
                                         128).to(dtype)
