@@ -53,6 +53,7 @@
 // frees its TMEM and exits.
 
 #include <cuda.h>
+#include <cstddef>
 #include <mutex>
 
 #include "gdr2_common.cuh"
@@ -111,6 +112,7 @@ struct Misc {
     float eg1[DK];   // ... of half-chunk 1: exp(g_1)
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
+static_assert(offsetof(Misc, gC) % 16 == 0, "per-channel vectors are 16-byte aligned");
 
 // Offset of the 16-byte chunk holding columns [8*o8, 8*o8 + 8) of `row`.
 __device__ __forceinline__ uint32_t sw_chunk(int row, int o8, int rows)
@@ -860,9 +862,10 @@ struct ScanMisc {
     uint64_t bar_mma;
     uint32_t tmem_base;
     int pad;
-    float gam[2][DK];
+    alignas(16) float gam[2][DK];  // bulk-copy destination and float4 reads: 16-byte aligned
 };
 static_assert(sizeof(ScanMisc) <= 1280, "scan misc region");
+static_assert(offsetof(ScanMisc, gam) % 16 == 0, "gamma rows are 16-byte aligned");
 
 struct ScanParams {
     int B, T, H, NC, ntasks;
