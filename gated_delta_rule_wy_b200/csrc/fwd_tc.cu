@@ -247,7 +247,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int Cn = min(C, p.T - n * C);
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
-        if (tid == 0) bulk_wait_group_read1();  // K~ and P of the previous task have left shared memory
+        if (tid == 64) bulk_wait_group_read0();  // K~ and P of the previous task have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
@@ -365,8 +365,6 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         const bool exact = __syncthreads_or(risky) != 0;
-        // the staging buffers are free once the operands are built: prefetch the next task
-        if (!exact && tid == 32 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
         if (exact) {
             // ---- exact path: G to shared memory, pairwise exponentials ----
             float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
@@ -441,7 +439,6 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             fence_proxy_async_smem();  // P and K~ -> the bulk stores below
             __syncthreads();
-            if (tid == 32 && task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
         } else {
             // ---- tensor-core path: [A;P] = STACK R_I^T ----
             mma_sync_point();
@@ -529,8 +526,10 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tc_fence_before_sync();
             __syncthreads();
         }
-        // K~ and P are final: copy them to the slot in the background
-        if (tid == 0) {
+        // The staging buffers are free: prefetch the next task. K~ and P are final: copy them to
+        // the slot in the background. Both are issued from warp 2, idle in the first solve levels.
+        if (tid == 64) {
+            if (task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
             bulk_store(slot + SLOT_KT, sm + OFF_KT, 16384);
             bulk_store(slot + SLOT_P, sm + OFF_P, 8192);
             bulk_commit_group();
@@ -834,7 +833,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bulk_commit_group();
         }
     }
-    if (tid == 0) bulk_wait_group0();
+    if (tid == 0 || tid == 64) bulk_wait_group0();  // each waits for the bulk groups it committed
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
