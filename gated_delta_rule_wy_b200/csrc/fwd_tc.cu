@@ -247,7 +247,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int Cn = min(C, p.T - n * C);
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
-        if (tid == 64) bulk_wait_group_read0();  // K~ and P of the previous task have left shared memory
+        if (tid == 64) bulk_wait_group_read0();  // K~, P and U~ of the previous task have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
@@ -286,7 +286,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ms.eg0[c] = __expf(g0);
             ms.eg1[c] = __expf(g1);
         }
-        if (tid == 0) bulk_wait_group_read0();  // ... and [Q'; M], U~ too, before the operands are rebuilt
+        if (tid == 0) bulk_wait_group_read0();  // ... and [Q'; M] too, before the operands are rebuilt
         __syncthreads();
         bool risky = false;
         float g0[8], g1[8], gC[8];
@@ -779,6 +779,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         mma_sync_point();
+        // U~^T is staged: to the slot in the background (from warp 2, which has nothing to issue)
+        if (tid == 64) {
+            bulk_store(slot + SLOT_U, sm + OFF_Z, 16384);
+            bulk_commit_group();
+        }
         // ================= Q' - Q^ = -P W (M = 64) ;  M = -K~^T W =================
         if (tid == 0) {
             const uint32_t idQ = idesc_bf16(64, 128, false, false, true);
@@ -824,12 +829,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (tid < DK) reinterpret_cast<float *>(p.ws + (size_t)p.ntasks * SLOT_BYTES + (size_t)task * GAMMA_BYTES)[tid] =
             ms.gC[tid];
-        fence_proxy_async_smem();  // [Q'; M] and U~^T -> the bulk stores below
+        fence_proxy_async_smem();  // [Q'; M] -> the bulk store below
         tc_fence_before_sync();
         __syncthreads();  // every TMEM read of this task is done before the next task's MMAs
         if (tid == 0) {
             bulk_store(slot + SLOT_B1, sm + OFF_STACK, 2 * B1_ROWS * 128);
-            bulk_store(slot + SLOT_U, sm + OFF_Z, 16384);
             bulk_commit_group();
         }
     }
