@@ -18,8 +18,9 @@ The JSON line carries:
                        copy of o and S_T, all inside the timed region
   roofline             HBM roofline of the forward kernel (algorithmic bytes / time)
   tensor               algorithmic FLOP/s against the dense bf16 peak
-  components           decode step (256 seq x 16 heads, fp32 state) and backward
-                       (B=2, T=4096) timings with their own rooflines
+  components           decode step (256 seq x 16 heads, fp32 state), backward
+                       (B=2, T=4096) and the sequence-length sweep (65,536 tokens
+                       per call, T = 2048 .. 32768), each with its own figures
   cpu_baseline         the fp64 oracle on the host cores (rank 0, N = 1)
   clocks               SM clocks and throttle reasons sampled during the timed region
 `--impl reference` times the oracle itself on the same workload (sampled heads).
@@ -288,6 +289,29 @@ def bench_components(dev, stream, peaks):
     t = statistics.median(ms)
     out["backward"] = {"workload": "B=2 H=16 T=4096 d=128 bf16, saved chunk states",
                        "ms_per_call": t, "tokens_per_s": cfg["B"] * cfg["T"] / (t * 1e-3)}
+    del x, dO, saved
+    # sequence-length sweep: 65,536 tokens per call at every T (B = 65536 / T), C1 laws
+    from gated_delta_rule_wy_b200 import gdr2_forward_workspace_bytes
+    sweep = []
+    for T in I.SWEEP_T:
+        c = I.sweep_config(T)
+        xs = I.make_forward_inputs(**c).to(dev)
+        o = torch.empty_like(xs.v)
+        ws = torch.empty(gdr2_forward_workspace_bytes(c["B"], c["T"], c["H"], c["dk"], c["dv"], c["dtype"]),
+                         dtype=torch.uint8, device=dev)
+
+        def fwd():
+            gdr2_forward(xs.q, xs.k, xs.v, xs.log_alpha, xs.b, xs.w, None, out=o, workspace=ws)
+
+        for _ in range(3):
+            fwd()
+        ms = statistics.median(time_steps(fwd, 10, stream))
+        tokens = c["B"] * T
+        alg = tokens * c["H"] * BYTES_PER_TOKEN_HEAD + c["B"] * c["H"] * c["dk"] * c["dv"] * 4
+        sweep.append({"T": T, "B": c["B"], "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3),
+                      "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+        del xs, o, ws
+    out["sweep"] = {"workload": "65,536 tokens per call, H=16, d=128, bf16, T = 2048 .. 32768", "points": sweep}
     return out
 
 

@@ -220,6 +220,9 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, h, t0, bb);
     };
     if (tid == 0 && (int)blockIdx.x < p.ntasks) issue_loads(blockIdx.x);
+    // the scan kernel may be scheduled now: its CTAs take an SM only once this (persistent) CTA
+    // has left it, and they read the workspace only after this whole grid has completed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     uint32_t ph_tma = 0, ph_mma = 0;
     bool timed_out = false;
@@ -911,6 +914,10 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
     const int j = quarter * 32 + lane;  // this thread's TMEM lane = value channel
 
+    // Launched as a programmatic dependent of the chunk kernel: everything above overlaps its
+    // tail; the workspace is read only after that grid has completed and flushed its memory.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     auto issue_slot = [&](int n) {
         const int sl = n & 1;
         const size_t task = (size_t)bh * NC + n;
@@ -1154,8 +1161,17 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     ScanParams sp{a.B, a.T, a.H, NC, ntasks, static_cast<const unsigned char *>(a.workspace), a.S0, a.S_T,
                   a.saved_states, a.status};
-    fwd_scan_kernel<<<a.B * a.H, NT, SC_SMEM_BYTES, s>>>(mo, sp);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * a.H);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = SC_SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fwd_scan_kernel, mo, sp);
 }
 
 }  // namespace gdr2
