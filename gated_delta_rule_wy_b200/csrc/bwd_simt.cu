@@ -12,15 +12,19 @@
 //   dSb  = dS - e ddelta^T   dlog_alpha = rowsum(dSb (.) Sb)
 //   dS   = Diag(a) dSb
 //
-// Schedule: one CTA per (batch, head). The states entering each chunk of 64
-// tokens come from the forward (saved_states) or from a forward sweep here.
-// For each chunk, last to first, the CTA replays the chunk forward from its
-// entry state, keeping every token's state and delta in the workspace, then
-// walks the chunk backwards. dS lives in registers: thread (c, half) owns the
-// half row dS[c, half*dv/2 : (half+1)*dv/2]. Row reductions (over value
-// columns) finish with one shuffle between the two halves; column
-// reductions (over key channels) use a shuffle transpose-reduce inside a
-// warp, then shared memory across warps.
+// Schedule: the columns of S (and of dS) evolve independently, so one CTA
+// owns (batch, head, block of JB = 32 value columns). The states entering each
+// chunk of 64 tokens come from the forward (saved_states) or from a forward
+// sweep here. For each chunk, last to first, the CTA replays the chunk forward
+// from its entry state, keeping every token's state block and delta in the
+// workspace, then walks the chunk backwards. Thread (c, half) owns the 16
+// columns half*16 .. +15 of row c of the block in registers. Column
+// reductions (over key channels) finish inside the CTA (a shuffle
+// transpose-reduce in each warp, then shared memory across warps); the
+// per-key-channel gradients dq, dk, de = dk's erase part and dlog_alpha are
+// partial sums over the block's columns, added into fp32 accumulators with
+// atomics; a finishing kernel forms dk = dk' + de (.) b, db = de (.) k and
+// converts to the output types.
 
 #include <mutex>
 
@@ -35,10 +39,16 @@ constexpr int C = 64;
 
 __host__ __device__ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr int JB = 32;  // value columns per CTA
+
 struct BwdLayout {
-    size_t cs_off, ts_off, dl_off, total;
+    size_t cs_off, ts_off, dl_off, acc_off, total;
 };
 
+// cs: chunk-entry states [BH][NC][dk][dv] (only without saved_states);
+// ts: per-CTA token states of one chunk [BH * NJ][C + 1][dk][JB];
+// dl: per-CTA deltas of one chunk [BH * NJ][C][JB];
+// acc: fp32 accumulators dq, dk', de, dlog_alpha, each [B][T][H][dk].
 __host__ __device__ inline BwdLayout bwd_layout(int B, int T, int H, int dk, int dv, bool need_cs)
 {
     const size_t BH = (size_t)B * H;
@@ -51,6 +61,8 @@ __host__ __device__ inline BwdLayout bwd_layout(int B, int T, int H, int dk, int
     off += align256(BH * (C + 1) * dk * dv * sizeof(float));
     L.dl_off = off;
     off += align256(BH * C * dv * sizeof(float));
+    L.acc_off = off;
+    off += align256(4 * (size_t)B * T * H * dk * sizeof(float));
     L.total = off;
     return L;
 }
@@ -73,14 +85,14 @@ __device__ __forceinline__ void transpose_reduce16(float (&vals)[N], int lane)
     }
 }
 
-template <int DK, int DV>
+template <int DK>
 struct BwdSmem {
-    float red[2 * DK / 32][DV];  // per-warp column partials
-    float vec[DV];               // reduced column vector (delta or ddelta)
-    float z[DV], dO[DV], v[DV], w[DV];
+    float red[2 * DK / 32][JB];  // per-warp column partials
+    float vec[JB];               // reduced column vector (delta or ddelta)
+    float z[JB], dO[JB], v[JB], w[JB];
 };
 
-template <typename TIn, int DK, int DV>
+template <typename TIn, int DK>
 __device__ __forceinline__ void load_row_gates(const BwdArgs &a, size_t ok, int c, float &kc, float &bc,
                                                float &al)
 {
@@ -89,30 +101,27 @@ __device__ __forceinline__ void load_row_gates(const BwdArgs &a, size_t ok, int 
     al = expf(clamp_log_alpha(a.log_alpha[ok + c]));
 }
 
-// One forward token on the register row S (this thread's half row). Leaves
-// delta in sm.vec and writes it to dl (when not null).
+// One forward token on this thread's 16 columns of row c (columns j0 + jb ..).
+// Leaves delta (the block's JB columns) in sm.vec and writes it to dl when not null.
 template <typename TIn, int DK, int DV>
-__device__ __forceinline__ void fwd_token(const BwdArgs &a, BwdSmem<DK, DV> &sm, float (&S)[DV / 2], int t,
-                                          int c, int jb, int lane, int warp, int tid, float *dl)
+__device__ __forceinline__ void fwd_token(const BwdArgs &a, BwdSmem<DK> &sm, float (&S)[JB / 2], int t, int bb,
+                                          int h, int j0, int c, int jb, int lane, int warp, int tid, float *dl)
 {
-    constexpr int HJ = DV / 2;
-    const int bb = blockIdx.x / a.H, h = blockIdx.x % a.H;
+    constexpr int HJ = JB / 2;
     const size_t ok = (((size_t)bb * a.T + t) * a.H + h) * DK;
-    const size_t ov = (((size_t)bb * a.T + t) * a.H + h) * DV;
-    if (tid < DV)
+    const size_t ov = (((size_t)bb * a.T + t) * a.H + h) * DV + j0;
+    if (tid < JB)
         sm.z[tid] = to_f32(static_cast<const TIn *>(a.w)[ov + tid]) * to_f32(static_cast<const TIn *>(a.v)[ov + tid]);
     float kc, bc, al;
-    load_row_gates<TIn, DK, DV>(a, ok, c, kc, bc, al);
+    load_row_gates<TIn, DK>(a, ok, c, kc, bc, al);
     const float ae = al * bc * kc;
     float part[HJ];
 #pragma unroll
     for (int j = 0; j < HJ; ++j) part[j] = ae * S[j];
     transpose_reduce16<HJ>(part, lane);
-    constexpr int PER = HJ / 16;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) sm.red[warp][jb + PER * (lane & 15) + i] = part[i];
+    sm.red[warp][jb + (lane & 15)] = part[0];
     __syncthreads();
-    if (tid < DV) {
+    if (tid < JB) {
         float r = 0.f;
 #pragma unroll
         for (int wv = 0; wv < 2 * DK / 32; ++wv) r += sm.red[wv][tid];
@@ -126,24 +135,28 @@ __device__ __forceinline__ void fwd_token(const BwdArgs &a, BwdSmem<DK, DV> &sm,
 }
 
 template <typename TIn, int DK, int DV>
-__global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, float *TS, float *DL)
+__global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, float *TS, float *DL, float *ACC)
 {
-    constexpr int NT = 2 * DK;
-    constexpr int HJ = DV / 2;
-    constexpr int PER = HJ / 16;
-    __shared__ BwdSmem<DK, DV> sm;
+    constexpr int HJ = JB / 2;
+    constexpr int NJ = DV / JB;
+    static_assert(HJ == 16, "one transpose-reduce step per column");
+    __shared__ BwdSmem<DK> sm;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c = warp * 16 + (lane & 15);
     const int half = lane >> 4;
-    const int jb = half * HJ;
-    const int bh = blockIdx.x;
+    const int jb = half * HJ;            // this thread's first column within the block
+    const int bh = blockIdx.x / NJ;
+    const int j0 = (blockIdx.x % NJ) * JB;  // the block's first value column
     const int bb = bh / a.H, h = bh % a.H;
     const int T = a.T, H = a.H;
     const int NC = (T + C - 1) / C;
-    const size_t SS = (size_t)DK * DV;
-    float *ts = TS + (size_t)bh * (C + 1) * SS;
-    float *dl = DL + (size_t)bh * C * DV;
-    (void)NT;
+    const size_t SS = (size_t)DK * DV;        // one full state
+    const size_t BS = (size_t)DK * JB;        // one state block
+    const size_t nacc = (size_t)a.B * T * H * DK;
+    float *ts = TS + (size_t)blockIdx.x * (C + 1) * BS;
+    float *dl = DL + (size_t)blockIdx.x * C * JB;
+    float *acc_dq = ACC, *acc_dk = ACC + nacc, *acc_de = ACC + 2 * nacc, *acc_dla = ACC + 3 * nacc;
+    const size_t srow = (size_t)c * DV + j0 + jb;  // this thread's columns in a full state
 
     float S[HJ];
     // ---- states entering each chunk ----
@@ -153,34 +166,34 @@ __global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, fl
     } else {
         float *cs = CS + (size_t)bh * NC * SS;
 #pragma unroll
-        for (int j = 0; j < HJ; ++j) S[j] = a.S0 ? a.S0[(size_t)bh * SS + (size_t)c * DV + jb + j] : 0.f;
+        for (int j = 0; j < HJ; ++j) S[j] = a.S0 ? a.S0[(size_t)bh * SS + srow + j] : 0.f;
         for (int t = 0; t < T; ++t) {
             if (t % C == 0) {
 #pragma unroll
-                for (int j = 0; j < HJ; ++j) cs[(size_t)(t / C) * SS + (size_t)c * DV + jb + j] = S[j];
+                for (int j = 0; j < HJ; ++j) cs[(size_t)(t / C) * SS + srow + j] = S[j];
             }
-            fwd_token<TIn, DK, DV>(a, sm, S, t, c, jb, lane, warp, tid, nullptr);
+            fwd_token<TIn, DK, DV>(a, sm, S, t, bb, h, j0, c, jb, lane, warp, tid, nullptr);
         }
         chunk_states = cs;
     }
 
     float dS[HJ];
 #pragma unroll
-    for (int j = 0; j < HJ; ++j) dS[j] = a.dS_T ? a.dS_T[(size_t)bh * SS + (size_t)c * DV + jb + j] : 0.f;
+    for (int j = 0; j < HJ; ++j) dS[j] = a.dS_T ? a.dS_T[(size_t)bh * SS + srow + j] : 0.f;
 
     for (int n = NC - 1; n >= 0; --n) {
         const int t0 = n * C;
         const int Cn = min(C, T - t0);
-        // ---- replay the chunk forward, keeping every state and delta ----
+        // ---- replay the chunk forward, keeping every state block and delta ----
 #pragma unroll
         for (int j = 0; j < HJ; ++j) {
-            S[j] = chunk_states[(size_t)n * SS + (size_t)c * DV + jb + j];
-            ts[(size_t)c * DV + jb + j] = S[j];
+            S[j] = chunk_states[(size_t)n * SS + srow + j];
+            ts[(size_t)c * JB + jb + j] = S[j];
         }
         for (int t = 0; t < Cn; ++t) {
-            fwd_token<TIn, DK, DV>(a, sm, S, t0 + t, c, jb, lane, warp, tid, dl + (size_t)t * DV);
+            fwd_token<TIn, DK, DV>(a, sm, S, t0 + t, bb, h, j0, c, jb, lane, warp, tid, dl + (size_t)t * JB);
 #pragma unroll
-            for (int j = 0; j < HJ; ++j) ts[(size_t)(t + 1) * SS + (size_t)c * DV + jb + j] = S[j];
+            for (int j = 0; j < HJ; ++j) ts[(size_t)(t + 1) * BS + (size_t)c * JB + jb + j] = S[j];
         }
         // Each thread reads back only the rows and deltas it wrote itself.
         __syncthreads();
@@ -188,20 +201,20 @@ __global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, fl
         for (int t = Cn - 1; t >= 0; --t) {
             const int tg = t0 + t;
             const size_t ok = (((size_t)bb * T + tg) * H + h) * DK;
-            const size_t ov = (((size_t)bb * T + tg) * H + h) * DV;
-            if (tid < DV) {
+            const size_t ov = (((size_t)bb * T + tg) * H + h) * DV + j0;
+            if (tid < JB) {
                 sm.dO[tid] = to_f32(static_cast<const TIn *>(a.dO)[ov + tid]);
                 sm.v[tid] = to_f32(static_cast<const TIn *>(a.v)[ov + tid]);
                 sm.w[tid] = to_f32(static_cast<const TIn *>(a.w)[ov + tid]);
-                sm.vec[tid] = dl[(size_t)t * DV + tid];  // delta_t
+                sm.vec[tid] = dl[(size_t)t * JB + tid];  // delta_t
             }
             const float qc = to_f32(static_cast<const TIn *>(a.q)[ok + c]);
             float kc, bc, al;
-            load_row_gates<TIn, DK, DV>(a, ok, c, kc, bc, al);
+            load_row_gates<TIn, DK>(a, ok, c, kc, bc, al);
             const float ec = bc * kc;
             __syncthreads();
-            const float *St = ts + (size_t)(t + 1) * SS + (size_t)c * DV + jb;
-            const float *Sp = ts + (size_t)t * SS + (size_t)c * DV + jb;
+            const float *St = ts + (size_t)(t + 1) * BS + (size_t)c * JB + jb;
+            const float *Sp = ts + (size_t)t * BS + (size_t)c * JB + jb;
             float dq = 0.f, dk = 0.f;
             float part[HJ];
 #pragma unroll
@@ -213,10 +226,9 @@ __global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, fl
                 part[j] = dS[j] * kc;
             }
             transpose_reduce16<HJ>(part, lane);
-#pragma unroll
-            for (int i = 0; i < PER; ++i) sm.red[warp][jb + PER * (lane & 15) + i] = part[i];
+            sm.red[warp][jb + (lane & 15)] = part[0];
             __syncthreads();
-            if (tid < DV) {
+            if (tid < JB) {
                 float dd = 0.f;
 #pragma unroll
                 for (int wv = 0; wv < 2 * DK / 32; ++wv) dd += sm.red[wv][tid];
@@ -240,17 +252,33 @@ __global__ void __launch_bounds__(2 * DK, 1) bwd_kernel(BwdArgs a, float *CS, fl
             de += __shfl_xor_sync(0xffffffffu, de, 16);
             dla += __shfl_xor_sync(0xffffffffu, dla, 16);
             if (half == 0) {
-                static_cast<TIn *>(a.gq)[ok + c] = from_f32<TIn>(dq);
-                static_cast<TIn *>(a.gk)[ok + c] = from_f32<TIn>(fmaf(de, bc, dk));
-                static_cast<TIn *>(a.gb)[ok + c] = from_f32<TIn>(de * kc);
-                a.glog_alpha[ok + c] = dla;
+                atomicAdd(acc_dq + ok + c, dq);
+                atomicAdd(acc_dk + ok + c, dk);
+                atomicAdd(acc_de + ok + c, de);
+                atomicAdd(acc_dla + ok + c, dla);
             }
             __syncthreads();
         }
     }
     if (a.gS0) {
 #pragma unroll
-        for (int j = 0; j < HJ; ++j) a.gS0[(size_t)bh * SS + (size_t)c * DV + jb + j] = dS[j];
+        for (int j = 0; j < HJ; ++j) a.gS0[(size_t)bh * SS + srow + j] = dS[j];
+    }
+}
+
+// dq = sum of the blocks' dq; dk = dk' + de (.) b; db = de (.) k; dlog_alpha, all per key channel.
+template <typename TIn>
+__global__ void bwd_finish_kernel(BwdArgs a, const float *ACC, size_t n)
+{
+    const float *acc_dq = ACC, *acc_dk = ACC + n, *acc_de = ACC + 2 * n, *acc_dla = ACC + 3 * n;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const float kc = to_f32(static_cast<const TIn *>(a.k)[i]);
+        const float bc = to_f32(static_cast<const TIn *>(a.b)[i]);
+        const float de = acc_de[i];
+        static_cast<TIn *>(a.gq)[i] = from_f32<TIn>(acc_dq[i]);
+        static_cast<TIn *>(a.gk)[i] = from_f32<TIn>(fmaf(de, bc, acc_dk[i]));
+        static_cast<TIn *>(a.gb)[i] = from_f32<TIn>(de * kc);
+        a.glog_alpha[i] = acc_dla[i];
     }
 }
 
@@ -259,9 +287,18 @@ cudaError_t launch_t(const BwdArgs &a, cudaStream_t s)
 {
     const BwdLayout L = bwd_layout(a.B, a.T, a.H, a.dk, a.dv, a.saved_states == nullptr);
     char *ws = static_cast<char *>(a.workspace);
-    bwd_kernel<TIn, DK, DV><<<a.B * a.H, 2 * DK, 0, s>>>(
+    float *acc = reinterpret_cast<float *>(ws + L.acc_off);
+    const size_t n = (size_t)a.B * a.T * a.H * DK;
+    cudaError_t e = cudaMemsetAsync(acc, 0, 4 * n * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    bwd_kernel<TIn, DK, DV><<<a.B * a.H * (DV / JB), 2 * DK, 0, s>>>(
         a, reinterpret_cast<float *>(ws + L.cs_off), reinterpret_cast<float *>(ws + L.ts_off),
-        reinterpret_cast<float *>(ws + L.dl_off));
+        reinterpret_cast<float *>(ws + L.dl_off), acc);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (n == 0) return cudaSuccess;
+    const size_t blocks = (n + 255) / 256;
+    bwd_finish_kernel<TIn><<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(a, acc, n);
     return cudaGetLastError();
 }
 
