@@ -142,7 +142,10 @@ size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_d
  * out: dq, dk_, db [B,T,H,dk] dt; dv_, dw [B,T,H,dv] dt;
  *      dlog_alpha [B,T,H,dk] fp32; dS0 [B,H,dk,dv] fp32 or NULL.
  * scratch: workspace of at least gdr2_backward_workspace_bytes(...) bytes,
- *      256-byte aligned; its contents on entry do not matter.
+ *      256-byte aligned; its contents on entry do not matter (the call clears
+ *      the part it accumulates into, on `stream`).
+ * The per-key-channel gradients (dq, dk, db, dlog_alpha) are summed over the
+ * value columns with fp32 atomics, so their last bits may differ between calls.
  */
 gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
                           const void *q, const void *k, const void *v,
@@ -176,7 +179,8 @@ gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
  * Limit: a problem whose scratch (gdr2_backward's workspace minus the chunk
  *      states when saved_states is given) exceeds GDR2_NOALLOC_SCRATCH_BYTES
  *      returns GDR2_ERR_UNSUPPORTED before any work is enqueued. At
- *      dk = dv = 128 with saved_states that is about 4.2 MiB per (batch, head).
+ *      dk = dv = 128 with saved_states that is about 4.2 MiB per (batch, head)
+ *      plus 2 KiB per (batch, head, token).
  * Arguments, layouts and results are those of gdr2_backward. The call itself
  * makes no cudaMalloc, cudaFree or other allocating call.
  */
