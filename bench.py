@@ -312,6 +312,32 @@ def bench_components(dev, stream, peaks):
                       "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
         del xs, o, ws
     out["sweep"] = {"workload": "65,536 tokens per call, H=16, d=128, bf16, T = 2048 .. 32768", "points": sweep}
+    # packed sequences: the same 65,536 tokens cut at 63 distinct random points into 64 sequences
+    import numpy as np
+
+    from gated_delta_rule_wy_b200 import gdr2_forward_varlen, gdr2_forward_varlen_workspace_bytes, gdr2_sync_status
+    rng = np.random.default_rng(1007)
+    cuts = np.sort(rng.choice(np.arange(1, I.SWEEP_TOKENS), size=63, replace=False))
+    lens = np.diff(np.concatenate([[0], cuts, [I.SWEEP_TOKENS]]))
+    Tt = int(lens.sum())
+    xs = I.make_forward_inputs(B=1, H=16, T=Tt, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=2.0,
+                               seed=1007).to(dev)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+    o = torch.empty((Tt, 16, 128), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(gdr2_forward_varlen_workspace_bytes(len(lens), Tt, 16, 128, 128), dtype=torch.uint8,
+                     device=dev)
+
+    def fwd_packed():
+        gdr2_forward_varlen(xs.q, xs.k, xs.v, xs.log_alpha, xs.b, xs.w, cu, None, out=o, workspace=ws)
+
+    for _ in range(3):
+        fwd_packed()
+    ms = statistics.median(time_steps(fwd_packed, 10, stream))
+    gdr2_sync_status()
+    out["packed"] = {"workload": f"{Tt} tokens as {len(lens)} packed sequences (random cuts; lengths "
+                                 f"{int(lens.min())} .. {int(lens.max())}), H=16, d=128, bf16",
+                     "ms_per_call": ms, "tokens_per_s": Tt / (ms * 1e-3)}
+    del xs, o, ws
     return out
 
 

@@ -7,10 +7,11 @@ package does not load the CUDA library; the first call does, and fails loudly
 if it is missing.
 """
 from .binding import (GDR2Error, gdr2_abi_version, gdr2_backward, gdr2_backward_noalloc,  # noqa: F401
-                      gdr2_backward_workspace_bytes, gdr2_decode_step, gdr2_forward, gdr2_forward_workspace_bytes,
-                      gdr2_last_error,
+                      gdr2_backward_workspace_bytes, gdr2_decode_step, gdr2_forward, gdr2_forward_varlen,
+                      gdr2_forward_varlen_workspace_bytes, gdr2_forward_workspace_bytes, gdr2_last_error,
                       gdr2_sync_status, load_library)
 
 __all__ = ["GDR2Error", "gdr2_abi_version", "gdr2_backward", "gdr2_backward_noalloc",
            "gdr2_backward_workspace_bytes", "gdr2_forward_workspace_bytes",
-           "gdr2_decode_step", "gdr2_forward", "gdr2_last_error", "gdr2_sync_status", "load_library"]
+           "gdr2_decode_step", "gdr2_forward", "gdr2_forward_varlen", "gdr2_forward_varlen_workspace_bytes",
+           "gdr2_last_error", "gdr2_sync_status", "load_library"]

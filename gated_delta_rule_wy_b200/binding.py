@@ -24,7 +24,7 @@ _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIM
 
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
 EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspace_bytes", "gdr2_forward",
-                    "gdr2_decode_step",
+                    "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen", "gdr2_decode_step",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
                     "gdr2_sync_status")
 NOALLOC_SCRATCH_BYTES = 64 << 20  # GDR2_NOALLOC_SCRATCH_BYTES
@@ -61,6 +61,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_forward.restype = I
         lib.gdr2_forward.argtypes = [I, I, I, I, I, I] + [P] * 11 + [Z, P]
         lib.gdr2_decode_step.restype = I
+        lib.gdr2_forward_varlen_workspace_bytes.restype = Z
+        lib.gdr2_forward_varlen_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        lib.gdr2_forward_varlen.restype = I
+        lib.gdr2_forward_varlen.argtypes = [I, I, I, I, I, I] + [P] * 12 + [Z, P]
         lib.gdr2_decode_step.argtypes = [I, I, I, I, I] + [P] * 9
         lib.gdr2_backward_workspace_bytes.restype = Z
         lib.gdr2_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
@@ -157,6 +161,52 @@ def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_st
     st = lib.gdr2_forward(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
                           _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
                           ctypes.c_size_t(ws_bytes), _stream(stream))
+    _raise(lib, st)
+    return o, S_T, saved
+
+
+def gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    lib = load_library()
+    return int(lib.gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv,
+                                                       GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
+
+
+def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_state=True, save_states=False,
+                        out=None, workspace=None, stream=None):
+    """Forward over packed sequences. Returns (o, S_T, saved_states).
+
+    q, k, b: [T, H, dk] (or [1, T, H, dk]); v, w: [T, H, dv]; bf16; log_alpha [T, H, dk] fp32;
+    cu_seqlens: int32 [N + 1] on the device; S0: [N, H, dk, dv] fp32 or None. saved_states,
+    when asked for, is [H * (ceil(T / 64) + N), dk, dv] (see include/gdr2.h for the order).
+    """
+    lib = load_library()
+    sq = lambda t: None if t is None else (t[0] if t.dim() == 4 else t)  # noqa: E731
+    q, k, v, log_alpha, b, w = (sq(t) for t in (q, k, v, log_alpha, b, w))
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    for name, t, shp in (("q", q, (T, H, dk)), ("k", k, (T, H, dk)), ("b", b, (T, H, dk)),
+                         ("v", v, (T, H, dv)), ("w", w, (T, H, dv))):
+        _check(t, name, shp, dt)
+    _check(log_alpha, "log_alpha", (T, H, dk), torch.float32)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous() \
+            or cu_seqlens.device != q.device:
+        raise ValueError("cu_seqlens must be a contiguous 1-D int32 tensor on the inputs' device")
+    N = cu_seqlens.numel() - 1
+    _check(S0, "S0", (N, H, dk, dv), torch.float32)
+    dev = q.device
+    o = out if out is not None else torch.empty((T, H, dv), dtype=dt, device=dev)
+    _check(sq(o), "o", (T, H, dv), dt)
+    S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if final_state else None
+    cap = H * ((T + CHUNK - 1) // CHUNK + N)
+    saved = torch.empty((cap, dk, dv), dtype=torch.float32, device=dev) if save_states else None
+    need = gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dt)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.gdr2_forward_varlen(N, T, H, dk, dv, _dt(q), _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved),
+                                 _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
     return o, S_T, saved
 

@@ -168,10 +168,88 @@ constexpr uint32_t GAMMA_BYTES = DK * 4;  // exp(G_C), stored after all slots
 
 struct ChunkParams {
     int B, T, H, NC;
-    int ntasks;            // B * H * NC, task = bh * NC + n
+    int ntasks;            // slot capacity: B * H * NC (dense), task = bh * NC + n
     unsigned char *ws;     // workspace: ntasks slots, then ntasks gamma vectors
     unsigned *status;
+    // packed sequences (null when dense): B sequences of cu_seqlens[s+1] - cu_seqlens[s]
+    // tokens in one [1, T, H, D] tensor; sequence s owns the H * nc_s tasks from
+    // H * cu_chunks[s] on (head-major, then chunk), nc_s = cu_chunks[s+1] - cu_chunks[s]
+    const int *cu_seqlens;
+    const int *cu_chunks;
+    const int *ntasks_dev;  // H * cu_chunks[B], written by the prefix kernel
 };
+
+// Where a task's chunk lives: tensor-map coordinates (token t0, sequence bb), head h, and the
+// number of real tokens Cn in it.
+struct ChunkLoc {
+    int h, t0, bb, Cn;
+};
+
+__device__ __forceinline__ ChunkLoc locate_chunk(const ChunkParams &p, int task)
+{
+    ChunkLoc L;
+    if (!p.cu_seqlens) {
+        const int bh = task / p.NC, n = task % p.NC;
+        L.bb = bh / p.H;
+        L.h = bh % p.H;
+        L.t0 = n * C;
+        L.Cn = min(C, p.T - n * C);
+        return L;
+    }
+    // the sequence s with H cu_chunks[s] <= task < H cu_chunks[s + 1] (binary search)
+    int lo = 0, hi = p.B;  // invariant: H cu_chunks[lo] <= task < H cu_chunks[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (p.H * p.cu_chunks[mid] <= task) lo = mid; else hi = mid;
+    }
+    const int nc = p.cu_chunks[lo + 1] - p.cu_chunks[lo];
+    const int rem = task - p.H * p.cu_chunks[lo];
+    const int n = rem % nc;
+    L.h = rem / nc;
+    L.bb = 0;
+    L.t0 = p.cu_seqlens[lo] + n * C;
+    L.Cn = min(C, p.cu_seqlens[lo + 1] - L.t0);
+    return L;
+}
+
+// Packed sequences: chunk offsets per sequence and the task count, after checking that
+// cu_seqlens runs from 0 to T without decreasing. If it does not, no task runs (the count
+// is 0 and every offset 0) and the status word records it. One block.
+__global__ void __launch_bounds__(1024) varlen_prefix_kernel(const int *cu, int N, int T, int H, int *cu_chunks,
+                                                             int *ntasks, unsigned *status)
+{
+    __shared__ int part[1024];
+    const int tid = threadIdx.x;
+    const int per = (N + 1023) / 1024;
+    const int i0 = tid * per, i1 = min(N, i0 + per);
+    int sum = 0;
+    bool bad = false;
+    for (int i = i0; i < i1; ++i) {
+        const int len = cu[i + 1] - cu[i];
+        bad |= len < 0;
+        sum += (max(len, 0) + C - 1) / C;
+    }
+    if (tid == 0) bad |= cu[0] != 0 || cu[N] != T;
+    bad = __syncthreads_or(bad) != 0;
+    part[tid] = sum;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan of the per-thread sums
+        const int v = tid >= off ? part[tid - off] : 0;
+        __syncthreads();
+        part[tid] += v;
+        __syncthreads();
+    }
+    int run = part[tid] - sum;  // exclusive
+    for (int i = i0; i < i1; ++i) {
+        cu_chunks[i] = bad ? 0 : run;
+        run += (max(cu[i + 1] - cu[i], 0) + C - 1) / C;
+    }
+    if (tid == 1023) {
+        cu_chunks[N] = bad ? 0 : part[1023];
+        *ntasks = bad ? 0 : H * part[1023];
+        if (bad) atomicOr(status, kStatusBadSeqlens);
+    }
+}
 
 // TMEM columns of the chunk kernel
 constexpr uint32_t CK_M = 0, CK_U = 128, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384, CK_AP1 = 416;
@@ -190,7 +268,6 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quarter = warp & 3, colhalf = warp >> 2;
-    const int NC = p.NC;
 
     if (tid == 0) {
         mbar_init(&ms.bar_tma, 1);
@@ -208,18 +285,18 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);  // this warp's TMEM lanes
     const int row = quarter * 32 + lane;                              // this thread's TMEM lane
 
+    const int ntasks = p.cu_seqlens ? *p.ntasks_dev : p.ntasks;
     auto issue_loads = [&](int task) {
-        const int bh = task / NC, n = task % NC;
-        const int bb = bh / p.H, h = bh % p.H, t0 = n * C;
+        const ChunkLoc L = locate_chunk(p, task);
         mbar_arrive_expect_tx(&ms.bar_tma, TX_BYTES);
-        tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_STG_V, &tm_v, &ms.bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, h, t0, bb);
+        tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        tma_load_4d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        tma_load_4d(sm + OFF_STG_V, &tm_v, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, L.h, L.t0, L.bb);
     };
-    if (tid == 0 && (int)blockIdx.x < p.ntasks) issue_loads(blockIdx.x);
+    if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
     // the scan kernel may be scheduled now: its CTAs take an SM only once this (persistent) CTA
     // has left it, and they read the workspace only after this whole grid has completed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -245,13 +322,29 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float *A32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
-    for (int task = blockIdx.x; task < p.ntasks && !timed_out; task += gridDim.x) {
-        const int n = task % NC;
-        const int Cn = min(C, p.T - n * C);
+    for (int task = blockIdx.x; task < ntasks && !timed_out; task += gridDim.x) {
+        const int Cn = locate_chunk(p, task).Cn;
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
         if (tid == 64) bulk_wait_group_read0();  // K~, P and U~ of the previous task have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
+        if (Cn < C) {
+            // a partial chunk: the rows past the sequence hold zeros (dense: the copy engine's
+            // fill past T) or the next sequence's tokens (packed); zero them, which makes those
+            // rows inert in every product
+            for (int i = tid; i < (C - Cn) * 16; i += NT) {
+                const int t = Cn + (i >> 4), o = i & 15;
+                const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_Q + t * 256 + o * 16) = z4;
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_K + t * 256 + o * 16) = z4;
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_B + t * 256 + o * 16) = z4;
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_V + t * 256 + o * 16) = z4;
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_W + t * 256 + o * 16) = z4;
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_LA + t * 512 + o * 32) = z4;
+                *reinterpret_cast<uint4 *>(sm + OFF_STG_LA + t * 512 + o * 32 + 16) = z4;
+            }
+            __syncthreads();
+        }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
         // Rows beyond T are zero-filled by TMA (per-sequence extent): padded tokens are inert.
@@ -532,7 +625,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // The staging buffers are free: prefetch the next task. K~ and P are final: copy them to
         // the slot in the background. Both are issued from warp 2, idle in the first solve levels.
         if (tid == 64) {
-            if (task + (int)gridDim.x < p.ntasks) issue_loads(task + gridDim.x);
+            if (task + (int)gridDim.x < ntasks) issue_loads(task + gridDim.x);
             bulk_store(slot + SLOT_KT, sm + OFF_KT, 16384);
             bulk_store(slot + SLOT_P, sm + OFF_P, 8192);
             bulk_commit_group();
@@ -880,6 +973,9 @@ struct ScanParams {
     float *S_T;
     float *saved_states;
     unsigned *status;
+    const int *cu_seqlens;  // packed sequences (null when dense), as in ChunkParams
+    const int *cu_chunks;
+    __nv_bfloat16 *o;       // for the row-by-row store of a packed sequence's last, partial tile
 };
 
 __global__ void __launch_bounds__(NT, 1)
@@ -892,10 +988,12 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quarter = warp & 3, colhalf = warp >> 2;
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x;  // (sequence, head)
     const int bb = bh / p.H, h = bh % p.H;
-    const int NC = p.NC;
     const int c0 = colhalf * 64;  // this thread's 64 state columns c (S^T columns)
+    // this (sequence, head)'s chunks: count, first task, first token and length, map batch
+    int NC = p.NC, tstart = 0, len = p.T, tb = bb;
+    size_t base = (size_t)bh * p.NC;
 
     if (tid == 0) {
         mbar_init(&ms.bar_full[0], 1);
@@ -917,10 +1015,17 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     // Launched as a programmatic dependent of the chunk kernel: everything above overlaps its
     // tail; the workspace is read only after that grid has completed and flushed its memory.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (p.cu_seqlens) {
+        NC = p.cu_chunks[bb + 1] - p.cu_chunks[bb];
+        base = (size_t)p.H * p.cu_chunks[bb] + (size_t)h * NC;
+        tstart = p.cu_seqlens[bb];
+        len = p.cu_seqlens[bb + 1] - tstart;
+        tb = 0;
+    }
 
     auto issue_slot = [&](int n) {
         const int sl = n & 1;
-        const size_t task = (size_t)bh * NC + n;
+        const size_t task = base + n;
         mbar_arrive_expect_tx(&ms.bar_full[sl], SLOT_BYTES + GAMMA_BYTES);
         bulk_load(sm + (sl ? SC_SLOT1 : SC_SLOT0), p.ws + task * SLOT_BYTES, SLOT_BYTES, &ms.bar_full[sl]);
         bulk_load(ms.gam[sl], p.ws + (size_t)p.ntasks * SLOT_BYTES + task * GAMMA_BYTES, GAMMA_BYTES,
@@ -974,8 +1079,17 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_barrier(1, 128);
-        if (tid == 0) {
-            tma_store_4d(&tm_o, sm + SC_O, 0, h, m * C, bb);
+        const int rows = min(C, len - m * C);
+        if (p.cu_seqlens && rows < C) {
+            // a packed sequence's partial last tile: its rows only (a tile store would write
+            // into the next sequence)
+            for (int i = tid; i < rows * 16; i += 128) {
+                const int r = i >> 4, c16 = i & 15;
+                *reinterpret_cast<uint4 *>(p.o + ((size_t)(tstart + m * C + r) * p.H + h) * DV + c16 * 8) =
+                    *reinterpret_cast<const uint4 *>(ot + r * DV + c16 * 8);
+            }
+        } else if (tid == 0) {
+            tma_store_4d(&tm_o, sm + SC_O, 0, h, tstart + m * C, tb);
             bulk_commit_group();
         }
     };
@@ -990,7 +1104,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
             float s0[32], s1[32];
             tmem_ld32x2(tm_lane + rg_prev + SC_ST + c0, tm_lane + rg_prev + SC_ST + c0 + 32, s0, s1);
             if (p.saved_states) {
-                float *dst = p.saved_states + (((size_t)bh * NC + n) * DK + c0) * DV + j;
+                float *dst = p.saved_states + ((base + n) * DK + c0) * DV + j;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     dst[(size_t)i * DV] = s0[i];
@@ -1138,13 +1252,24 @@ size_t forward_tc_workspace_bytes(int B, int T, int H)
     return ntasks * (SLOT_BYTES + GAMMA_BYTES);
 }
 
+// Packed sequences: at most H (ceil(T / 64) + N) tasks (each sequence adds at most one
+// partial chunk), then the chunk offsets (N + 1 ints) and the task count.
+static size_t varlen_task_capacity(int N, int T, int H) { return (size_t)H * ((T + C - 1) / C + N); }
+
+size_t forward_tc_varlen_workspace_bytes(int N, int T, int H)
+{
+    return varlen_task_capacity(N, T, H) * (SLOT_BYTES + GAMMA_BYTES) + (((size_t)N + 2) * sizeof(int) + 255) / 256 * 256;
+}
+
 cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
 {
+    const bool varlen = a.cu_seqlens != nullptr;
+    const int Bm = varlen ? 1 : a.B;  // tensor-map batch extent: packed sequences share one
     CUtensorMap mq, mk, mb, mv, mw, mla, mo;
-    if (!make_map(&mq, a.q, false, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, false, a.B, a.T, a.H, DK) ||
-        !make_map(&mb, a.b, false, a.B, a.T, a.H, DK) || !make_map(&mv, a.v, false, a.B, a.T, a.H, DV) ||
-        !make_map(&mw, a.w, false, a.B, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK) ||
-        !make_map(&mo, a.o, false, a.B, a.T, a.H, DV))
+    if (!make_map(&mq, a.q, false, Bm, a.T, a.H, DK) || !make_map(&mk, a.k, false, Bm, a.T, a.H, DK) ||
+        !make_map(&mb, a.b, false, Bm, a.T, a.H, DK) || !make_map(&mv, a.v, false, Bm, a.T, a.H, DV) ||
+        !make_map(&mw, a.w, false, Bm, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, Bm, a.T, a.H, DK) ||
+        !make_map(&mo, a.o, false, Bm, a.T, a.H, DV))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
@@ -1154,13 +1279,23 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const int NC = (a.T + C - 1) / C;
-    const int ntasks = a.B * a.H * NC;
-    ChunkParams cp{a.B, a.T, a.H, NC, ntasks, static_cast<unsigned char *>(a.workspace), a.status};
+    const int ntasks = varlen ? (int)varlen_task_capacity(a.B, a.T, a.H) : a.B * a.H * NC;
+    unsigned char *ws = static_cast<unsigned char *>(a.workspace);
+    int *cu_chunks = nullptr, *ntasks_dev = nullptr;
+    if (varlen) {
+        cu_chunks = reinterpret_cast<int *>(ws + (size_t)ntasks * (SLOT_BYTES + GAMMA_BYTES));
+        ntasks_dev = cu_chunks + a.B + 1;
+        varlen_prefix_kernel<<<1, 1024, 0, s>>>(a.cu_seqlens, a.B, a.T, a.H, cu_chunks, ntasks_dev, a.status);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    ChunkParams cp{a.B, a.T, a.H, NC, ntasks, ws, a.status, a.cu_seqlens, cu_chunks, ntasks_dev};
     fwd_chunk_kernel<<<ntasks < nsm ? ntasks : nsm, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    ScanParams sp{a.B, a.T, a.H, NC, ntasks, static_cast<const unsigned char *>(a.workspace), a.S0, a.S_T,
-                  a.saved_states, a.status};
+    ScanParams sp{a.B,          a.T,          a.H,    NC,       ntasks,    ws,
+                  a.S0,         a.S_T,        a.saved_states, a.status, a.cu_seqlens, cu_chunks,
+                  static_cast<__nv_bfloat16 *>(a.o)};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.H);
     cfg.blockDim = dim3(NT);

@@ -152,6 +152,60 @@ gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, con
     return launched(gdr2::launch_forward_simt(a, s), "gdr2_forward (simt)");
 }
 
+size_t gdr2_forward_varlen_workspace_bytes(int N, int T, int H, int dk, int dv, gdr2_dtype dt)
+{
+    if (N < 0 || T < 0 || H < 0) return 0;
+    if (dt != GDR2_BF16 || dk != 128 || dv != 128) return 0;
+    return gdr2::forward_tc_varlen_workspace_bytes(N, T, H);
+}
+
+gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype dt, const int *cu_seqlens,
+                                const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                                const void *w, const float *S0, void *o, float *S_T, float *saved_states,
+                                void *workspace, size_t workspace_bytes, void *stream)
+{
+    GDR2_TRY(check_dims(N, T, H, dk, dv));
+    GDR2_TRY(check_dtype(dt));
+    if (dt != GDR2_BF16 || dk != 128 || dv != 128)
+        return fail(GDR2_ERR_UNSUPPORTED, "packed sequences need bf16 inputs with dk = dv = 128");
+    if ((long long)N * H == 0) return GDR2_OK;
+    const bool has_tokens = (long long)T * H > 0;
+    if (!cu_seqlens) return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+        return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+    GDR2_TRY(check_ptr(q, "q", !has_tokens));
+    GDR2_TRY(check_ptr(k, "k", !has_tokens));
+    GDR2_TRY(check_ptr(v, "v", !has_tokens));
+    GDR2_TRY(check_ptr(log_alpha, "log_alpha", !has_tokens));
+    GDR2_TRY(check_ptr(b, "b", !has_tokens));
+    GDR2_TRY(check_ptr(w, "w", !has_tokens));
+    GDR2_TRY(check_ptr(o, "o", !has_tokens));
+    GDR2_TRY(check_ptr(S0, "S0", true));
+    GDR2_TRY(check_ptr(S_T, "S_T", true));
+    GDR2_TRY(check_ptr(saved_states, "saved_states", true));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (S_T && S_T != S0) {
+            const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
+            cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(S_T, 0, bytes, s);
+            return launched(e, "gdr2_forward_varlen (T = 0)");
+        }
+        return GDR2_OK;
+    }
+    const size_t need = gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dt);
+    if (!workspace || workspace_bytes < need)
+        return fail(GDR2_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    gdr2::FwdArgs a{N, T, H, dk, dv, true, q, k, v, log_alpha, b, w, S0, o, S_T, saved_states, workspace,
+                    workspace_bytes, nullptr, cu_seqlens};
+    GDR2_TRY(device_status(&a.status));
+    if (!gdr2::forward_tc_supported(a))
+        return fail(GDR2_ERR_UNSUPPORTED, "the tensor-core forward is not available on this device");
+    return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward_varlen (tcgen05)");
+}
+
 gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
                              const void *v, const float *log_alpha, const void *b, const void *w, float *S,
                              void *o, void *stream)
@@ -270,6 +324,9 @@ gdr2_status gdr2_sync_status(void *stream)
     if (e != cudaSuccess) return fail(GDR2_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(e));
     if (word & gdr2::kStatusTimeout)
         return fail(GDR2_ERR_TIMEOUT, "a kernel gave up a bounded device wait (status 0x%x)", word);
+    if (word & gdr2::kStatusBadSeqlens)
+        return fail(GDR2_ERR_INVALID_ARG,
+                    "cu_seqlens was not a nondecreasing sequence from 0 to T; that call computed nothing");
     g_last_error[0] = '\0';
     return GDR2_OK;
 }

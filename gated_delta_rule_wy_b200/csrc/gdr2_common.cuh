@@ -13,7 +13,8 @@ constexpr float kLogAlphaFloor = -64.0f;
 
 // Bits of the device status word (one per device, read by gdr2_sync_status).
 enum : unsigned {
-    kStatusTimeout = 1u,  // a kernel gave up a bounded wait
+    kStatusTimeout = 1u,      // a kernel gave up a bounded wait
+    kStatusBadSeqlens = 2u,   // cu_seqlens was not a nondecreasing run from 0 to T (no work done)
 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -20,6 +20,7 @@ struct FwdArgs {
     void *workspace;   // chunk intermediates of the tensor-core path
     size_t workspace_bytes;
     unsigned *status;  // device status word
+    const int *cu_seqlens;  // packed sequences: B = their number, T = total tokens (null = dense)
 };
 
 struct DecodeArgs {
@@ -56,6 +57,7 @@ cudaError_t launch_forward_simt(const FwdArgs &a, cudaStream_t s);
 cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s);
 bool forward_tc_supported(const FwdArgs &a);
 size_t forward_tc_workspace_bytes(int B, int T, int H);
+size_t forward_tc_varlen_workspace_bytes(int N, int T, int H);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf16);
 cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s);

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 2
+#define GDR2_ABI_VERSION 3
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -127,6 +127,37 @@ gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt,
                              const void *q, const void *k, const void *v,
                              const float *log_alpha, const void *b, const void *w,
                              float *S, void *o, void *stream);
+
+/* Bytes of device scratch gdr2_forward_varlen needs (N sequences, T tokens in all). */
+size_t gdr2_forward_varlen_workspace_bytes(int N, int T, int H, int dk, int dv, gdr2_dtype dt);
+
+/*
+ * gdr2_forward_varlen -- gdr2_forward over N packed sequences of different
+ * lengths. The pages' chunkwise forward applied to each sequence on its own:
+ * each starts from its own S0 and stops at its own end, and no state or
+ * product crosses from one sequence to the next. (The pages train on
+ * sequences of one length; packing is how such layers are fed mixed lengths.)
+ * in:  cu_seqlens [N + 1] int32, DEVICE memory: 0 = cu_seqlens[0] <=
+ *      cu_seqlens[1] <= ... <= cu_seqlens[N] = T; sequence i is tokens
+ *      cu_seqlens[i] .. cu_seqlens[i+1] - 1 (empty sequences are allowed).
+ *      q, k, b [T, H, dk] (= [1, T, H, dk]) bf16; v, w [T, H, dv] bf16;
+ *      log_alpha [T, H, dk] fp32; S0 [N, H, dk, dv] fp32 or NULL (zeros).
+ * out: o [T, H, dv] bf16; S_T [N, H, dk, dv] fp32 or NULL.
+ *      saved_states or NULL: the state entering each chunk, [C_total][dk][dv]
+ *      fp32 with C_total <= H * (ceil(T / 64) + N) (allocate that many);
+ *      sequence i's entries start at H * sum_{j<i} ceil(len_j / 64), head
+ *      by head, its chunks in order within a head.
+ * scratch: workspace of at least gdr2_forward_varlen_workspace_bytes(...)
+ *      bytes, 256-byte aligned.
+ * Supported: bf16 inputs with dk = dv = 128 (GDR2_ERR_UNSUPPORTED otherwise).
+ * cu_seqlens is read on the device only: if it breaks the rule above, the call
+ * computes nothing and the next gdr2_sync_status returns GDR2_ERR_INVALID_ARG.
+ */
+gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype dt, const int *cu_seqlens,
+                                const void *q, const void *k, const void *v, const float *log_alpha,
+                                const void *b, const void *w, const float *S0,
+                                void *o, float *S_T, float *saved_states,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /* Bytes of device scratch gdr2_backward needs for this problem. */
 size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt);

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 2
+    assert lib.gdr2_abi_version() == 3
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -86,6 +86,26 @@ def test_backward_workspace_query_and_checks(lib):
     st = lib.gdr2_backward(2, 64, 16, 128, 128, 1, *p, ctypes.c_size_t(16), ctypes.c_void_p(0))
     assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
     assert lib.gdr2_backward_workspace_bytes(-1, 1, 1, 64, 64, 1) == 0
+
+
+def test_varlen_forward_workspace_query_and_checks(lib):
+    # slots and gamma vectors for at most H (ceil(T / 64) + N) tasks, then N + 2 ints
+    n = lib.gdr2_forward_varlen_workspace_bytes(8, 1000, 16, 128, 128, 1)
+    assert n >= 16 * (16 + 8) * (90112 + 512) + 10 * 4 and n % 256 == 0
+    assert lib.gdr2_forward_varlen_workspace_bytes(8, 1000, 16, 128, 128, 0) == 0  # fp32: not supported
+    p = ctypes.c_void_p(0x10000)
+    args = [p] * 12 + [ctypes.c_size_t(1 << 30), ctypes.c_void_p(0)]
+    assert lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 0, *args) == binding.GDR2_ERR_UNSUPPORTED
+    assert lib.gdr2_forward_varlen(2, 64, 4, 64, 128, 1, *args) == binding.GDR2_ERR_UNSUPPORTED
+    nul = [ctypes.c_void_p(0)] + [p] * 11 + [ctypes.c_size_t(1 << 30), ctypes.c_void_p(0)]
+    st = lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, *nul)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"cu_seqlens" in lib.gdr2_last_error()
+    small = [p] * 12 + [ctypes.c_size_t(16), ctypes.c_void_p(0)]
+    st = lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, *small)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
+    # no sequences or no heads: nothing to do, no pointer needed
+    assert lib.gdr2_forward_varlen(0, 0, 4, 128, 128, 1, *([ctypes.c_void_p(0)] * 12),
+                                   ctypes.c_size_t(0), ctypes.c_void_p(0)) == binding.GDR2_OK
 
 
 def test_binding_validates_before_calling():
