@@ -338,6 +338,28 @@ def bench_components(dev, stream, peaks):
                                  f"{int(lens.min())} .. {int(lens.max())}), H=16, d=128, bf16",
                      "ms_per_call": ms, "tokens_per_s": Tt / (ms * 1e-3)}
     del xs, o, ws
+    # the 1.3B-layer forward with KDA / Gated DeltaNet gates: b = w = beta, one value per token-head
+    c = I.FWD_1P3B_BF16
+    xs = I.make_forward_inputs(**c).to(dev)
+    beta = torch.sigmoid(torch.randn((c["B"], c["T"], c["H"]), generator=torch.Generator().manual_seed(1008)))
+    beta = beta.to(c["dtype"]).to(dev)
+    o = torch.empty_like(xs.v)
+    ws = torch.empty(gdr2_forward_workspace_bytes(c["B"], c["T"], c["H"], c["dk"], c["dv"], c["dtype"]),
+                     dtype=torch.uint8, device=dev)
+
+    def fwd_kda():
+        gdr2_forward(xs.q, xs.k, xs.v, xs.log_alpha, beta, beta, None, out=o, workspace=ws)
+
+    for _ in range(3):
+        fwd_kda()
+    ms = statistics.median(time_steps(fwd_kda, 20, stream))
+    gdr2_sync_status()
+    tokens = c["B"] * c["T"]
+    alg = tokens * c["H"] * (BYTES_PER_TOKEN_HEAD - 2 * 256 + 2 * 2) + c["B"] * c["H"] * c["dk"] * c["dv"] * 4
+    out["kda_gates"] = {"workload": "B=4 H=16 T=4096 d=128 bf16 with b = w = beta scalar per token-head",
+                        "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3),
+                        "algorithmic_bytes": alg, "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del xs, o, ws, beta
     return out
 
 

@@ -24,7 +24,8 @@ _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIM
 
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
 EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspace_bytes", "gdr2_forward",
-                    "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen", "gdr2_decode_step",
+                    "gdr2_forward_gated", "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen",
+                    "gdr2_decode_step", "gdr2_decode_step_gated",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
                     "gdr2_sync_status")
 NOALLOC_SCRATCH_BYTES = 64 << 20  # GDR2_NOALLOC_SCRATCH_BYTES
@@ -64,7 +65,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_forward_varlen_workspace_bytes.restype = Z
         lib.gdr2_forward_varlen_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.gdr2_forward_varlen.restype = I
-        lib.gdr2_forward_varlen.argtypes = [I, I, I, I, I, I] + [P] * 12 + [Z, P]
+        lib.gdr2_forward_varlen.argtypes = [I, I, I, I, I, I, I] + [P] * 12 + [Z, P]
+        lib.gdr2_forward_gated.restype = I
+        lib.gdr2_forward_gated.argtypes = [I, I, I, I, I, I, I] + [P] * 11 + [Z, P]
+        lib.gdr2_decode_step_gated.restype = I
+        lib.gdr2_decode_step_gated.argtypes = [I, I, I, I, I, I] + [P] * 9
         lib.gdr2_decode_step.argtypes = [I, I, I, I, I] + [P] * 9
         lib.gdr2_backward_workspace_bytes.restype = Z
         lib.gdr2_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
@@ -108,6 +113,19 @@ def _check(t, name, shape, dtype):
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
 
 
+GATE_SCALAR_B, GATE_SCALAR_W = 1, 2  # GDR2_GATE_* of include/gdr2.h
+
+
+def _gates(b, w, lead):
+    """Gate layout bits from the shapes: a gate shaped `lead` (no channel dim) is a scalar."""
+    g = 0
+    if tuple(b.shape) == tuple(lead):
+        g |= GATE_SCALAR_B
+    if tuple(w.shape) == tuple(lead):
+        g |= GATE_SCALAR_W
+    return g
+
+
 def _raise(lib, st):
     if st != GDR2_OK:
         raise GDR2Error(st, lib.gdr2_last_error().decode(errors="replace"))
@@ -138,13 +156,16 @@ def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_st
 
     q, k, b: [B, T, H, dk]; v, w: [B, T, H, dv] (fp32 or bf16, one dtype);
     log_alpha: [B, T, H, dk] fp32; S0: [B, H, dk, dv] fp32 or None.
+    b and/or w may instead be [B, T, H]: one gate value per token-head (scalar gates).
     """
     lib = load_library()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("b", b, (B, T, H, dk)),
-                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H, dv))):
+    gates = _gates(b, w, (B, T, H))
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)),
+                         ("b", b, (B, T, H) if gates & GATE_SCALAR_B else (B, T, H, dk)),
+                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H) if gates & GATE_SCALAR_W else (B, T, H, dv))):
         _check(t, name, shp, dt)
     _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32)
     _check(S0, "S0", (B, H, dk, dv), torch.float32)
@@ -158,9 +179,9 @@ def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_st
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.gdr2_forward(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
-                          _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
-                          ctypes.c_size_t(ws_bytes), _stream(stream))
+    st = lib.gdr2_forward_gated(B, T, H, dk, dv, _dt(q), gates, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
+                                ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
     return o, S_T, saved
 
@@ -176,17 +197,22 @@ def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_
     """Forward over packed sequences. Returns (o, S_T, saved_states).
 
     q, k, b: [T, H, dk] (or [1, T, H, dk]); v, w: [T, H, dv]; bf16; log_alpha [T, H, dk] fp32;
-    cu_seqlens: int32 [N + 1] on the device; S0: [N, H, dk, dv] fp32 or None. saved_states,
+    cu_seqlens: int32 [N + 1] on the device; S0: [N, H, dk, dv] fp32 or None; b and/or w may
+    be [T, H] (scalar gates). saved_states,
     when asked for, is [H * (ceil(T / 64) + N), dk, dv] (see include/gdr2.h for the order).
     """
     lib = load_library()
-    sq = lambda t: None if t is None else (t[0] if t.dim() == 4 else t)  # noqa: E731
-    q, k, v, log_alpha, b, w = (sq(t) for t in (q, k, v, log_alpha, b, w))
+    sq4 = lambda t: None if t is None else (t[0] if t.dim() == 4 else t)  # noqa: E731
+    q, k, v, log_alpha = (sq4(t) for t in (q, k, v, log_alpha))
     T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    for name, t, shp in (("q", q, (T, H, dk)), ("k", k, (T, H, dk)), ("b", b, (T, H, dk)),
-                         ("v", v, (T, H, dv)), ("w", w, (T, H, dv))):
+    sqg = lambda t: t[0] if t.dim() == 4 or (t.dim() == 3 and tuple(t.shape) == (1, T, H)) else t  # noqa: E731
+    b, w = sqg(b), sqg(w)
+    gates = _gates(b, w, (T, H))
+    for name, t, shp in (("q", q, (T, H, dk)), ("k", k, (T, H, dk)),
+                         ("b", b, (T, H) if gates & GATE_SCALAR_B else (T, H, dk)),
+                         ("v", v, (T, H, dv)), ("w", w, (T, H) if gates & GATE_SCALAR_W else (T, H, dv))):
         _check(t, name, shp, dt)
     _check(log_alpha, "log_alpha", (T, H, dk), torch.float32)
     if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous() \
@@ -196,7 +222,7 @@ def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_
     _check(S0, "S0", (N, H, dk, dv), torch.float32)
     dev = q.device
     o = out if out is not None else torch.empty((T, H, dv), dtype=dt, device=dev)
-    _check(sq(o), "o", (T, H, dv), dt)
+    _check(sq4(o), "o", (T, H, dv), dt)
     S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if final_state else None
     cap = H * ((T + CHUNK - 1) // CHUNK + N)
     saved = torch.empty((cap, dk, dv), dtype=torch.float32, device=dev) if save_states else None
@@ -204,7 +230,7 @@ def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.gdr2_forward_varlen(N, T, H, dk, dv, _dt(q), _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+    st = lib.gdr2_forward_varlen(N, T, H, dk, dv, _dt(q), gates, _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved),
                                  _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
@@ -212,20 +238,25 @@ def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_
 
 
 def gdr2_decode_step(q, k, v, log_alpha, b, w, S, *, out=None, stream=None):
-    """One decode token; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv]."""
+    """One decode token; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv].
+
+    b and/or w may be [N, H]: one gate value per token-head (scalar gates).
+    """
     lib = load_library()
     N, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    for name, t, shp in (("q", q, (N, H, dk)), ("k", k, (N, H, dk)), ("b", b, (N, H, dk)),
-                         ("v", v, (N, H, dv)), ("w", w, (N, H, dv))):
+    gates = _gates(b, w, (N, H))
+    for name, t, shp in (("q", q, (N, H, dk)), ("k", k, (N, H, dk)),
+                         ("b", b, (N, H) if gates & GATE_SCALAR_B else (N, H, dk)),
+                         ("v", v, (N, H, dv)), ("w", w, (N, H) if gates & GATE_SCALAR_W else (N, H, dv))):
         _check(t, name, shp, dt)
     _check(log_alpha, "log_alpha", (N, H, dk), torch.float32)
     _check(S, "S", (N, H, dk, dv), torch.float32)
     o = out if out is not None else torch.empty((N, H, dv), dtype=dt, device=q.device)
     _check(o, "o", (N, H, dv), dt)
-    st = lib.gdr2_decode_step(N, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
-                              _ptr(w), _ptr(S), _ptr(o), _stream(stream))
+    st = lib.gdr2_decode_step_gated(N, H, dk, dv, _dt(q), gates, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                    _ptr(b), _ptr(w), _ptr(S), _ptr(o), _stream(stream))
     _raise(lib, st)
     return o
 

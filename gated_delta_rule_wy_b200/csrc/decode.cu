@@ -50,22 +50,23 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a)
 
     const TIn *q = static_cast<const TIn *>(a.q) + (size_t)nh * DK;
     const TIn *k = static_cast<const TIn *>(a.k) + (size_t)nh * DK;
-    const TIn *bg = static_cast<const TIn *>(a.b) + (size_t)nh * DK;
+    const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
+    const TIn *bg = static_cast<const TIn *>(a.b) + (size_t)nh * (bsc ? 1 : DK);
     const float *la = a.log_alpha + (size_t)nh * DK;
     const TIn *v = static_cast<const TIn *>(a.v) + (size_t)nh * DV;
-    const TIn *wg = static_cast<const TIn *>(a.w) + (size_t)nh * DV;
+    const TIn *wg = static_cast<const TIn *>(a.w) + (size_t)nh * (wsc ? 1 : DV);
 
     float kq = 0.f;
     if (tid < DK) {
         const float kv = to_f32(k[tid]), qv = to_f32(q[tid]);
         const float al = expf(clamp_log_alpha(la[tid]));
-        s_ae[tid] = al * to_f32(bg[tid]) * kv;
+        s_ae[tid] = al * to_f32(bg[bsc ? 0 : tid]) * kv;
         s_aq[tid] = al * qv;
         s_al[tid] = al;
         s_k[tid] = kv;
         kq = kv * qv;
     }
-    if (tid < DV) s_z[tid] = to_f32(wg[tid]) * to_f32(v[tid]);
+    if (tid < DV) s_z[tid] = to_f32(wg[wsc ? 0 : tid]) * to_f32(v[tid]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
     if (lane == 0) s_kq[warp] = kq;

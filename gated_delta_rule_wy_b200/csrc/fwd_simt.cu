@@ -88,10 +88,11 @@ __global__ void __launch_bounds__(NT, 1) fwd_simt_kernel(FwdArgs a)
             const int t = idx / DK, c = idx % DK;
             float qv = 0.f, kv = 0.f, bv = 0.f, la = 0.f;
             if (t < Cn) {
-                const size_t off = (((size_t)bb * T + t0 + t) * H + h) * DK + c;
+                const size_t row = ((size_t)bb * T + t0 + t) * H + h;
+                const size_t off = row * DK + c;
                 qv = to_f32(q[off]);
                 kv = to_f32(k[off]);
-                bv = to_f32(bg[off]);
+                bv = to_f32(bg[(a.gates & kGateScalarB) ? row : off]);
                 la = clamp_log_alpha(a.log_alpha[off]);
             }
             sm.Q[t][c] = qv;
@@ -103,8 +104,9 @@ __global__ void __launch_bounds__(NT, 1) fwd_simt_kernel(FwdArgs a)
             const int t = idx / DVT, j = idx % DVT;
             float z = 0.f;
             if (t < Cn) {
-                const size_t off = (((size_t)bb * T + t0 + t) * H + h) * dv + j0 + j;
-                z = to_f32(wg[off]) * to_f32(v[off]);
+                const size_t row = ((size_t)bb * T + t0 + t) * H + h;
+                const size_t off = row * dv + j0 + j;
+                z = to_f32(wg[(a.gates & kGateScalarW) ? row : off]) * to_f32(v[off]);
             }
             sm.Z[t][j] = z;
         }

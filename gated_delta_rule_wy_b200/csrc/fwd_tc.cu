@@ -177,6 +177,8 @@ struct ChunkParams {
     const int *cu_seqlens;
     const int *cu_chunks;
     const int *ntasks_dev;  // H * cu_chunks[B], written by the prefix kernel
+    int gates;              // kGate* bits: a scalar gate is read here, not by the copy engine
+    const __nv_bfloat16 *bg, *wg;
 };
 
 // Where a task's chunk lives: tensor-map coordinates (token t0, sequence bb), head h, and the
@@ -286,14 +288,16 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int row = quarter * 32 + lane;                              // this thread's TMEM lane
 
     const int ntasks = p.cu_seqlens ? *p.ntasks_dev : p.ntasks;
+    const bool bsc = (p.gates & kGateScalarB) != 0, wsc = (p.gates & kGateScalarW) != 0;
+    const uint32_t tx_bytes = TX_BYTES - (bsc ? 16384u : 0u) - (wsc ? 16384u : 0u);
     auto issue_loads = [&](int task) {
         const ChunkLoc L = locate_chunk(p, task);
-        mbar_arrive_expect_tx(&ms.bar_tma, TX_BYTES);
+        mbar_arrive_expect_tx(&ms.bar_tma, tx_bytes);
         tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, L.h, L.t0, L.bb);
         tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, L.h, L.t0, L.bb);
-        tma_load_4d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        if (!bsc) tma_load_4d(sm + OFF_STG_B, &tm_b, &ms.bar_tma, 0, L.h, L.t0, L.bb);
         tma_load_4d(sm + OFF_STG_V, &tm_v, &ms.bar_tma, 0, L.h, L.t0, L.bb);
-        tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, L.h, L.t0, L.bb);
+        if (!wsc) tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, L.h, L.t0, L.bb);
         tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, L.h, L.t0, L.bb);
     };
     if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
@@ -323,7 +327,8 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
     for (int task = blockIdx.x; task < ntasks && !timed_out; task += gridDim.x) {
-        const int Cn = locate_chunk(p, task).Cn;
+        const ChunkLoc loc = locate_chunk(p, task);
+        const int Cn = loc.Cn;
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
         if (tid == 64) bulk_wait_group_read0();  // K~, P and U~ of the previous task have left shared memory
@@ -342,6 +347,30 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 *reinterpret_cast<uint4 *>(sm + OFF_STG_W + t * 256 + o * 16) = z4;
                 *reinterpret_cast<uint4 *>(sm + OFF_STG_LA + t * 512 + o * 32) = z4;
                 *reinterpret_cast<uint4 *>(sm + OFF_STG_LA + t * 512 + o * 32 + 16) = z4;
+            }
+            __syncthreads();
+        }
+        if (bsc || wsc) {
+            // a gate given as one value per token-head: its rows of the staging buffer hold
+            // that value in every channel (zero past the chunk's tokens), so that everything
+            // below treats it as the vector gate it stands for
+            for (int i = tid; i < C * 16; i += NT) {
+                const int t = i >> 4, o = i & 15;
+                const size_t row = ((size_t)loc.bb * p.T + loc.t0 + t) * p.H + loc.h;
+                if (bsc) {
+                    const __nv_bfloat16 g = t < Cn ? p.bg[row] : __float2bfloat16_rn(0.f);
+                    const __nv_bfloat162 g2 = __halves2bfloat162(g, g);
+                    uint4 u;
+                    u.x = u.y = u.z = u.w = *reinterpret_cast<const uint32_t *>(&g2);
+                    *reinterpret_cast<uint4 *>(sm + OFF_STG_B + t * 256 + o * 16) = u;
+                }
+                if (wsc) {
+                    const __nv_bfloat16 g = t < Cn ? p.wg[row] : __float2bfloat16_rn(0.f);
+                    const __nv_bfloat162 g2 = __halves2bfloat162(g, g);
+                    uint4 u;
+                    u.x = u.y = u.z = u.w = *reinterpret_cast<const uint32_t *>(&g2);
+                    *reinterpret_cast<uint4 *>(sm + OFF_STG_W + t * 256 + o * 16) = u;
+                }
             }
             __syncthreads();
         }
@@ -1265,12 +1294,15 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
 {
     const bool varlen = a.cu_seqlens != nullptr;
     const int Bm = varlen ? 1 : a.B;  // tensor-map batch extent: packed sequences share one
+    const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
     CUtensorMap mq, mk, mb, mv, mw, mla, mo;
     if (!make_map(&mq, a.q, false, Bm, a.T, a.H, DK) || !make_map(&mk, a.k, false, Bm, a.T, a.H, DK) ||
-        !make_map(&mb, a.b, false, Bm, a.T, a.H, DK) || !make_map(&mv, a.v, false, Bm, a.T, a.H, DV) ||
-        !make_map(&mw, a.w, false, Bm, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, Bm, a.T, a.H, DK) ||
+        !make_map(&mv, a.v, false, Bm, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, Bm, a.T, a.H, DK) ||
         !make_map(&mo, a.o, false, Bm, a.T, a.H, DV))
         return cudaErrorInvalidValue;
+    // a scalar gate has no tile to copy: its map slot is never used (the q map stands in)
+    if (bsc) mb = mq; else if (!make_map(&mb, a.b, false, Bm, a.T, a.H, DK)) return cudaErrorInvalidValue;
+    if (wsc) mw = mq; else if (!make_map(&mw, a.w, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -1289,7 +1321,10 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    ChunkParams cp{a.B, a.T, a.H, NC, ntasks, ws, a.status, a.cu_seqlens, cu_chunks, ntasks_dev};
+    ChunkParams cp{a.B,         a.T,       a.H,        NC,
+                   ntasks,      ws,        a.status,   a.cu_seqlens,
+                   cu_chunks,   ntasks_dev, a.gates,   static_cast<const __nv_bfloat16 *>(a.b),
+                   static_cast<const __nv_bfloat16 *>(a.w)};
     fwd_chunk_kernel<<<ntasks < nsm ? ntasks : nsm, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

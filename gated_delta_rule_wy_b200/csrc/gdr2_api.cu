@@ -63,6 +63,26 @@ gdr2_status check_ptr(const void *p, const char *name, bool nullable)
     return GDR2_OK;
 }
 
+gdr2_status check_gates(int gates)
+{
+    if (gates < 0 || gates > (GDR2_GATE_SCALAR_B | GDR2_GATE_SCALAR_W))
+        return fail(GDR2_ERR_INVALID_ARG, "gates must combine GDR2_GATE_SCALAR_B and GDR2_GATE_SCALAR_W (got %d)",
+                    gates);
+    return GDR2_OK;
+}
+
+// A vector gate is read by tiles (16-byte aligned, like every tensor); a scalar gate
+// ([..., T, H], one value per token-head) element by element.
+gdr2_status check_gate_ptr(const void *p, const char *name, bool nullable, int scalar, gdr2_dtype dt)
+{
+    if (!scalar) return check_ptr(p, name, nullable);
+    if (!p && !nullable) return fail(GDR2_ERR_INVALID_ARG, "%s is NULL", name);
+    const uintptr_t esz = dt == GDR2_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(p) & (esz - 1)) != 0)
+        return fail(GDR2_ERR_INVALID_ARG, "%s is not aligned to its element size", name);
+    return GDR2_OK;
+}
+
 #define GDR2_TRY(expr)                      \
     do {                                    \
         gdr2_status st_ = (expr);           \
@@ -107,20 +127,21 @@ size_t gdr2_forward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dt
     return gdr2::forward_tc_workspace_bytes(B, T, H);
 }
 
-gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
-                         const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
-                         void *o, float *S_T, float *saved_states, void *workspace, size_t workspace_bytes,
-                         void *stream)
+gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
+                               const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                               const float *S0, void *o, float *S_T, float *saved_states, void *workspace,
+                               size_t workspace_bytes, void *stream)
 {
     GDR2_TRY(check_dims(B, T, H, dk, dv));
     GDR2_TRY(check_dtype(dt));
+    GDR2_TRY(check_gates(gates));
     const bool has_tokens = (long long)B * T * H > 0;
     GDR2_TRY(check_ptr(q, "q", !has_tokens));
     GDR2_TRY(check_ptr(k, "k", !has_tokens));
     GDR2_TRY(check_ptr(v, "v", !has_tokens));
     GDR2_TRY(check_ptr(log_alpha, "log_alpha", !has_tokens));
-    GDR2_TRY(check_ptr(b, "b", !has_tokens));
-    GDR2_TRY(check_ptr(w, "w", !has_tokens));
+    GDR2_TRY(check_gate_ptr(b, "b", !has_tokens, gates & GDR2_GATE_SCALAR_B, dt));
+    GDR2_TRY(check_gate_ptr(w, "w", !has_tokens, gates & GDR2_GATE_SCALAR_W, dt));
     GDR2_TRY(check_ptr(o, "o", !has_tokens));
     GDR2_TRY(check_ptr(S0, "S0", true));
     GDR2_TRY(check_ptr(S_T, "S_T", true));
@@ -146,10 +167,20 @@ gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, con
             return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
     }
     gdr2::FwdArgs a{B,  T,    H,  dk,  dv,           dt == GDR2_BF16, q,         k,               v,      log_alpha,
-                    b,  w,    S0, o,   S_T,          saved_states,    workspace, workspace_bytes, nullptr};
+                    b,  w,    S0, o,   S_T,          saved_states,    workspace, workspace_bytes, nullptr,
+                    nullptr, gates};
     GDR2_TRY(device_status(&a.status));
     if (gdr2::forward_tc_supported(a)) return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward (tcgen05)");
     return launched(gdr2::launch_forward_simt(a, s), "gdr2_forward (simt)");
+}
+
+gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                         const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                         void *o, float *S_T, float *saved_states, void *workspace, size_t workspace_bytes,
+                         void *stream)
+{
+    return gdr2_forward_gated(B, T, H, dk, dv, dt, 0, q, k, v, log_alpha, b, w, S0, o, S_T, saved_states,
+                              workspace, workspace_bytes, stream);
 }
 
 size_t gdr2_forward_varlen_workspace_bytes(int N, int T, int H, int dk, int dv, gdr2_dtype dt)
@@ -159,13 +190,14 @@ size_t gdr2_forward_varlen_workspace_bytes(int N, int T, int H, int dk, int dv, 
     return gdr2::forward_tc_varlen_workspace_bytes(N, T, H);
 }
 
-gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype dt, const int *cu_seqlens,
+gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const int *cu_seqlens,
                                 const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
                                 const void *w, const float *S0, void *o, float *S_T, float *saved_states,
                                 void *workspace, size_t workspace_bytes, void *stream)
 {
     GDR2_TRY(check_dims(N, T, H, dk, dv));
     GDR2_TRY(check_dtype(dt));
+    GDR2_TRY(check_gates(gates));
     if (dt != GDR2_BF16 || dk != 128 || dv != 128)
         return fail(GDR2_ERR_UNSUPPORTED, "packed sequences need bf16 inputs with dk = dv = 128");
     if ((long long)N * H == 0) return GDR2_OK;
@@ -177,8 +209,8 @@ gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype 
     GDR2_TRY(check_ptr(k, "k", !has_tokens));
     GDR2_TRY(check_ptr(v, "v", !has_tokens));
     GDR2_TRY(check_ptr(log_alpha, "log_alpha", !has_tokens));
-    GDR2_TRY(check_ptr(b, "b", !has_tokens));
-    GDR2_TRY(check_ptr(w, "w", !has_tokens));
+    GDR2_TRY(check_gate_ptr(b, "b", !has_tokens, gates & GDR2_GATE_SCALAR_B, dt));
+    GDR2_TRY(check_gate_ptr(w, "w", !has_tokens, gates & GDR2_GATE_SCALAR_W, dt));
     GDR2_TRY(check_ptr(o, "o", !has_tokens));
     GDR2_TRY(check_ptr(S0, "S0", true));
     GDR2_TRY(check_ptr(S_T, "S_T", true));
@@ -199,32 +231,40 @@ gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype 
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
     gdr2::FwdArgs a{N, T, H, dk, dv, true, q, k, v, log_alpha, b, w, S0, o, S_T, saved_states, workspace,
-                    workspace_bytes, nullptr, cu_seqlens};
+                    workspace_bytes, nullptr, cu_seqlens, gates};
     GDR2_TRY(device_status(&a.status));
     if (!gdr2::forward_tc_supported(a))
         return fail(GDR2_ERR_UNSUPPORTED, "the tensor-core forward is not available on this device");
     return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward_varlen (tcgen05)");
 }
 
-gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
-                             const void *v, const float *log_alpha, const void *b, const void *w, float *S,
-                             void *o, void *stream)
+gdr2_status gdr2_decode_step_gated(int N, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
+                                   const void *k, const void *v, const float *log_alpha, const void *b,
+                                   const void *w, float *S, void *o, void *stream)
 {
     GDR2_TRY(check_dims(N, 1, H, dk, dv));
     GDR2_TRY(check_dtype(dt));
+    GDR2_TRY(check_gates(gates));
     const bool any = (long long)N * H > 0;
     GDR2_TRY(check_ptr(q, "q", !any));
     GDR2_TRY(check_ptr(k, "k", !any));
     GDR2_TRY(check_ptr(v, "v", !any));
     GDR2_TRY(check_ptr(log_alpha, "log_alpha", !any));
-    GDR2_TRY(check_ptr(b, "b", !any));
-    GDR2_TRY(check_ptr(w, "w", !any));
+    GDR2_TRY(check_gate_ptr(b, "b", !any, gates & GDR2_GATE_SCALAR_B, dt));
+    GDR2_TRY(check_gate_ptr(w, "w", !any, gates & GDR2_GATE_SCALAR_W, dt));
     GDR2_TRY(check_ptr(S, "S", !any));
     GDR2_TRY(check_ptr(o, "o", !any));
     if (!any) return GDR2_OK;
-    gdr2::DecodeArgs a{N, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S, o, nullptr};
+    gdr2::DecodeArgs a{N, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S, o, nullptr, gates};
     GDR2_TRY(device_status(&a.status));
     return launched(gdr2::launch_decode(a, static_cast<cudaStream_t>(stream)), "gdr2_decode_step");
+}
+
+gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                             const void *v, const float *log_alpha, const void *b, const void *w, float *S,
+                             void *o, void *stream)
+{
+    return gdr2_decode_step_gated(N, H, dk, dv, dt, 0, q, k, v, log_alpha, b, w, S, o, stream);
 }
 
 size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt)

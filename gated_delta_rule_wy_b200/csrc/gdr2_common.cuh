@@ -11,6 +11,13 @@ namespace gdr2 {
 // cumulative decays finite.
 constexpr float kLogAlphaFloor = -64.0f;
 
+// Gate layouts (the gates argument of the gated entry points): a set bit means the gate
+// is one value per token-head ([..., T, H]) instead of a vector over its channels.
+enum : int {
+    kGateScalarB = 1,
+    kGateScalarW = 2,
+};
+
 // Bits of the device status word (one per device, read by gdr2_sync_status).
 enum : unsigned {
     kStatusTimeout = 1u,      // a kernel gave up a bounded wait

@@ -21,6 +21,7 @@ struct FwdArgs {
     size_t workspace_bytes;
     unsigned *status;  // device status word
     const int *cu_seqlens;  // packed sequences: B = their number, T = total tokens (null = dense)
+    int gates;              // kGate* bits: b and/or w one value per token-head
 };
 
 struct DecodeArgs {
@@ -32,6 +33,7 @@ struct DecodeArgs {
     float *S;
     void *o;
     unsigned *status;
+    int gates;  // kGate* bits
 };
 
 struct BwdArgs {

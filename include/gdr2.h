@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 3
+#define GDR2_ABI_VERSION 4
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -74,6 +74,17 @@ typedef enum {
     GDR2_F32 = 0,
     GDR2_BF16 = 1
 } gdr2_dtype;
+
+/*
+ * Gate layouts for the *_gated entry points and gdr2_forward_varlen (bits of
+ * `gates`): by default the erase gate b has d_k entries per token-head and the
+ * write gate w d_v; with a bit set that gate is one value per token-head
+ * ([B, T, H], or [T, H] packed, or [N, H] for decode), the same value in every
+ * channel -- the scalar-gate ablations of the Gated DeltaNet-2 note (sec. 4),
+ * and with both bits and b = w = beta the KDA / Gated DeltaNet gates (sec. 2).
+ */
+#define GDR2_GATE_SCALAR_B 1
+#define GDR2_GATE_SCALAR_W 2
 
 /* ABI version of the loaded library (GDR2_ABI_VERSION it was built with). */
 int gdr2_abi_version(void);
@@ -114,6 +125,17 @@ gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdr2_forward_gated -- gdr2_forward with the gate layouts of `gates`
+ * (GDR2_GATE_* bits); a scalar gate is [B, T, H] in the dtype dt, any element
+ * alignment. Everything else as gdr2_forward; gates = 0 is gdr2_forward.
+ */
+gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates,
+                               const void *q, const void *k, const void *v, const float *log_alpha,
+                               const void *b, const void *w, const float *S0,
+                               void *o, float *S_T, float *saved_states,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdr2_decode_step -- one recurrent token for N*H resident states
  *   (constant-memory decoding, Gated DeltaNet-2 note sec. 1; the per-token
  *   steps of sec. 3). One read and one write of S: with r = S^T(a (.) e) and
@@ -127,6 +149,15 @@ gdr2_status gdr2_decode_step(int N, int H, int dk, int dv, gdr2_dtype dt,
                              const void *q, const void *k, const void *v,
                              const float *log_alpha, const void *b, const void *w,
                              float *S, void *o, void *stream);
+
+/*
+ * gdr2_decode_step_gated -- gdr2_decode_step with the gate layouts of `gates`
+ * (GDR2_GATE_* bits); a scalar gate is [N, H]. gates = 0 is gdr2_decode_step.
+ */
+gdr2_status gdr2_decode_step_gated(int N, int H, int dk, int dv, gdr2_dtype dt, int gates,
+                                   const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const void *b, const void *w,
+                                   float *S, void *o, void *stream);
 
 /* Bytes of device scratch gdr2_forward_varlen needs (N sequences, T tokens in all). */
 size_t gdr2_forward_varlen_workspace_bytes(int N, int T, int H, int dk, int dv, gdr2_dtype dt);
@@ -149,11 +180,12 @@ size_t gdr2_forward_varlen_workspace_bytes(int N, int T, int H, int dk, int dv, 
  *      by head, its chunks in order within a head.
  * scratch: workspace of at least gdr2_forward_varlen_workspace_bytes(...)
  *      bytes, 256-byte aligned.
+ * gates: GDR2_GATE_* bits (0 = vector gates); a scalar gate is [T, H].
  * Supported: bf16 inputs with dk = dv = 128 (GDR2_ERR_UNSUPPORTED otherwise).
  * cu_seqlens is read on the device only: if it breaks the rule above, the call
  * computes nothing and the next gdr2_sync_status returns GDR2_ERR_INVALID_ARG.
  */
-gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype dt, const int *cu_seqlens,
+gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const int *cu_seqlens,
                                 const void *q, const void *k, const void *v, const float *log_alpha,
                                 const void *b, const void *w, const float *S0,
                                 void *o, float *S_T, float *saved_states,

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 3
+    assert lib.gdr2_abi_version() == 4
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -95,17 +95,39 @@ def test_varlen_forward_workspace_query_and_checks(lib):
     assert lib.gdr2_forward_varlen_workspace_bytes(8, 1000, 16, 128, 128, 0) == 0  # fp32: not supported
     p = ctypes.c_void_p(0x10000)
     args = [p] * 12 + [ctypes.c_size_t(1 << 30), ctypes.c_void_p(0)]
-    assert lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 0, *args) == binding.GDR2_ERR_UNSUPPORTED
-    assert lib.gdr2_forward_varlen(2, 64, 4, 64, 128, 1, *args) == binding.GDR2_ERR_UNSUPPORTED
+    assert lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 0, 0, *args) == binding.GDR2_ERR_UNSUPPORTED
+    assert lib.gdr2_forward_varlen(2, 64, 4, 64, 128, 1, 0, *args) == binding.GDR2_ERR_UNSUPPORTED
+    assert lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, 4, *args) == binding.GDR2_ERR_INVALID_ARG
     nul = [ctypes.c_void_p(0)] + [p] * 11 + [ctypes.c_size_t(1 << 30), ctypes.c_void_p(0)]
-    st = lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, *nul)
+    st = lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, 0, *nul)
     assert st == binding.GDR2_ERR_INVALID_ARG and b"cu_seqlens" in lib.gdr2_last_error()
     small = [p] * 12 + [ctypes.c_size_t(16), ctypes.c_void_p(0)]
-    st = lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, *small)
+    st = lib.gdr2_forward_varlen(2, 64, 4, 128, 128, 1, 0, *small)
     assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
     # no sequences or no heads: nothing to do, no pointer needed
-    assert lib.gdr2_forward_varlen(0, 0, 4, 128, 128, 1, *([ctypes.c_void_p(0)] * 12),
+    assert lib.gdr2_forward_varlen(0, 0, 4, 128, 128, 1, 0, *([ctypes.c_void_p(0)] * 12),
                                    ctypes.c_size_t(0), ctypes.c_void_p(0)) == binding.GDR2_OK
+
+
+def test_gated_entry_points_check_the_gate_layout(lib):
+    p = ctypes.c_void_p(0x10000)
+    fwd = [p] * 11 + [ctypes.c_size_t(1 << 30), ctypes.c_void_p(0)]
+    for bad in (-1, 4, 7):
+        st = lib.gdr2_forward_gated(1, 64, 2, 128, 128, 1, bad, *fwd)
+        assert st == binding.GDR2_ERR_INVALID_ARG and b"gates" in lib.gdr2_last_error()
+        st = lib.gdr2_decode_step_gated(4, 2, 128, 128, 1, bad, *([p] * 9))
+        assert st == binding.GDR2_ERR_INVALID_ARG and b"gates" in lib.gdr2_last_error()
+    # a scalar gate needs element alignment only; a vector gate 16 bytes
+    odd = ctypes.c_void_p(0x10002)
+    args = [p, p, p, p, odd, odd] + [p] * 5 + [ctypes.c_size_t(0), ctypes.c_void_p(0)]
+    st = lib.gdr2_forward_gated(1, 64, 2, 128, 128, 1, 0, *args)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"16-byte" in lib.gdr2_last_error()
+    st = lib.gdr2_forward_gated(1, 64, 2, 128, 128, 1, 3, *args)  # passes the gates, stops at the workspace
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
+    odd1 = ctypes.c_void_p(0x10001)
+    args = [p, p, p, p, odd1, p] + [p] * 5 + [ctypes.c_size_t(0), ctypes.c_void_p(0)]
+    st = lib.gdr2_forward_gated(1, 64, 2, 128, 128, 1, 1, *args)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"element size" in lib.gdr2_last_error()
 
 
 def test_binding_validates_before_calling():
