@@ -329,6 +329,18 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int task = blockIdx.x; task < ntasks && !timed_out; task += gridDim.x) {
         const ChunkLoc loc = locate_chunk(p, task);
         const int Cn = loc.Cn;
+        // a scalar gate: this thread's four rows (t = tid / 16 + 16 k), read while the copies land
+        static_assert(C * 16 == 4 * NT, "four 16-byte pieces of a staging row set per thread");
+        __nv_bfloat16 gb4[4], gw4[4];
+        if (bsc || wsc) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = (tid >> 4) + 16 * k;
+                const size_t row = ((size_t)loc.bb * p.T + loc.t0 + t) * p.H + loc.h;
+                gb4[k] = (bsc && t < Cn) ? p.bg[row] : __float2bfloat16_rn(0.f);
+                gw4[k] = (wsc && t < Cn) ? p.wg[row] : __float2bfloat16_rn(0.f);
+            }
+        }
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
         if (tid == 64) bulk_wait_group_read0();  // K~, P and U~ of the previous task have left shared memory
@@ -353,26 +365,24 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (bsc || wsc) {
             // a gate given as one value per token-head: its rows of the staging buffer hold
             // that value in every channel (zero past the chunk's tokens), so that everything
-            // below treats it as the vector gate it stands for
-            for (int i = tid; i < C * 16; i += NT) {
-                const int t = i >> 4, o = i & 15;
-                const size_t row = ((size_t)loc.bb * p.T + loc.t0 + t) * p.H + loc.h;
+            // below treats it as the vector gate it stands for (first read after the barrier
+            // that ends the decay scan)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = (tid >> 4) + 16 * k, o = tid & 15;
                 if (bsc) {
-                    const __nv_bfloat16 g = t < Cn ? p.bg[row] : __float2bfloat16_rn(0.f);
-                    const __nv_bfloat162 g2 = __halves2bfloat162(g, g);
+                    const __nv_bfloat162 g2 = __halves2bfloat162(gb4[k], gb4[k]);
                     uint4 u;
                     u.x = u.y = u.z = u.w = *reinterpret_cast<const uint32_t *>(&g2);
                     *reinterpret_cast<uint4 *>(sm + OFF_STG_B + t * 256 + o * 16) = u;
                 }
                 if (wsc) {
-                    const __nv_bfloat16 g = t < Cn ? p.wg[row] : __float2bfloat16_rn(0.f);
-                    const __nv_bfloat162 g2 = __halves2bfloat162(g, g);
+                    const __nv_bfloat162 g2 = __halves2bfloat162(gw4[k], gw4[k]);
                     uint4 u;
                     u.x = u.y = u.z = u.w = *reinterpret_cast<const uint32_t *>(&g2);
                     *reinterpret_cast<uint4 *>(sm + OFF_STG_W + t * 256 + o * 16) = u;
                 }
             }
-            __syncthreads();
         }
 
         // ================= prep: cumulative decay and decay-weighted operands =================
