@@ -25,7 +25,8 @@ namespace {
 constexpr int NT = 256;
 constexpr int NW = NT / 32;
 
-template <typename TIn, int DK, int DV>
+// GATED: a scalar gate may be in use (the other instantiation has vector gates only).
+template <typename TIn, int DK, int DV, bool GATED>
 __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a)
 {
     constexpr int LPR = DV / 4;        // lanes per state row
@@ -50,7 +51,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeArgs a)
 
     const TIn *q = static_cast<const TIn *>(a.q) + (size_t)nh * DK;
     const TIn *k = static_cast<const TIn *>(a.k) + (size_t)nh * DK;
-    const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
+    const bool bsc = GATED && (a.gates & kGateScalarB) != 0, wsc = GATED && (a.gates & kGateScalarW) != 0;
     const TIn *bg = static_cast<const TIn *>(a.b) + (size_t)nh * (bsc ? 1 : DK);
     const float *la = a.log_alpha + (size_t)nh * DK;
     const TIn *v = static_cast<const TIn *>(a.v) + (size_t)nh * DV;
@@ -133,10 +134,17 @@ template <typename TIn>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s)
 {
     const int grid = a.N * a.H;
-    if (a.dk == 128 && a.dv == 128) decode_kernel<TIn, 128, 128><<<grid, NT, 0, s>>>(a);
-    else if (a.dk == 128 && a.dv == 64) decode_kernel<TIn, 128, 64><<<grid, NT, 0, s>>>(a);
-    else if (a.dk == 64 && a.dv == 128) decode_kernel<TIn, 64, 128><<<grid, NT, 0, s>>>(a);
-    else decode_kernel<TIn, 64, 64><<<grid, NT, 0, s>>>(a);
+    if (a.gates) {
+        if (a.dk == 128 && a.dv == 128) decode_kernel<TIn, 128, 128, true><<<grid, NT, 0, s>>>(a);
+        else if (a.dk == 128 && a.dv == 64) decode_kernel<TIn, 128, 64, true><<<grid, NT, 0, s>>>(a);
+        else if (a.dk == 64 && a.dv == 128) decode_kernel<TIn, 64, 128, true><<<grid, NT, 0, s>>>(a);
+        else decode_kernel<TIn, 64, 64, true><<<grid, NT, 0, s>>>(a);
+    } else {
+        if (a.dk == 128 && a.dv == 128) decode_kernel<TIn, 128, 128, false><<<grid, NT, 0, s>>>(a);
+        else if (a.dk == 128 && a.dv == 64) decode_kernel<TIn, 128, 64, false><<<grid, NT, 0, s>>>(a);
+        else if (a.dk == 64 && a.dv == 128) decode_kernel<TIn, 64, 128, false><<<grid, NT, 0, s>>>(a);
+        else decode_kernel<TIn, 64, 64, false><<<grid, NT, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 

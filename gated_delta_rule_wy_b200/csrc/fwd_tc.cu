@@ -187,10 +187,11 @@ struct ChunkLoc {
     int h, t0, bb, Cn;
 };
 
+template <bool GENERAL>
 __device__ __forceinline__ ChunkLoc locate_chunk(const ChunkParams &p, int task)
 {
     ChunkLoc L;
-    if (!p.cu_seqlens) {
+    if (!GENERAL || !p.cu_seqlens) {
         const int bh = task / p.NC, n = task % p.NC;
         L.bb = bh / p.H;
         L.h = bh % p.H;
@@ -257,6 +258,9 @@ __global__ void __launch_bounds__(1024) varlen_prefix_kernel(const int *cu, int 
 constexpr uint32_t CK_M = 0, CK_U = 128, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384, CK_AP1 = 416;
 constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W_0, W_1 once those are read
 
+// GENERAL: packed sequences and/or scalar gates may be in use; the other instantiation is
+// the dense, vector-gate kernel with those branches compiled away.
+template <bool GENERAL>
 __global__ void __launch_bounds__(NT, 1)
 fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
@@ -287,11 +291,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);  // this warp's TMEM lanes
     const int row = quarter * 32 + lane;                              // this thread's TMEM lane
 
-    const int ntasks = p.cu_seqlens ? *p.ntasks_dev : p.ntasks;
-    const bool bsc = (p.gates & kGateScalarB) != 0, wsc = (p.gates & kGateScalarW) != 0;
+    const int ntasks = (GENERAL && p.cu_seqlens) ? *p.ntasks_dev : p.ntasks;
+    const bool bsc = GENERAL && (p.gates & kGateScalarB) != 0, wsc = GENERAL && (p.gates & kGateScalarW) != 0;
     const uint32_t tx_bytes = TX_BYTES - (bsc ? 16384u : 0u) - (wsc ? 16384u : 0u);
     auto issue_loads = [&](int task) {
-        const ChunkLoc L = locate_chunk(p, task);
+        const ChunkLoc L = locate_chunk<GENERAL>(p, task);
         mbar_arrive_expect_tx(&ms.bar_tma, tx_bytes);
         tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, L.h, L.t0, L.bb);
         tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, L.h, L.t0, L.bb);
@@ -327,7 +331,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
     for (int task = blockIdx.x; task < ntasks && !timed_out; task += gridDim.x) {
-        const ChunkLoc loc = locate_chunk(p, task);
+        const ChunkLoc loc = locate_chunk<GENERAL>(p, task);
         const int Cn = loc.Cn;
         // a scalar gate: this thread's four rows (t = tid / 16 + 16 k), read while the copies land
         static_assert(C * 16 == 4 * NT, "four 16-byte pieces of a staging row set per thread");
@@ -345,10 +349,10 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
         if (tid == 64) bulk_wait_group_read0();  // K~, P and U~ of the previous task have left shared memory
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
-        if (Cn < C) {
-            // a partial chunk: the rows past the sequence hold zeros (dense: the copy engine's
-            // fill past T) or the next sequence's tokens (packed); zero them, which makes those
-            // rows inert in every product
+        if (GENERAL && Cn < C) {
+            // a packed sequence's partial chunk: the rows past its end hold the next sequence's
+            // tokens (dense chunks get zeros from the copy engine's fill past T); zero them,
+            // which makes those rows inert in every product
             for (int i = tid; i < (C - Cn) * 16; i += NT) {
                 const int t = Cn + (i >> 4), o = i & 15;
                 const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
@@ -1313,8 +1317,9 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     // a scalar gate has no tile to copy: its map slot is never used (the q map stands in)
     if (bsc) mb = mq; else if (!make_map(&mb, a.b, false, Bm, a.T, a.H, DK)) return cudaErrorInvalidValue;
     if (wsc) mw = mq; else if (!make_map(&mw, a.w, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    const bool general = varlen || bsc || wsc;
+    cudaError_t e = cudaFuncSetAttribute(general ? fwd_chunk_kernel<true> : fwd_chunk_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(fwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC_SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -1335,7 +1340,11 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
                    ntasks,      ws,        a.status,   a.cu_seqlens,
                    cu_chunks,   ntasks_dev, a.gates,   static_cast<const __nv_bfloat16 *>(a.b),
                    static_cast<const __nv_bfloat16 *>(a.w)};
-    fwd_chunk_kernel<<<ntasks < nsm ? ntasks : nsm, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
+    const int grid = ntasks < nsm ? ntasks : nsm;
+    if (general)
+        fwd_chunk_kernel<true><<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
+    else
+        fwd_chunk_kernel<false><<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     ScanParams sp{a.B,          a.T,          a.H,    NC,       ntasks,    ws,
