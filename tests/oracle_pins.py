@@ -346,6 +346,44 @@ def check_decode_matches_forward(orc, seed=13):
     assert o0.shape == (B, 0, H, dv) and np.array_equal(S00, S0)
 
 
+# ---------------------------------------------------------------------------
+# P12  Block epilogue, y = RMSNorm(o) weight (.) silu(g) (GDN2 sec. 3, block data flow):
+#      closed forms and invariants of the norm and of the gate
+# ---------------------------------------------------------------------------
+def pin_output_norm_gate(orc=None, seed=14, OB=None):
+    if OB is None:
+        from oracle import block as OB
+
+    rng = np.random.default_rng(seed)
+    n, dv, eps = 7, 16, 1e-6
+    o = rng.standard_normal((n, dv))
+    wgt = rng.uniform(0.5, 1.5, dv)
+    g = rng.standard_normal((n, dv))
+    # silu: silu(x) - silu(-x) = x; silu(0) = 0; silu(x) ~ x for large x, ~ 0 for very negative x
+    x = rng.standard_normal(50) * 3
+    _close(OB.silu(x) - OB.silu(-x), x, 1e-14, "silu odd part")
+    assert OB.silu(0.0) == 0.0 and abs(OB.silu(40.0) - 40.0) < 1e-12 and abs(OB.silu(-40.0)) < 1e-15
+    # a constant row c 1 normalises to sign(c) |c| / sqrt(c^2 + eps)
+    c = -2.5
+    y = OB.output_norm_gate(np.full((1, dv), c), weight=wgt, eps=eps)
+    _close(y, np.sign(c) * abs(c) / np.sqrt(c * c + eps) * wgt[None], 1e-14, "constant row")
+    # the normalised row (unit weight, no gate) has mean square ms / (ms + eps) and scale invariance
+    y1 = OB.output_norm_gate(o, weight=np.ones(dv), eps=eps)
+    ms = np.mean(o * o, axis=-1)
+    _close(np.mean(y1 * y1, axis=-1), ms / (ms + eps), 1e-13, "rms of the output")
+    _close(OB.output_norm_gate(37.0 * o, weight=wgt, eps=0.0), OB.output_norm_gate(o, weight=wgt, eps=0.0), 1e-13,
+           "scale invariance")
+    # a zero gate closes the output; the gate factor is the same with or without the norm
+    assert np.all(OB.output_norm_gate(o, g=np.zeros_like(o), weight=wgt) == 0.0)
+    _close(OB.output_norm_gate(o, g=g, weight=wgt) / OB.output_norm_gate(o, weight=wgt),
+           OB.output_norm_gate(np.ones_like(o), g=g), 1e-12, "gate factor")
+    # an open gate (g large and positive) passes the normalised output through, scaled by g
+    _close(OB.output_norm_gate(o, g=np.full_like(o, 40.0), weight=wgt), 40.0 * OB.output_norm_gate(o, weight=wgt),
+           1e-12, "open gate")
+    # absent factors: identity
+    assert np.array_equal(OB.output_norm_gate(o), o)
+
+
 ALL_PINS = [pin_kda, pin_gated_deltanet, pin_deltanet, pin_full_reset, pin_no_erase_closed_form,
             pin_one_hot_slots, pin_objective_stationarity, pin_exact_write, pin_dense_product,
-            pin_split_and_linearity, pin_backward_fd, pin_backward_fd_t32_d16]
+            pin_split_and_linearity, pin_backward_fd, pin_backward_fd_t32_d16, pin_output_norm_gate]

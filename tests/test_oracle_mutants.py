@@ -66,3 +66,32 @@ def test_mutant_is_caught(tmp_path, name, old, new):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"mutant '{name}' passed every pin"
+
+
+# Mistakes planted in the block epilogue (oracle/block.py); pin P12 must reject each.
+BLOCK_MUTANTS = [
+    ("rms over the sum, not the mean", "np.mean(y * y, axis=-1, keepdims=True)", "np.sum(y * y, axis=-1, keepdims=True)"),
+    ("epsilon dropped", "np.sqrt(ms + eps)", "np.sqrt(ms)"),
+    ("epsilon outside the root", "np.sqrt(ms + eps)", "(np.sqrt(ms) + eps)"),
+    ("sigmoid gate instead of silu", "return x / (1.0 + np.exp(-x))", "return 1.0 / (1.0 + np.exp(-x))"),
+    ("gate sign flipped", "y = y * silu(g)", "y = y * silu(-np.asarray(g))"),
+    ("weight inside the norm", "y = y / np.sqrt(ms + eps) * np.asarray(weight, dtype=np.float64)",
+     "y = y * np.asarray(weight, dtype=np.float64) / np.sqrt(np.mean((y * weight) ** 2, axis=-1, keepdims=True) + eps)"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", BLOCK_MUTANTS, ids=[m[0] for m in BLOCK_MUTANTS])
+def test_block_mutant_is_caught(tmp_path, name, old, new):
+    import importlib.util
+
+    import oracle_pins as P
+
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "block.py")).read()
+    assert src.count(old) == 1, f"mutation site not found: {old}"
+    mpath = tmp_path / "block_mutant.py"
+    mpath.write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location("block_mutant", mpath)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with pytest.raises(AssertionError):
+        P.pin_output_norm_gate(OB=mod)
