@@ -360,6 +360,28 @@ def bench_components(dev, stream, peaks):
                         "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3),
                         "algorithmic_bytes": alg, "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del xs, o, ws, beta
+    # the same forward with the block's output epilogue (RMSNorm and SiLU gate) in the output store
+    xs = I.make_forward_inputs(**c).to(dev)
+    g, wt = I.make_epilogue_inputs((c["B"], c["T"], c["H"], c["dv"]), c["dv"], seed=1009)
+    g, wt = g.to(dev), wt.to(dev)
+    o = torch.empty_like(xs.v)
+    ws = torch.empty(gdr2_forward_workspace_bytes(c["B"], c["T"], c["H"], c["dk"], c["dv"], c["dtype"]),
+                     dtype=torch.uint8, device=dev)
+
+    def fwd_epi():
+        gdr2_forward(xs.q, xs.k, xs.v, xs.log_alpha, xs.b, xs.w, None, out=o, workspace=ws, out_gate=g,
+                     norm_weight=wt)
+
+    for _ in range(3):
+        fwd_epi()
+    ms = statistics.median(time_steps(fwd_epi, 20, stream))
+    gdr2_sync_status()
+    alg = tokens * c["H"] * (BYTES_PER_TOKEN_HEAD + 2 * c["dv"]) + c["B"] * c["H"] * c["dk"] * c["dv"] * 4
+    out["epilogue"] = {"workload": "B=4 H=16 T=4096 d=128 bf16, output RMSNorm x weight x SiLU(gate) fused "
+                                   "into the output store",
+                       "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3),
+                       "algorithmic_bytes": alg, "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del xs, o, ws, g, wt
     return out
 
 

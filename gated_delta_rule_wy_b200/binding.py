@@ -25,6 +25,7 @@ _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIM
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
 EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspace_bytes", "gdr2_forward",
                     "gdr2_forward_gated", "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen",
+                    "gdr2_forward_ex",
                     "gdr2_decode_step", "gdr2_decode_step_gated",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
                     "gdr2_sync_status")
@@ -66,6 +67,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_forward_varlen_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.gdr2_forward_varlen.restype = I
         lib.gdr2_forward_varlen.argtypes = [I, I, I, I, I, I, I] + [P] * 12 + [Z, P]
+        lib.gdr2_forward_ex.restype = I
+        lib.gdr2_forward_ex.argtypes = [I, I, I, I, I, I, I] + [P] * 8 + [P, P, ctypes.c_float] + [P] * 4 + [Z, P]
         lib.gdr2_forward_gated.restype = I
         lib.gdr2_forward_gated.argtypes = [I, I, I, I, I, I, I] + [P] * 11 + [Z, P]
         lib.gdr2_decode_step_gated.restype = I
@@ -126,6 +129,19 @@ def _gates(b, w, lead):
     return g
 
 
+def _epilogue(out_gate, norm_weight, o_shape, dv, dt, dev):
+    """Checks the output gate and norm weight; True when either is given."""
+    if out_gate is not None:
+        _check(out_gate, "out_gate", o_shape, dt)
+        if out_gate.device != dev:
+            raise ValueError("out_gate must be on the inputs' device")
+    if norm_weight is not None:
+        _check(norm_weight, "norm_weight", (dv,), torch.float32)
+        if norm_weight.device != dev:
+            raise ValueError("norm_weight must be on the inputs' device")
+    return out_gate is not None or norm_weight is not None
+
+
 def _raise(lib, st):
     if st != GDR2_OK:
         raise GDR2Error(st, lib.gdr2_last_error().decode(errors="replace"))
@@ -151,12 +167,14 @@ def gdr2_forward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
 
 
 def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_states=False,
-                 out=None, workspace=None, stream=None):
+                 out=None, workspace=None, stream=None, out_gate=None, norm_weight=None, norm_eps=1e-6):
     """Chunkwise forward. Returns (o, S_T, saved_states); S_T / saved_states may be None.
 
     q, k, b: [B, T, H, dk]; v, w: [B, T, H, dv] (fp32 or bf16, one dtype);
     log_alpha: [B, T, H, dk] fp32; S0: [B, H, dk, dv] fp32 or None.
     b and/or w may instead be [B, T, H]: one gate value per token-head (scalar gates).
+    out_gate ([B, T, H, dv], o's dtype) and norm_weight ([dv] fp32) apply the block's output
+    epilogue o / rms(o) * norm_weight * silu(out_gate) in the kernel (bf16, d = 128 only).
     """
     lib = load_library()
     B, T, H, dk = q.shape
@@ -179,9 +197,15 @@ def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_st
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.gdr2_forward_gated(B, T, H, dk, dv, _dt(q), gates, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-                                _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
-                                ctypes.c_size_t(ws_bytes), _stream(stream))
+    if _epilogue(out_gate, norm_weight, (B, T, H, dv), dv, dt, dev):
+        st = lib.gdr2_forward_ex(B, T, H, dk, dv, _dt(q), gates, None, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                 _ptr(b), _ptr(w), _ptr(S0), _ptr(out_gate), _ptr(norm_weight),
+                                 ctypes.c_float(norm_eps), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
+                                 ctypes.c_size_t(ws_bytes), _stream(stream))
+    else:
+        st = lib.gdr2_forward_gated(B, T, H, dk, dv, _dt(q), gates, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                    _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
+                                    ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
     return o, S_T, saved
 
@@ -193,13 +217,14 @@ def gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dtype=torch.bfloat16) -
 
 
 def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_state=True, save_states=False,
-                        out=None, workspace=None, stream=None):
+                        out=None, workspace=None, stream=None, out_gate=None, norm_weight=None, norm_eps=1e-6):
     """Forward over packed sequences. Returns (o, S_T, saved_states).
 
     q, k, b: [T, H, dk] (or [1, T, H, dk]); v, w: [T, H, dv]; bf16; log_alpha [T, H, dk] fp32;
     cu_seqlens: int32 [N + 1] on the device; S0: [N, H, dk, dv] fp32 or None; b and/or w may
     be [T, H] (scalar gates). saved_states,
     when asked for, is [H * (ceil(T / 64) + N), dk, dv] (see include/gdr2.h for the order).
+    out_gate ([T, H, dv] bf16) and norm_weight ([dv] fp32): the output epilogue, as in gdr2_forward.
     """
     lib = load_library()
     sq4 = lambda t: None if t is None else (t[0] if t.dim() == 4 else t)  # noqa: E731
@@ -230,9 +255,16 @@ def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.gdr2_forward_varlen(N, T, H, dk, dv, _dt(q), gates, _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
-                                 _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved),
-                                 _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream(stream))
+    out_gate = sq4(out_gate)
+    if _epilogue(out_gate, norm_weight, (T, H, dv), dv, dt, dev):
+        st = lib.gdr2_forward_ex(N, T, H, dk, dv, _dt(q), gates, _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(out_gate), _ptr(norm_weight),
+                                 ctypes.c_float(norm_eps), _ptr(o), _ptr(S_T), _ptr(saved), _ptr(workspace),
+                                 ctypes.c_size_t(ws_bytes), _stream(stream))
+    else:
+        st = lib.gdr2_forward_varlen(N, T, H, dk, dv, _dt(q), gates, _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(saved),
+                                     _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
     return o, S_T, saved
 

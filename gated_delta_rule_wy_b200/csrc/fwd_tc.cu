@@ -993,7 +993,10 @@ constexpr uint32_t SC_SLOT0 = 0;
 constexpr uint32_t SC_SLOT1 = SLOT_BYTES;          // 90112, 1024-aligned
 constexpr uint32_t SC_O = 2 * SLOT_BYTES;          // O tile [64 t][128 j] bf16
 constexpr uint32_t SC_MISC = SC_O + 16384;
-constexpr uint32_t SC_SMEM_BYTES = SC_MISC + 1280 + 1024;
+constexpr uint32_t SC_EPI = SC_MISC + 1280;        // output norm: per-warp sums [4][64], then 1/rms [64]
+constexpr uint32_t SC_G = SC_MISC + 4096;          // output gate tile [64 t][128 j] bf16 (1024-aligned)
+static_assert(SC_EPI + 1280 <= SC_G, "norm scratch overlaps the gate tile");
+static_assert(SC_G % 1024 == 0, "gate tile alignment");
 constexpr uint32_t SC_REG = 256;                    // region r at columns 256 r: O^T then S^T
 constexpr uint32_t SC_OT = 0, SC_ST = 64;           // offsets within a region
 constexpr uint32_t SC_SA = 448;                     // S^T in bf16, two values per column (64 columns)
@@ -1002,8 +1005,9 @@ constexpr uint32_t SC_COLS = 512;
 struct ScanMisc {
     uint64_t bar_full[2];
     uint64_t bar_mma;
+    uint64_t bar_g;   // the output gate tile of the chunk being stored
     uint32_t tmem_base;
-    int pad;
+    int g_ok;         // that tile arrived (as seen by thread 0, for warps 0-3)
     alignas(16) float gam[2][DK];  // bulk-copy destination and float4 reads: 16-byte aligned
 };
 static_assert(sizeof(ScanMisc) <= 1280, "scan misc region");
@@ -1019,10 +1023,41 @@ struct ScanParams {
     const int *cu_seqlens;  // packed sequences (null when dense), as in ChunkParams
     const int *cu_chunks;
     __nv_bfloat16 *o;       // for the row-by-row store of a packed sequence's last, partial tile
+    // block epilogue on the way out: o <- o / rms(o) * norm_weight (.) silu(gate), each optional
+    const float *norm_weight;  // [DV] (with kEpiNorm)
+    float norm_eps;
 };
 
+// Output epilogue of fwd_scan_kernel (template bits): RMSNorm with a weight, SiLU gate.
+constexpr int kEpiNorm = 1, kEpiGate = 2;
+
+// Dynamic shared memory of an instantiation (+1 KB for aligning the base): the regions
+// an epilogue does not use are left out.
+constexpr uint32_t scan_smem_bytes(int epi)
+{
+    return ((epi & kEpiGate) ? SC_G + 16384 : (epi & kEpiNorm) ? SC_EPI + 1280 : SC_MISC + 1280) + 1024;
+}
+
+// Sum vals over the 32 lanes of a warp for each of its N entries; on return lane L holds, in
+// vals[0 .. N/32), the sums of the N/32 entries from (N/32) L on.
+template <int N>
+__device__ __forceinline__ void transpose_reduce32(float (&vals)[N], int lane)
+{
+#pragma unroll
+    for (int o = 16, n = N; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? vals[i] : vals[i + n / 2];
+            const float keep = upper ? vals[i + n / 2] : vals[i];
+            vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
+template <int EPI>
 __global__ void __launch_bounds__(NT, 1)
-fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
+fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g, ScanParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm =
@@ -1042,6 +1077,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         mbar_init(&ms.bar_full[0], 1);
         mbar_init(&ms.bar_full[1], 1);
         mbar_init(&ms.bar_mma, 1);
+        mbar_init(&ms.bar_g, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1074,10 +1110,19 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         bulk_load(ms.gam[sl], p.ws + (size_t)p.ntasks * SLOT_BYTES + task * GAMMA_BYTES, GAMMA_BYTES,
                   &ms.bar_full[sl]);
     };
+    bool g_inflight = false;  // thread 0: a gate tile was issued and not yet seen to land
+    auto issue_gate = [&](int m) {  // the output gate tile of chunk m (rows past the sequence unused)
+        mbar_arrive_expect_tx(&ms.bar_g, C * DV * 2);
+        tma_load_4d(sm + SC_G, &tm_g, &ms.bar_g, 0, h, tstart + m * C, tb);
+        g_inflight = true;
+    };
     if (tid == 0) {
         if (NC > 0) issue_slot(0);
         if (NC > 1) issue_slot(1);
+        if ((EPI & kEpiGate) && NC > 0) issue_gate(0);
     }
+    uint32_t ph_g = 0;
+    bool g_failed = false;  // a gate tile that never arrived: stop waiting for the later ones
     // initial state S^T[j][c] = S0[c][j] into region 1 (chunk 0 reads the region of "chunk -1")
     {
         float v[32];
@@ -1104,15 +1149,63 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         return __syncthreads_or(!ok) == 0;
     };
 
-    // O^T of chunk m -> bf16 tile [t][j] -> one TMA store (rows past T are clipped).
-    // Warps 0-3 only (thread = TMEM lane, all 64 columns), under named barrier 1, so
-    // they run while the MMA issuer in warp 4 is busy with the next chunk.
+    // O^T of chunk m -> (epilogue) -> bf16 tile [t][j] -> one TMA store (rows past T are
+    // clipped). Warps 0-3 only (thread = TMEM lane = value channel j, all 64 tokens), under
+    // named barrier 1, so they run while the MMA issuer in warp 4 is busy with the next
+    // chunk (spreading this over all 8 warps measured slower: the extra TMEM traffic
+    // stretches the chunk's MMAs).
     auto store_o = [&](int m) {
         if (tid == 0) bulk_wait_group_read0();  // the previous tile has left shared memory
         named_barrier(1, 128);
         float o0[32], o1[32];
         const uint32_t ot_col = SC_REG * (m & 1) + SC_OT;
         tmem_ld32x2(tm_lane + ot_col, tm_lane + ot_col + 32, o0, o1);
+        if constexpr ((EPI & kEpiNorm) != 0) {
+            // RMSNorm over the value channels of each token: this thread holds channel j of all
+            // 64 tokens; sums of squares over a warp's 32 channels, then over the 4 warps
+            float *red = reinterpret_cast<float *>(sm + SC_EPI);  // [4][64], then 1/rms at [256 ..)
+            float sq[64];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                sq[i] = o0[i] * o0[i];
+                sq[32 + i] = o1[i] * o1[i];
+            }
+            transpose_reduce32<64>(sq, lane);  // lane L: tokens 2L and 2L + 1
+            red[quarter * 64 + 2 * lane] = sq[0];
+            red[quarter * 64 + 2 * lane + 1] = sq[1];
+            named_barrier(1, 128);
+            if (tid < 64)
+                red[256 + tid] = rsqrtf((red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid]) * (1.f / DV) +
+                                        p.norm_eps);
+            named_barrier(1, 128);
+            const float wj = p.norm_weight[j];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                o0[i] *= red[256 + i] * wj;
+                o1[i] *= red[256 + 32 + i] * wj;
+            }
+        }
+        if constexpr ((EPI & kEpiGate) != 0) {
+            if (tid == 0) {
+                ms.g_ok = (!g_failed && mbar_wait_bounded(&ms.bar_g, ph_g, kWaitLimitNs)) ? 1 : 0;
+                if (ms.g_ok) g_inflight = false;
+            }
+            named_barrier(1, 128);
+            ph_g ^= 1u;
+            if (ms.g_ok) {
+                const __nv_bfloat16 *gt = reinterpret_cast<const __nv_bfloat16 *>(sm + SC_G) + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    // silu(g) = g / (1 + exp(-g)); a huge denominator (g below about -87) gives 0
+                    const float g0 = __bfloat162float(gt[i * DV]), g1 = __bfloat162float(gt[(32 + i) * DV]);
+                    o0[i] *= __fdividef(g0, 1.f + __expf(-g0));
+                    o1[i] *= __fdividef(g1, 1.f + __expf(-g1));
+                }
+            } else {
+                g_failed = true;
+                if (tid == 0) atomicOr(p.status, kStatusTimeout);
+            }
+        }
         __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -1122,6 +1215,8 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_barrier(1, 128);
+        // every read of this chunk's gate tile is done: the next one may land
+        if ((EPI & kEpiGate) && !g_failed && tid == 0 && m + 1 < NC) issue_gate(m + 1);
         const int rows = min(C, len - m * C);
         if (p.cu_seqlens && rows < C) {
             // a packed sequence's partial last tile: its rows only (a tile store would write
@@ -1238,6 +1333,8 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
         }
     }
     if (tid == 0) bulk_wait_group0();
+    // a gate tile still on its way (only after a timeout): let it land before shared memory goes
+    if (tid == 0 && g_inflight) mbar_wait_bounded(&ms.bar_g, ph_g, kWaitLimitNs);
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
@@ -1309,7 +1406,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     const bool varlen = a.cu_seqlens != nullptr;
     const int Bm = varlen ? 1 : a.B;  // tensor-map batch extent: packed sequences share one
     const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
-    CUtensorMap mq, mk, mb, mv, mw, mla, mo;
+    CUtensorMap mq, mk, mb, mv, mw, mla, mo, mg;
     if (!make_map(&mq, a.q, false, Bm, a.T, a.H, DK) || !make_map(&mk, a.k, false, Bm, a.T, a.H, DK) ||
         !make_map(&mv, a.v, false, Bm, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, Bm, a.T, a.H, DK) ||
         !make_map(&mo, a.o, false, Bm, a.T, a.H, DV))
@@ -1317,11 +1414,17 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     // a scalar gate has no tile to copy: its map slot is never used (the q map stands in)
     if (bsc) mb = mq; else if (!make_map(&mb, a.b, false, Bm, a.T, a.H, DK)) return cudaErrorInvalidValue;
     if (wsc) mw = mq; else if (!make_map(&mw, a.w, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
+    // the output gate has the layout of o; without one the o map stands in, unused
+    if (!a.out_gate) mg = mo; else if (!make_map(&mg, a.out_gate, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
     const bool general = varlen || bsc || wsc;
     cudaError_t e = cudaFuncSetAttribute(general ? fwd_chunk_kernel<true> : fwd_chunk_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(fwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC_SMEM_BYTES);
+    const int epi = (a.norm_weight ? kEpiNorm : 0) | (a.out_gate ? kEpiGate : 0);
+    void (*scan)(const CUtensorMap, const CUtensorMap, ScanParams) =
+        epi == 0 ? fwd_scan_kernel<0> : epi == kEpiNorm ? fwd_scan_kernel<kEpiNorm>
+        : epi == kEpiGate ? fwd_scan_kernel<kEpiGate> : fwd_scan_kernel<kEpiNorm | kEpiGate>;
+    e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem_bytes(epi));
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1349,18 +1452,18 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     ScanParams sp{a.B,          a.T,          a.H,    NC,       ntasks,    ws,
                   a.S0,         a.S_T,        a.saved_states, a.status, a.cu_seqlens, cu_chunks,
-                  static_cast<__nv_bfloat16 *>(a.o)};
+                  static_cast<__nv_bfloat16 *>(a.o), a.norm_weight, a.norm_eps};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.H);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = SC_SMEM_BYTES;
+    cfg.dynamicSmemBytes = scan_smem_bytes(epi);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fwd_scan_kernel, mo, sp);
+    return cudaLaunchKernelEx(&cfg, scan, mo, mg, sp);
 }
 
 }  // namespace gdr2

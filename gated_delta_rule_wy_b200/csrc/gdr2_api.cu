@@ -127,15 +127,29 @@ size_t gdr2_forward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dt
     return gdr2::forward_tc_workspace_bytes(B, T, H);
 }
 
-gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
-                               const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
-                               const float *S0, void *o, float *S_T, float *saved_states, void *workspace,
-                               size_t workspace_bytes, void *stream)
+// All forward entry points: dense (cu_seqlens = NULL) or packed, gates, epilogue.
+static gdr2_status forward_impl(const char *who, int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates,
+                                const int *cu_seqlens, bool packed, const void *q, const void *k, const void *v,
+                                const float *log_alpha, const void *b, const void *w, const float *S0,
+                                const void *out_gate, const float *norm_weight, float norm_eps, void *o, float *S_T,
+                                float *saved_states, void *workspace, size_t workspace_bytes, void *stream)
 {
     GDR2_TRY(check_dims(B, T, H, dk, dv));
     GDR2_TRY(check_dtype(dt));
     GDR2_TRY(check_gates(gates));
+    const bool epilogue = out_gate || norm_weight;
+    const bool tc_shape = dt == GDR2_BF16 && dk == 128 && dv == 128;
+    if (packed && !tc_shape)
+        return fail(GDR2_ERR_UNSUPPORTED, "%s: packed sequences need bf16 inputs with dk = dv = 128", who);
+    if (epilogue && !tc_shape)
+        return fail(GDR2_ERR_UNSUPPORTED, "%s: the output norm and gate need bf16 inputs with dk = dv = 128", who);
+    if ((long long)B * H == 0) return GDR2_OK;
     const bool has_tokens = (long long)B * T * H > 0;
+    if (packed) {
+        if (!cu_seqlens) return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is NULL");
+        if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+            return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+    }
     GDR2_TRY(check_ptr(q, "q", !has_tokens));
     GDR2_TRY(check_ptr(k, "k", !has_tokens));
     GDR2_TRY(check_ptr(v, "v", !has_tokens));
@@ -146,7 +160,13 @@ gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype d
     GDR2_TRY(check_ptr(S0, "S0", true));
     GDR2_TRY(check_ptr(S_T, "S_T", true));
     GDR2_TRY(check_ptr(saved_states, "saved_states", true));
-    if ((long long)B * H == 0) return GDR2_OK;
+    GDR2_TRY(check_ptr(out_gate, "out_gate", true));
+    if (norm_weight) {
+        if ((reinterpret_cast<uintptr_t>(norm_weight) & 3u) != 0)
+            return fail(GDR2_ERR_INVALID_ARG, "norm_weight is not 4-byte aligned");
+        if (!(norm_eps >= 0.f && norm_eps <= 3.4e38f))
+            return fail(GDR2_ERR_INVALID_ARG, "norm_eps must be finite and >= 0 (got %g)", (double)norm_eps);
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0) {
         // No tokens: S_T = S0 (or zeros); nothing to save.
@@ -154,11 +174,12 @@ gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype d
             const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
             cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
                                : cudaMemsetAsync(S_T, 0, bytes, s);
-            return launched(e, "gdr2_forward (T = 0)");
+            return launched(e, who);
         }
         return GDR2_OK;
     }
-    const size_t need = gdr2_forward_workspace_bytes(B, T, H, dk, dv, dt);
+    const size_t need = packed ? gdr2_forward_varlen_workspace_bytes(B, T, H, dk, dv, dt)
+                               : gdr2_forward_workspace_bytes(B, T, H, dk, dv, dt);
     if (need > 0) {
         if (!workspace || workspace_bytes < need)
             return fail(GDR2_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes,
@@ -166,12 +187,24 @@ gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype d
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
             return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
     }
-    gdr2::FwdArgs a{B,  T,    H,  dk,  dv,           dt == GDR2_BF16, q,         k,               v,      log_alpha,
-                    b,  w,    S0, o,   S_T,          saved_states,    workspace, workspace_bytes, nullptr,
-                    nullptr, gates};
+    gdr2::FwdArgs a{B,         T,         H,       dk,       dv,     dt == GDR2_BF16,
+                    q,         k,         v,       log_alpha, b,     w,
+                    S0,        o,         S_T,     saved_states, workspace, workspace_bytes,
+                    nullptr,   packed ? cu_seqlens : nullptr, gates, out_gate, norm_weight, norm_eps};
     GDR2_TRY(device_status(&a.status));
-    if (gdr2::forward_tc_supported(a)) return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward (tcgen05)");
-    return launched(gdr2::launch_forward_simt(a, s), "gdr2_forward (simt)");
+    if (gdr2::forward_tc_supported(a)) return launched(gdr2::launch_forward_tc(a, s), who);
+    if (packed || epilogue)
+        return fail(GDR2_ERR_UNSUPPORTED, "%s: the tensor-core forward is not available on this device", who);
+    return launched(gdr2::launch_forward_simt(a, s), who);
+}
+
+gdr2_status gdr2_forward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
+                               const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                               const float *S0, void *o, float *S_T, float *saved_states, void *workspace,
+                               size_t workspace_bytes, void *stream)
+{
+    return forward_impl("gdr2_forward", B, T, H, dk, dv, dt, gates, nullptr, false, q, k, v, log_alpha, b, w, S0,
+                        nullptr, nullptr, 0.f, o, S_T, saved_states, workspace, workspace_bytes, stream);
 }
 
 gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
@@ -195,47 +228,19 @@ gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype 
                                 const void *w, const float *S0, void *o, float *S_T, float *saved_states,
                                 void *workspace, size_t workspace_bytes, void *stream)
 {
-    GDR2_TRY(check_dims(N, T, H, dk, dv));
-    GDR2_TRY(check_dtype(dt));
-    GDR2_TRY(check_gates(gates));
-    if (dt != GDR2_BF16 || dk != 128 || dv != 128)
-        return fail(GDR2_ERR_UNSUPPORTED, "packed sequences need bf16 inputs with dk = dv = 128");
-    if ((long long)N * H == 0) return GDR2_OK;
-    const bool has_tokens = (long long)T * H > 0;
-    if (!cu_seqlens) return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is NULL");
-    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
-        return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
-    GDR2_TRY(check_ptr(q, "q", !has_tokens));
-    GDR2_TRY(check_ptr(k, "k", !has_tokens));
-    GDR2_TRY(check_ptr(v, "v", !has_tokens));
-    GDR2_TRY(check_ptr(log_alpha, "log_alpha", !has_tokens));
-    GDR2_TRY(check_gate_ptr(b, "b", !has_tokens, gates & GDR2_GATE_SCALAR_B, dt));
-    GDR2_TRY(check_gate_ptr(w, "w", !has_tokens, gates & GDR2_GATE_SCALAR_W, dt));
-    GDR2_TRY(check_ptr(o, "o", !has_tokens));
-    GDR2_TRY(check_ptr(S0, "S0", true));
-    GDR2_TRY(check_ptr(S_T, "S_T", true));
-    GDR2_TRY(check_ptr(saved_states, "saved_states", true));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (T == 0) {
-        if (S_T && S_T != S0) {
-            const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
-            cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
-                               : cudaMemsetAsync(S_T, 0, bytes, s);
-            return launched(e, "gdr2_forward_varlen (T = 0)");
-        }
-        return GDR2_OK;
-    }
-    const size_t need = gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dt);
-    if (!workspace || workspace_bytes < need)
-        return fail(GDR2_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-        return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
-    gdr2::FwdArgs a{N, T, H, dk, dv, true, q, k, v, log_alpha, b, w, S0, o, S_T, saved_states, workspace,
-                    workspace_bytes, nullptr, cu_seqlens, gates};
-    GDR2_TRY(device_status(&a.status));
-    if (!gdr2::forward_tc_supported(a))
-        return fail(GDR2_ERR_UNSUPPORTED, "the tensor-core forward is not available on this device");
-    return launched(gdr2::launch_forward_tc(a, s), "gdr2_forward_varlen (tcgen05)");
+    return forward_impl("gdr2_forward_varlen", N, T, H, dk, dv, dt, gates, cu_seqlens, true, q, k, v, log_alpha, b,
+                        w, S0, nullptr, nullptr, 0.f, o, S_T, saved_states, workspace, workspace_bytes, stream);
+}
+
+gdr2_status gdr2_forward_ex(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const int *cu_seqlens,
+                            const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                            const void *w, const float *S0, const void *out_gate, const float *norm_weight,
+                            float norm_eps, void *o, float *S_T, float *saved_states, void *workspace,
+                            size_t workspace_bytes, void *stream)
+{
+    return forward_impl("gdr2_forward_ex", B, T, H, dk, dv, dt, gates, cu_seqlens, cu_seqlens != nullptr, q, k, v,
+                        log_alpha, b, w, S0, out_gate, norm_weight, norm_eps, o, S_T, saved_states, workspace,
+                        workspace_bytes, stream);
 }
 
 gdr2_status gdr2_decode_step_gated(int N, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,

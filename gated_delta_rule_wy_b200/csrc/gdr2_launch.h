@@ -22,6 +22,10 @@ struct FwdArgs {
     unsigned *status;  // device status word
     const int *cu_seqlens;  // packed sequences: B = their number, T = total tokens (null = dense)
     int gates;              // kGate* bits: b and/or w one value per token-head
+    // block epilogue on o (tensor-core path only): o / rms(o) * norm_weight (.) silu(out_gate)
+    const void *out_gate;      // bf16, the layout of o, or null
+    const float *norm_weight;  // [dv], or null for no norm
+    float norm_eps;
 };
 
 struct DecodeArgs {

@@ -110,3 +110,16 @@ def make_upstream_grad(B, T, H, dv, seed, dtype=torch.float32):
     """dO ~ N(0, 1) in the output layout [B, T, H, dv]."""
     gen = torch.Generator().manual_seed(int(seed) + 7919)
     return torch.randn((B, T, H, dv), generator=gen).to(dtype)
+
+
+def make_epilogue_inputs(o_shape, dv, dtype=torch.bfloat16, seed=0, gate_scale=1.0):
+    """Output-gate pre-activations and RMSNorm weight for the block epilogue.
+
+    g ~ gate_scale * N(0, 1) in o's layout and dtype (a linear projection of the block
+    input); weight = 1 + 0.1 N(0, 1) over the dv channels, fp32 (a learned norm weight
+    near its initial value of one).
+    """
+    gen = torch.Generator().manual_seed(int(seed) + 104729)
+    g = (torch.randn(tuple(o_shape), generator=gen) * gate_scale).to(dtype)
+    weight = 1.0 + 0.1 * torch.randn((dv,), generator=gen)
+    return g, weight

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 4
+#define GDR2_ABI_VERSION 5
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -190,6 +190,39 @@ gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype 
                                 const void *b, const void *w, const float *S0,
                                 void *o, float *S_T, float *saved_states,
                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdr2_forward_ex -- the forward with every option in one call: dense
+ * ([B, T, H, .], cu_seqlens = NULL; B = batch) or packed sequences
+ * (cu_seqlens as in gdr2_forward_varlen; B = N sequences), the gate layouts of
+ * `gates`, and the output epilogue of the Gated DeltaNet-2 block (note sec. 3,
+ * block data-flow paragraph: the mixer output goes through an RMSNorm combined
+ * with a SiLU output gate), applied to o in fp32 before its bf16 rounding:
+ *
+ *   o[t, j] <- o[t, j] / sqrt(mean_j' o[t, j']^2 + norm_eps) * norm_weight[j]
+ *              * silu(out_gate[t, j]),        silu(x) = x / (1 + exp(-x))
+ *
+ * with the mean over the dv channels of one token and head. Each factor is
+ * optional: norm_weight = NULL skips the normalisation, out_gate = NULL the
+ * gate. S_T and saved_states are the recurrence's own states, untouched by
+ * the epilogue.
+ * in:  out_gate same layout and dtype as o ([B, T, H, dv], or [T, H, dv]
+ *      packed), 16-byte aligned, or NULL; norm_weight [dv] fp32 (4-byte
+ *      aligned) or NULL; norm_eps finite and >= 0 (used only with
+ *      norm_weight; with 0, a token whose o is all zero gives NaN).
+ * scratch: gdr2_forward_workspace_bytes(...) dense,
+ *      gdr2_forward_varlen_workspace_bytes(...) packed.
+ * Supported: any case gdr2_forward_gated runs; packed sequences or an
+ * epilogue need bf16 inputs with dk = dv = 128 (GDR2_ERR_UNSUPPORTED
+ * otherwise). With cu_seqlens = NULL and no epilogue this is
+ * gdr2_forward_gated; with cu_seqlens and no epilogue, gdr2_forward_varlen.
+ */
+gdr2_status gdr2_forward_ex(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const int *cu_seqlens,
+                            const void *q, const void *k, const void *v, const float *log_alpha,
+                            const void *b, const void *w, const float *S0,
+                            const void *out_gate, const float *norm_weight, float norm_eps,
+                            void *o, float *S_T, float *saved_states,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /* Bytes of device scratch gdr2_backward needs for this problem. */
 size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt);

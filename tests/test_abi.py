@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 4
+    assert lib.gdr2_abi_version() == 5
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -156,3 +156,36 @@ def test_forward_workspace_query_and_check(lib):
     p = [ctypes.c_void_p(0x10000)] * 11  # 10 tensors + the workspace
     st = lib.gdr2_forward(1, 100, 1, 128, 128, 1, *p, ctypes.c_size_t(1024), None)
     assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
+
+
+def _ex_args(out_gate, norm_weight, eps, cu=None, ws_bytes=1 << 30):
+    p = ctypes.c_void_p(0x10000)
+    return ([cu] + [p] * 6 + [None] + [out_gate, norm_weight, ctypes.c_float(eps)] + [p, None, None, p] +
+            [ctypes.c_size_t(ws_bytes), ctypes.c_void_p(0)])
+
+
+def test_forward_ex_checks_the_epilogue_on_the_host(lib):
+    p, odd = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10008)
+    # the epilogue runs on the tensor-core path only: fp32 or d = 64 are UNSUPPORTED
+    st = lib.gdr2_forward_ex(1, 64, 2, 128, 128, 0, 0, *_ex_args(None, p, 1e-6))
+    assert st == binding.GDR2_ERR_UNSUPPORTED and b"norm" in lib.gdr2_last_error()
+    st = lib.gdr2_forward_ex(1, 64, 2, 64, 64, 1, 0, *_ex_args(p, None, 1e-6))
+    assert st == binding.GDR2_ERR_UNSUPPORTED
+    # the gate has o's layout: 16-byte aligned; the weight 4-byte aligned; eps finite, >= 0
+    st = lib.gdr2_forward_ex(1, 64, 2, 128, 128, 1, 0, *_ex_args(odd, None, 1e-6))
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"out_gate" in lib.gdr2_last_error()
+    st = lib.gdr2_forward_ex(1, 64, 2, 128, 128, 1, 0, *_ex_args(None, ctypes.c_void_p(0x10002), 1e-6))
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"norm_weight" in lib.gdr2_last_error()
+    for eps in (-1e-6, float("nan"), float("inf")):
+        st = lib.gdr2_forward_ex(1, 64, 2, 128, 128, 1, 0, *_ex_args(None, p, eps))
+        assert st == binding.GDR2_ERR_INVALID_ARG and b"norm_eps" in lib.gdr2_last_error()
+    # eps is not looked at without a norm; valid arguments stop at the workspace check here
+    st = lib.gdr2_forward_ex(1, 64, 2, 128, 128, 1, 0, *_ex_args(p, None, -1.0, ws_bytes=16))
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
+    # packed: the varlen workspace is the one asked for
+    cu = ctypes.c_void_p(0x20000)
+    need = lib.gdr2_forward_varlen_workspace_bytes(3, 64, 2, 128, 128, 1)
+    st = lib.gdr2_forward_ex(3, 64, 2, 128, 128, 1, 0, *_ex_args(p, p, 1e-6, cu=cu, ws_bytes=need - 256))
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
+    st = lib.gdr2_forward_ex(3, 64, 2, 128, 128, 0, 0, *_ex_args(None, None, 0.0, cu=cu))
+    assert st == binding.GDR2_ERR_UNSUPPORTED and b"packed" in lib.gdr2_last_error()
