@@ -997,6 +997,7 @@ constexpr uint32_t SC_EPI = SC_MISC + 1280;        // output norm: per-warp sums
 constexpr uint32_t SC_G = SC_MISC + 4096;          // output gate tile [64 t][128 j] bf16 (1024-aligned)
 static_assert(SC_EPI + 1280 <= SC_G, "norm scratch overlaps the gate tile");
 static_assert(SC_G % 1024 == 0, "gate tile alignment");
+constexpr int SC_NT = NT + 32;  // 8 warps on the TMEM lanes + warp 8, which issues the MMAs
 constexpr uint32_t SC_REG = 256;                    // region r at columns 256 r: O^T then S^T
 constexpr uint32_t SC_OT = 0, SC_ST = 64;           // offsets within a region
 constexpr uint32_t SC_SA = 448;                     // S^T in bf16, two values per column (64 columns)
@@ -1055,8 +1056,20 @@ __device__ __forceinline__ void transpose_reduce32(float (&vals)[N], int lane)
     }
 }
 
+// 1 / d for 1 <= d < 2^126. Seed: the bit pattern of a float is close to 2^23 (log2 d + 127),
+// so subtracting it from a constant negates log2 d: one integer operation gives 1 / d to
+// within 5.1% in every binade (the constant minimises that error over one binade). Two
+// Newton steps r <- r + r (1 - d r), each squaring the relative error, leave 6.6e-6.
+// All of it on the FMA and integer pipes: the special-function unit is the scarce one.
+__device__ __forceinline__ float recip_newton2(float d)
+{
+    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
+    r = fmaf(r, fmaf(-d, r, 1.f), r);
+    return fmaf(r, fmaf(-d, r, 1.f), r);
+}
+
 template <int EPI>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(SC_NT, 1)  // 168 registers: allocation rounds 9 warps up to 12
 fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g, ScanParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -1124,7 +1137,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
     uint32_t ph_g = 0;
     bool g_failed = false;  // a gate tile that never arrived: stop waiting for the later ones
     // initial state S^T[j][c] = S0[c][j] into region 1 (chunk 0 reads the region of "chunk -1")
-    {
+    if (warp < 8) {
         float v[32];
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
@@ -1150,56 +1163,48 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
     };
 
     // O^T of chunk m -> (epilogue) -> bf16 tile [t][j] -> one TMA store (rows past T are
-    // clipped). Warps 0-3 only (thread = TMEM lane = value channel j, all 64 tokens), under
-    // named barrier 1, so they run while the MMA issuer in warp 4 is busy with the next
-    // chunk (spreading this over all 8 warps measured slower: the extra TMEM traffic
-    // stretches the chunk's MMAs).
+    // clipped). Warps 0-7 under named barrier 1, while warp 8 keeps the tensor core busy with
+    // the next chunk: warp quarter q reads TMEM lanes (value channels) j = 32 q + lane, warp
+    // group colhalf the tokens t = 32 colhalf .. 32 colhalf + 31.
     auto store_o = [&](int m) {
         if (tid == 0) bulk_wait_group_read0();  // the previous tile has left shared memory
-        named_barrier(1, 128);
-        float o0[32], o1[32];
-        const uint32_t ot_col = SC_REG * (m & 1) + SC_OT;
-        tmem_ld32x2(tm_lane + ot_col, tm_lane + ot_col + 32, o0, o1);
+        named_barrier(1, 256);
+        const int t0 = colhalf * 32;
+        float o0[32];
+        tmem_ld32(tm_lane + SC_REG * (m & 1) + SC_OT + t0, o0);
         if constexpr ((EPI & kEpiNorm) != 0) {
-            // RMSNorm over the value channels of each token: this thread holds channel j of all
-            // 64 tokens; sums of squares over a warp's 32 channels, then over the 4 warps
+            // RMSNorm over the value channels of each token: sums of squares over a warp's
+            // 32 channels (lane L ends with token t0 + L), then over the 4 warp quarters
             float *red = reinterpret_cast<float *>(sm + SC_EPI);  // [4][64], then 1/rms at [256 ..)
-            float sq[64];
+            float sq[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                sq[i] = o0[i] * o0[i];
-                sq[32 + i] = o1[i] * o1[i];
-            }
-            transpose_reduce32<64>(sq, lane);  // lane L: tokens 2L and 2L + 1
-            red[quarter * 64 + 2 * lane] = sq[0];
-            red[quarter * 64 + 2 * lane + 1] = sq[1];
-            named_barrier(1, 128);
+            for (int i = 0; i < 32; ++i) sq[i] = o0[i] * o0[i];
+            transpose_reduce32<32>(sq, lane);
+            red[quarter * 64 + t0 + lane] = sq[0];
+            named_barrier(1, 256);
             if (tid < 64)
                 red[256 + tid] = rsqrtf((red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid]) * (1.f / DV) +
                                         p.norm_eps);
-            named_barrier(1, 128);
+            named_barrier(1, 256);
             const float wj = p.norm_weight[j];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                o0[i] *= red[256 + i] * wj;
-                o1[i] *= red[256 + 32 + i] * wj;
-            }
+            for (int i = 0; i < 32; ++i) o0[i] *= red[256 + t0 + i] * wj;
         }
         if constexpr ((EPI & kEpiGate) != 0) {
             if (tid == 0) {
                 ms.g_ok = (!g_failed && mbar_wait_bounded(&ms.bar_g, ph_g, kWaitLimitNs)) ? 1 : 0;
                 if (ms.g_ok) g_inflight = false;
             }
-            named_barrier(1, 128);
+            named_barrier(1, 256);
             ph_g ^= 1u;
             if (ms.g_ok) {
-                const __nv_bfloat16 *gt = reinterpret_cast<const __nv_bfloat16 *>(sm + SC_G) + j;
+                const __nv_bfloat16 *gt = reinterpret_cast<const __nv_bfloat16 *>(sm + SC_G) + t0 * DV + j;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    // silu(g) = g / (1 + exp(-g)); a huge denominator (g below about -87) gives 0
-                    const float g0 = __bfloat162float(gt[i * DV]), g1 = __bfloat162float(gt[(32 + i) * DV]);
-                    o0[i] *= __fdividef(g0, 1.f + __expf(-g0));
-                    o1[i] *= __fdividef(g1, 1.f + __expf(-g1));
+                    // silu(g) = g / (1 + exp(-g)), exp argument kept below 80 so 1 + exp stays
+                    // finite (for g < -80, silu(g) is below 2e-33 in magnitude either way)
+                    const float g = __bfloat162float(gt[i * DV]);
+                    o0[i] *= g * recip_newton2(1.f + __expf(-fmaxf(g, -80.f)));
                 }
             } else {
                 g_failed = true;
@@ -1208,20 +1213,17 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         }
         __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            ot[i * DV + j] = __float2bfloat16_rn(o0[i]);
-            ot[(32 + i) * DV + j] = __float2bfloat16_rn(o1[i]);
-        }
+        for (int i = 0; i < 32; ++i) ot[(t0 + i) * DV + j] = __float2bfloat16_rn(o0[i]);
         fence_proxy_async_smem();
         tc_fence_before_sync();
-        named_barrier(1, 128);
+        named_barrier(1, 256);
         // every read of this chunk's gate tile is done: the next one may land
         if ((EPI & kEpiGate) && !g_failed && tid == 0 && m + 1 < NC) issue_gate(m + 1);
         const int rows = min(C, len - m * C);
         if (p.cu_seqlens && rows < C) {
             // a packed sequence's partial last tile: its rows only (a tile store would write
             // into the next sequence)
-            for (int i = tid; i < rows * 16; i += 128) {
+            for (int i = tid; i < rows * 16; i += 256) {
                 const int r = i >> 4, c16 = i & 15;
                 *reinterpret_cast<uint4 *>(p.o + ((size_t)(tstart + m * C + r) * p.H + h) * DV + c16 * 8) =
                     *reinterpret_cast<const uint4 *>(ot + r * DV + c16 * 8);
@@ -1238,7 +1240,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         const uint32_t slot = sbase + (sl ? SC_SLOT1 : SC_SLOT0);
         const uint32_t rg = SC_REG * (uint32_t)sl, rg_prev = SC_REG * (uint32_t)(sl ^ 1);
         // ---- S^T (previous region) -> bf16 operand; gamma-scaled S^T -> this region ----
-        {
+        if (warp < 8) {
             float s0[32], s1[32];
             tmem_ld32x2(tm_lane + rg_prev + SC_ST + c0, tm_lane + rg_prev + SC_ST + c0 + 32, s0, s1);
             if (p.saved_states) {
@@ -1273,7 +1275,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         __syncthreads();
         tc_fence_after_sync();
         // ---- [O^T | S^T] += S_bf16^T [Q'; M]^T ;  S^T += U~^T K~ ;  O^T += U~^T P^T ----
-        if (tid == 128) {
+        if (warp == 8 && lane == 0) {
             const uint32_t id1 = idesc_bf16(128, B1_ROWS, false, false);
             const uint32_t idS = idesc_bf16(128, 128, false, true);
             const uint32_t idO = idesc_bf16(128, 64, false, false);
@@ -1293,15 +1295,14 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
             }
             mma_commit(&ms.bar_mma);
         }
-        if (warp < 4) {
+        if (warp < 8) {
             // overlaps this chunk's MMAs (the other region), then clears that region's O^T
-            // for chunk n + 1 (each thread rewrites only the lane it has just read)
+            // for chunk n + 1 (each thread rewrites only the lane and columns it has just read)
             if (n > 0) store_o(n - 1);
             float zz[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) zz[i] = 0.f;
-            tmem_st32_nw(tm_lane + rg_prev + SC_OT, zz);
-            tmem_st32_nw(tm_lane + rg_prev + SC_OT + 32, zz);
+            tmem_st32_nw(tm_lane + rg_prev + SC_OT + colhalf * 32, zz);
             tmem_wait_st();
         }
         // the next slot (issued two chunks ago) and this chunk's MMAs, one barrier for both
@@ -1319,8 +1320,8 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         }
         if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
     }
-    if (!timed_out && NC > 0 && warp < 4) store_o(NC - 1);
-    if (!timed_out && p.S_T) {
+    if (!timed_out && NC > 0 && warp < 8) store_o(NC - 1);
+    if (!timed_out && p.S_T && warp < 8) {
         const uint32_t rg_last = SC_REG * (uint32_t)((NC + 1) & 1);  // region of chunk NC - 1 (region 1 if NC = 0)
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
@@ -1455,7 +1456,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
                   static_cast<__nv_bfloat16 *>(a.o), a.norm_weight, a.norm_eps};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.H);
-    cfg.blockDim = dim3(NT);
+    cfg.blockDim = dim3(SC_NT);
     cfg.dynamicSmemBytes = scan_smem_bytes(epi);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
