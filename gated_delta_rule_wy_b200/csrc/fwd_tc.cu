@@ -187,6 +187,18 @@ struct ChunkLoc {
     int h, t0, bb, Cn;
 };
 
+// 1 / d for 2^-126 <= d < 2^126 (normal, positive). Seed: the bit pattern of a float is close to 2^23 (log2 d + 127),
+// so subtracting it from a constant negates log2 d: one integer operation gives 1 / d to
+// within 5.1% in every binade (the constant minimises that error over one binade). Two
+// Newton steps r <- r + r (1 - d r), each squaring the relative error, leave 6.6e-6.
+// All of it on the FMA and integer pipes: the special-function unit is the scarce one.
+__device__ __forceinline__ float recip_newton2(float d)
+{
+    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
+    r = fmaf(r, fmaf(-d, r, 1.f), r);
+    return fmaf(r, fmaf(-d, r, 1.f), r);
+}
+
 template <bool GENERAL>
 __device__ __forceinline__ ChunkLoc locate_chunk(const ChunkParams &p, int task)
 {
@@ -477,7 +489,9 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int x = 0; x < 8; ++x) {
                     const float d = G[m][x] - gr[x];
                     risky |= fabsf(d) > kFactorLimit;
-                    const float xl = __expf(d), yr = __expf(-d);
+                    // |d| <= 70 here (or the exact path replaces these): exp(-d) as the
+                    // reciprocal of exp(d), off the special-function unit
+                    const float xl = __expf(d), yr = recip_newton2(xl);
                     le[x] = bv[x] * kv[x] * xl;
                     lq[x] = qv[x] * xl;
                     r[x] = kv[x] * yr;
@@ -1054,18 +1068,6 @@ __device__ __forceinline__ void transpose_reduce32(float (&vals)[N], int lane)
             vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
         }
     }
-}
-
-// 1 / d for 1 <= d < 2^126. Seed: the bit pattern of a float is close to 2^23 (log2 d + 127),
-// so subtracting it from a constant negates log2 d: one integer operation gives 1 / d to
-// within 5.1% in every binade (the constant minimises that error over one binade). Two
-// Newton steps r <- r + r (1 - d r), each squaring the relative error, leave 6.6e-6.
-// All of it on the FMA and integer pipes: the special-function unit is the scarce one.
-__device__ __forceinline__ float recip_newton2(float d)
-{
-    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
-    r = fmaf(r, fmaf(-d, r, 1.f), r);
-    return fmaf(r, fmaf(-d, r, 1.f), r);
 }
 
 template <int EPI>
