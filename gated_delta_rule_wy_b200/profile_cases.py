@@ -1,6 +1,6 @@
 """Run one libgdr2.so kernel on its benchmark workload, for profilers.
 
-    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd} [--launches N] [--batch B]
+    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd} [--launches N] [--batch B] [--epilogue]
 
 fwd     gdr2_forward   B=4 H=16 T=4096 d=128 bf16 (the 1.3B-model layer)
 decode  gdr2_decode_step  256 sequences x 16 heads, d=128, fp32 state (256 MiB)
@@ -9,7 +9,8 @@ bwd     gdr2_backward  B=2 H=16 T=4096 d=128 bf16 with saved chunk states
 Inputs are drawn once (seeded) and stay on the device; the kernel is then
 launched N times back to back (use ncu -s/-c to pick one launch). --batch
 overrides B of the forward and backward cases (a smaller capture whose inputs
-still exceed the 126 MB L2 at B >= 2).
+still exceed the 126 MB L2 at B >= 2). --epilogue runs the forward with the block's
+output epilogue (RMSNorm weight and SiLU gate, seeded like the bench's).
 """
 from __future__ import annotations
 
@@ -26,6 +27,7 @@ def main():
     ap.add_argument("kernel", choices=("fwd", "decode", "bwd"))
     ap.add_argument("--launches", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--epilogue", action="store_true")
     args = ap.parse_args()
     torch.cuda.set_device(0)
     if args.kernel == "fwd":
@@ -36,8 +38,13 @@ def main():
         o = torch.empty_like(x.v)
         ws = torch.empty(gdr2_forward_workspace_bytes(c["B"], c["T"], c["H"], c["dk"], c["dv"], c["dtype"]),
                          dtype=torch.uint8, device="cuda")
+        g = wt = None
+        if args.epilogue:
+            g, wt = I.make_epilogue_inputs((c["B"], c["T"], c["H"], c["dv"]), c["dv"], seed=1009)
+            g, wt = g.to("cuda"), wt.to("cuda")
         for _ in range(args.launches):
-            gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o, workspace=ws)
+            gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, out=o, workspace=ws, out_gate=g,
+                         norm_weight=wt)
     elif args.kernel == "decode":
         c = I.DECODE_1P3B
         gen = torch.Generator(device="cuda").manual_seed(c["seed"])
