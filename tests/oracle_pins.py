@@ -384,6 +384,88 @@ def pin_output_norm_gate(orc=None, seed=14, OB=None):
     assert np.array_equal(OB.output_norm_gate(o), o)
 
 
+# ---------------------------------------------------------------------------
+# P13  Block prologue (GDN2 sec. 3, block data flow): the causal depthwise convolution
+#      against numpy's convolution, its state and causality, packed sequences, the L2
+#      norm per head, the decay and gate activations against their direct formulas
+# ---------------------------------------------------------------------------
+def pin_block_prologue(orc=None, seed=15, OB=None):
+    if OB is None:
+        from oracle import block as OB
+
+    rng = np.random.default_rng(seed)
+    W, T, C = 4, 11, 5
+    x = rng.standard_normal((1, T, C))
+    wgt = rng.standard_normal((C, W))
+    st = rng.standard_normal((1, W - 1, C))
+    # the convolution is numpy's ("valid" over [state; x], taps reversed: tap W-1 on the current token)
+    for state in (None, st):
+        y = OB.causal_conv(x, wgt, state)
+        pad = np.zeros((W - 1, C)) if state is None else state[0]
+        z = np.concatenate([pad, x[0]], axis=0)
+        for c in range(C):
+            _close(y[0, :, c], np.convolve(z[:, c], wgt[c, ::-1], mode="valid"), 1e-13, "conv vs numpy")
+    # delta taps: the identity and a one-token delay
+    delta = np.zeros((C, W))
+    delta[:, W - 1] = 1.0
+    _close(OB.causal_conv(x, delta, st), x, 0, "delta taps")
+    delay = np.zeros((C, W))
+    delay[:, W - 2] = 1.0
+    _close(OB.causal_conv(x, delay, st), np.concatenate([st[:, -1:], x[:, :-1]], axis=1), 0, "one-token delay")
+    # conv then SiLU: with delta taps the prologue of v is silu(x)
+    yv, _ = OB.short_conv_silu(x, delta, st)
+    _close(yv, OB.silu(x), 1e-15, "delta taps then silu")
+    # causality and reach: a change at t0 moves outputs t0 .. t0 + W - 1 only
+    x2 = x.copy()
+    x2[0, 4] += 1.0
+    dy = np.abs(OB.causal_conv(x2, wgt, st) - OB.causal_conv(x, wgt, st))[0].max(axis=1)
+    assert np.all(dy[:4] == 0) and np.all(dy[4 + W:] == 0) and np.all(dy[4:4 + W] > 0), "causality"
+    # continuing from the state: one call over [x1; x2] equals two calls, also when the second
+    # part is shorter than the state
+    for cut in (6, T - 2):
+        y_all, s_all = OB.short_conv_silu(x, wgt, st)
+        y1, s1 = OB.short_conv_silu(x[:, :cut], wgt, st)
+        y2, s2 = OB.short_conv_silu(x[:, cut:], wgt, s1)
+        _close(np.concatenate([y1, y2], axis=1), y_all, 1e-14, "split outputs")
+        _close(s2, s_all, 0, "split state")
+    _close(s_all[0], np.concatenate([st[0], x[0]])[-(W - 1):], 0, "state = last W - 1 inputs")
+    # packed sequences convolve on their own, each from its own state (empty ones keep it)
+    lens = [3, 0, 1, 7]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    xs = rng.standard_normal((1, int(cu[-1]), C))
+    sts = rng.standard_normal((len(lens), W - 1, C))
+    yp, sp = OB.short_conv_silu(xs, wgt, cu_seqlens=cu, states=sts)
+    for i in range(len(lens)):
+        yi, si = OB.short_conv_silu(xs[:, cu[i]:cu[i + 1]], wgt, sts[i][None])
+        if lens[i]:
+            _close(yp[:, cu[i]:cu[i + 1]], yi, 0, f"packed seq {i}")
+        _close(sp[i], si[0], 0, f"packed state {i}")
+    _close(sp[1], sts[1], 0, "empty sequence keeps its state")
+    # L2 norm per head: |y| = sqrt(s / (s + eps)); scale invariance at eps = 0; heads apart
+    v = rng.standard_normal((6, 8))
+    v[0] *= 1e-4  # a row whose squared norm is comparable to eps
+    for eps in (0.0, 1e-6):
+        s = np.sum(v * v, axis=-1)
+        _close(np.linalg.norm(OB.l2_normalize(v, eps), axis=-1), np.sqrt(s / (s + eps)), 1e-13, "l2 norms")
+    _close(OB.l2_normalize(3.7 * v, 0.0), OB.l2_normalize(v, 0.0), 1e-14, "l2 scale invariance")
+    xh = rng.standard_normal((1, T, 2 * C))
+    wh = rng.standard_normal((2 * C, W))
+    yh, _ = OB.short_conv_silu(xh, wh, l2norm=True, eps=0.0, heads=2)
+    _close(np.linalg.norm(yh.reshape(1, T, 2, C), axis=-1), np.ones((1, T, 2)), 1e-13, "unit norm per head")
+    xh2 = xh.copy()
+    xh2[..., C:] *= 5.0  # head 1's input only
+    yh2, _ = OB.short_conv_silu(xh2, wh, l2norm=True, eps=0.0, heads=2)
+    _close(yh2[..., :C], yh[..., :C], 0, "head 0 independent of head 1")
+    # activations against their direct formulas
+    a = rng.standard_normal(40) * 4
+    _close(np.exp(OB.neg_softplus(a)), 1.0 / (1.0 + np.exp(a)), 1e-14, "alpha = 1 / (1 + e^a)")
+    _close(np.exp(OB.neg_softplus(a)) + OB.sigmoid(a), np.ones_like(a), 1e-14, "alpha + sigmoid(a) = 1")
+    _close(OB.sigmoid(a), 1.0 / (1.0 + np.exp(-a)), 1e-14, "sigmoid")
+    assert abs(OB.neg_softplus(40.0) + 40.0) < 1e-15 and abs(OB.neg_softplus(-40.0) + np.exp(-40.0)) < 1e-30
+    assert OB.sigmoid(0.0) == 0.5
+
+
 ALL_PINS = [pin_kda, pin_gated_deltanet, pin_deltanet, pin_full_reset, pin_no_erase_closed_form,
             pin_one_hot_slots, pin_objective_stationarity, pin_exact_write, pin_dense_product,
-            pin_split_and_linearity, pin_backward_fd, pin_backward_fd_t32_d16, pin_output_norm_gate]
+            pin_split_and_linearity, pin_backward_fd, pin_backward_fd_t32_d16, pin_output_norm_gate,
+            pin_block_prologue]

@@ -95,3 +95,39 @@ def test_block_mutant_is_caught(tmp_path, name, old, new):
     spec.loader.exec_module(mod)
     with pytest.raises(AssertionError):
         P.pin_output_norm_gate(OB=mod)
+
+
+PROLOGUE_MUTANTS = [
+    ("taps reversed", "y += wgt[:, i] * xp[..., i:i + T, :]", "y += wgt[:, W - 1 - i] * xp[..., i:i + T, :]"),
+    ("state read newest first",
+     "pad = np.zeros(lead + (W - 1, x.shape[-1])) if state is None else np.asarray(state, dtype=np.float64)",
+     "pad = np.zeros(lead + (W - 1, x.shape[-1])) if state is None else np.asarray(state, dtype=np.float64)[..., ::-1, :]"),
+    ("SiLU dropped", "        y = silu(causal_conv(x, weight, state))", "        y = causal_conv(x, weight, state)"),
+    ("L2 epsilon outside the root", "x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)",
+     "x / (np.sqrt(np.sum(x * x, axis=-1, keepdims=True)) + eps)"),
+    ("L2 over all heads together", "y.reshape(sh[:-1] + (heads, sh[-1] // heads))", "y.reshape(sh[:-1] + (1, sh[-1]))"),
+    ("softplus of the wrong sign", "-(np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x))))",
+     "-(np.maximum(-x, 0.0) + np.log1p(np.exp(-np.abs(x))))"),
+    ("convolution runs across packed sequences", "y[:, s:e] = silu(causal_conv(x[:, s:e], weight, si))",
+     "y[:, s:e] = silu(causal_conv(x, weight, None)[:, s:e])"),
+    ("state after a short call ignores the old state",
+     "    return np.concatenate([pad, x], axis=-2)[..., x.shape[-2]:, :]",
+     "    return np.concatenate([np.zeros_like(pad), x], axis=-2)[..., x.shape[-2]:, :]"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", PROLOGUE_MUTANTS, ids=[m[0] for m in PROLOGUE_MUTANTS])
+def test_prologue_mutant_is_caught(tmp_path, name, old, new):
+    import importlib.util
+
+    import oracle_pins as P
+
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "block.py")).read()
+    assert src.count(old) == 1, f"mutation site not found: {old}"
+    mpath = tmp_path / "block_mutant.py"
+    mpath.write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location("block_mutant", mpath)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with pytest.raises(AssertionError):
+        P.pin_block_prologue(OB=mod)
