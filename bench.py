@@ -382,6 +382,29 @@ def bench_components(dev, stream, peaks):
                        "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3),
                        "algorithmic_bytes": alg, "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del xs, o, ws, g, wt
+    # the block prologue in front of that forward: short convolutions + SiLU (+ L2) and the
+    # decay and gate activations, from the projections' outputs
+    from gated_delta_rule_wy_b200 import gdr2_block_prologue
+    pin = {k: v.to(dev) for k, v in I.make_prologue_inputs(c["B"], c["T"], c["H"], c["dk"], c["dv"], 4, c["dtype"],
+                                                             seed=1010).items()}
+
+    def prologue():
+        gdr2_block_prologue(pin["xq"], pin["xk"], pin["xv"], pin["conv_q"], pin["conv_k"], pin["conv_v"], pin["a"],
+                            pin["b"], pin["w"])
+
+    for _ in range(3):
+        prologue()
+    ms = statistics.median(time_steps(prologue, 20, stream))
+    gdr2_sync_status()
+    th = tokens * c["H"]
+    # per token-head: q, k, v read and written in bf16; a read in bf16, log alpha written in fp32;
+    # b and w read and written in bf16 (3328 B at d = 128)
+    alg = th * (2 * (2 * c["dk"] + c["dv"]) * 2 + c["dk"] * (2 + 4) + 4 * (c["dk"] + c["dv"]))
+    out["prologue"] = {"workload": "B=4 H=16 T=4096 d=128 bf16: q, k = L2(SiLU(conv4(x))), v = SiLU(conv4(x)), "
+                                   "log alpha = -softplus(a), b, w = sigmoid",
+                       "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3), "algorithmic_bytes": alg,
+                       "hbm_frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del pin
     return out
 
 
@@ -452,7 +475,7 @@ def run_ours(args, world, rank, local):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": alg_bytes,
-                "kernel": "one gdr2_forward call: fwd_chunk_kernel (73% of its device time) + fwd_scan_kernel"}
+                "kernel": "one gdr2_forward call: fwd_chunk_kernel (74% of its device time) + fwd_scan_kernel"}
     tflops = alg_flop / t_launch / 1e12
     tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
               "frac": tflops / peaks["bf16_tflops"], "algorithmic_flop_per_launch": alg_flop,

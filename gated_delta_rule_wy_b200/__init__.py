@@ -7,11 +7,13 @@ package does not load the CUDA library; the first call does, and fails loudly
 if it is missing.
 """
 from .binding import (GDR2Error, gdr2_abi_version, gdr2_backward, gdr2_backward_noalloc,  # noqa: F401
-                      gdr2_backward_workspace_bytes, gdr2_decode_step, gdr2_forward, gdr2_forward_varlen,
-                      gdr2_forward_varlen_workspace_bytes, gdr2_forward_workspace_bytes, gdr2_last_error,
-                      gdr2_sync_status, load_library)
+                      gdr2_backward_workspace_bytes, gdr2_block_prologue, gdr2_decode_step, gdr2_forward,
+                      gdr2_forward_varlen, gdr2_forward_varlen_workspace_bytes, gdr2_forward_workspace_bytes,
+                      gdr2_gate_activations, gdr2_last_error, gdr2_short_conv_silu, gdr2_sync_status,
+                      load_library)
 
 __all__ = ["GDR2Error", "gdr2_abi_version", "gdr2_backward", "gdr2_backward_noalloc",
            "gdr2_backward_workspace_bytes", "gdr2_forward_workspace_bytes",
            "gdr2_decode_step", "gdr2_forward", "gdr2_forward_varlen", "gdr2_forward_varlen_workspace_bytes",
-           "gdr2_last_error", "gdr2_sync_status", "load_library"]
+           "gdr2_last_error", "gdr2_sync_status", "load_library", "gdr2_block_prologue", "gdr2_gate_activations",
+           "gdr2_short_conv_silu"]

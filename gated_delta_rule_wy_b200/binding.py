@@ -25,7 +25,7 @@ _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIM
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
 EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspace_bytes", "gdr2_forward",
                     "gdr2_forward_gated", "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen",
-                    "gdr2_forward_ex",
+                    "gdr2_forward_ex", "gdr2_short_conv_silu", "gdr2_gate_activations",
                     "gdr2_decode_step", "gdr2_decode_step_gated",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
                     "gdr2_sync_status")
@@ -69,6 +69,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_forward_varlen.argtypes = [I, I, I, I, I, I, I] + [P] * 12 + [Z, P]
         lib.gdr2_forward_ex.restype = I
         lib.gdr2_forward_ex.argtypes = [I, I, I, I, I, I, I] + [P] * 8 + [P, P, ctypes.c_float] + [P] * 4 + [Z, P]
+        lib.gdr2_short_conv_silu.restype = I
+        lib.gdr2_short_conv_silu.argtypes = [I] * 7 + [ctypes.c_float] + [P] * 7
+        lib.gdr2_gate_activations.restype = I
+        lib.gdr2_gate_activations.argtypes = [I] + [ctypes.c_longlong, P, P] * 3 + [P]
         lib.gdr2_forward_gated.restype = I
         lib.gdr2_forward_gated.argtypes = [I, I, I, I, I, I, I] + [P] * 11 + [Z, P]
         lib.gdr2_decode_step_gated.restype = I
@@ -267,6 +271,83 @@ def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_
                                      _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream(stream))
     _raise(lib, st)
     return o, S_T, saved
+
+
+def _check_cu_seqlens(cu_seqlens, device):
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous() \
+            or cu_seqlens.device != device:
+        raise ValueError("cu_seqlens must be a contiguous 1-D int32 tensor on the inputs' device")
+
+
+def gdr2_short_conv_silu(x, weight, state=None, *, l2norm=False, eps=1e-6, cu_seqlens=None, final_state=False,
+                         state_out=None, out=None, stream=None):
+    """Block prologue of one branch: SiLU(causal depthwise convolution of x), then with
+    l2norm the per-head L2 norm (query and key); without it, the value branch.
+
+    x: [N, T, H, d] (dense) or [T, H, d] with cu_seqlens ([N + 1] int32); weight: [H * d, W]
+    fp32 (a depthwise Conv1d weight [H * d, 1, W] too; the last tap is the current token);
+    state: [N, W - 1, H, d] in x's dtype, the inputs before each sequence, or None (zeros).
+    Returns (y, state_out): the state after the call when final_state or when a state_out
+    tensor is given (state_out=state updates a decode step's state in place, T = 1), else None.
+    """
+    lib = load_library()
+    if cu_seqlens is not None:
+        T, H, d = x.shape
+        _check_cu_seqlens(cu_seqlens, x.device)
+        N = cu_seqlens.numel() - 1
+    else:
+        N, T, H, d = x.shape
+    wgt = weight.reshape(weight.shape[0], weight.shape[-1]) if weight.dim() == 3 else weight
+    W = int(wgt.shape[-1])
+    dt = x.dtype
+    _check(x, "x", tuple(x.shape), dt)
+    _check(wgt, "weight", (H * d, W), torch.float32)
+    _check(state, "state", (N, W - 1, H, d), dt)
+    y = out if out is not None else torch.empty_like(x)
+    _check(y, "out", tuple(x.shape), dt)
+    if state_out is None and final_state:
+        state_out = torch.empty((N, W - 1, H, d), dtype=dt, device=x.device)
+    _check(state_out, "state_out", (N, W - 1, H, d), dt)
+    ptr = lambda t: None if t is None or t.numel() == 0 else _ptr(t)  # noqa: E731
+    st = lib.gdr2_short_conv_silu(N, T, H, d, _dt(x), W, int(bool(l2norm)), ctypes.c_float(eps), _ptr(cu_seqlens),
+                                  ptr(x), ptr(wgt), ptr(state), ptr(state_out), ptr(y), _stream(stream))
+    _raise(lib, st)
+    return y, state_out
+
+
+def gdr2_gate_activations(a=None, b=None, w=None, *, stream=None):
+    """The decay and gate branches' activations, element by element, any of them None:
+    log_alpha = -softplus(a) (fp32), sigmoid(b) and sigmoid(w) in the inputs' dtype."""
+    lib = load_library()
+    given = [t for t in (a, b, w) if t is not None]
+    if not given:
+        return None, None, None
+    dt = given[0].dtype
+    for name, t in (("a", a), ("b", b), ("w", w)):
+        if t is not None:
+            _check(t, name, tuple(t.shape), dt)
+    la = None if a is None else torch.empty(tuple(a.shape), dtype=torch.float32, device=a.device)
+    bo = None if b is None else torch.empty_like(b)
+    wo = None if w is None else torch.empty_like(w)
+    n = lambda t: 0 if t is None else t.numel()  # noqa: E731
+    st = lib.gdr2_gate_activations(_dt(given[0]), n(a), _ptr(a), _ptr(la), n(b), _ptr(b), _ptr(bo), n(w), _ptr(w),
+                                   _ptr(wo), _stream(stream))
+    _raise(lib, st)
+    return la, bo, wo
+
+
+def gdr2_block_prologue(xq, xk, xv, conv_q, conv_k, conv_v, a, b, w, *, states=None, eps=1e-6, cu_seqlens=None,
+                        final_state=False, stream=None):
+    """The whole prologue: q, k = L2(SiLU(conv(x))) per head, v = SiLU(conv(x)), and the
+    activations of a, b, w. states: (state_q, state_k, state_v) or None. Returns
+    (q, k, v, log_alpha, b, w, new_states); new_states is a triple when final_state, else None."""
+    sq, sk, sv = states if states is not None else (None, None, None)
+    kw = dict(eps=eps, cu_seqlens=cu_seqlens, final_state=final_state, stream=stream)
+    q, nq = gdr2_short_conv_silu(xq, conv_q, sq, l2norm=True, **kw)
+    k, nk = gdr2_short_conv_silu(xk, conv_k, sk, l2norm=True, **kw)
+    v, nv = gdr2_short_conv_silu(xv, conv_v, sv, l2norm=False, **kw)
+    la, bo, wo = gdr2_gate_activations(a, b, w, stream=stream)
+    return q, k, v, la, bo, wo, ((nq, nk, nv) if final_state else None)
 
 
 def gdr2_decode_step(q, k, v, log_alpha, b, w, S, *, out=None, stream=None):

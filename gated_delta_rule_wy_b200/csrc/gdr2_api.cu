@@ -243,6 +243,73 @@ gdr2_status gdr2_forward_ex(int B, int T, int H, int dk, int dv, gdr2_dtype dt, 
                         workspace_bytes, stream);
 }
 
+gdr2_status gdr2_short_conv_silu(int N, int T, int H, int d, gdr2_dtype dt, int width, int l2norm, float l2_eps,
+                                 const int *cu_seqlens, const void *x, const float *weight, const void *state_in,
+                                 void *state_out, void *y, void *stream)
+{
+    GDR2_TRY(check_dtype(dt));
+    if (N < 0 || T < 0 || H < 0) return fail(GDR2_ERR_INVALID_ARG, "negative size (N=%d T=%d H=%d)", N, T, H);
+    if (d != 64 && d != 128) return fail(GDR2_ERR_UNSUPPORTED, "d must be 64 or 128 (d=%d)", d);
+    if (width < 1 || width > 4) return fail(GDR2_ERR_UNSUPPORTED, "width must be 1 .. 4 (width=%d)", width);
+    if (l2norm != 0 && l2norm != 1) return fail(GDR2_ERR_INVALID_ARG, "l2norm must be 0 or 1");
+    if (!(l2_eps >= 0.f && l2_eps <= 3.4e38f))
+        return fail(GDR2_ERR_INVALID_ARG, "l2_eps must be finite and >= 0 (got %g)", (double)l2_eps);
+    const long long rows = cu_seqlens ? (long long)T : (long long)N * T;
+    if (rows * H * d > (1ll << 40)) return fail(GDR2_ERR_INVALID_ARG, "problem too large");
+    if ((long long)N * H == 0) return GDR2_OK;
+    const bool has_tokens = rows * H > 0;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+        return fail(GDR2_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+    GDR2_TRY(check_ptr(x, "x", !has_tokens));
+    GDR2_TRY(check_ptr(y, "y", !has_tokens));
+    if (has_tokens && x == y) return fail(GDR2_ERR_INVALID_ARG, "y must not be x");
+    if (!weight && has_tokens) return fail(GDR2_ERR_INVALID_ARG, "weight is NULL");
+    if ((reinterpret_cast<uintptr_t>(weight) & 3u) != 0)
+        return fail(GDR2_ERR_INVALID_ARG, "weight is not 4-byte aligned");
+    GDR2_TRY(check_ptr(state_in, "state_in", true));
+    GDR2_TRY(check_ptr(state_out, "state_out", true));
+    if (state_in && state_in == state_out && (cu_seqlens || T != 1))
+        return fail(GDR2_ERR_INVALID_ARG, "state_out may be state_in only for T = 1 without cu_seqlens");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!has_tokens && !cu_seqlens) {
+        // no tokens: the state passes through
+        if (state_out && width > 1 && state_out != state_in) {
+            const size_t bytes = (size_t)N * (width - 1) * H * d * (dt == GDR2_BF16 ? 2 : 4);
+            cudaError_t e = state_in ? cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, s)
+                                     : cudaMemsetAsync(state_out, 0, bytes, s);
+            return launched(e, "gdr2_short_conv_silu (T = 0)");
+        }
+        return GDR2_OK;
+    }
+    gdr2::ConvArgs a{N, T, H, d, width, dt == GDR2_BF16, l2norm != 0, l2_eps, cu_seqlens, x, weight,
+                     width > 1 ? state_in : nullptr, width > 1 ? state_out : nullptr, y};
+    return launched(gdr2::launch_short_conv(a, s), "gdr2_short_conv_silu");
+}
+
+gdr2_status gdr2_gate_activations(gdr2_dtype dt, long long n_alpha, const void *a, float *log_alpha, long long n_b,
+                                  const void *b_pre, void *b, long long n_w, const void *w_pre, void *w,
+                                  void *stream)
+{
+    GDR2_TRY(check_dtype(dt));
+    if (n_alpha < 0 || n_b < 0 || n_w < 0) return fail(GDR2_ERR_INVALID_ARG, "negative element count");
+    const void *ins[3] = {a, b_pre, w_pre};
+    const void *outs[3] = {log_alpha, b, w};
+    const long long ns[3] = {n_alpha, n_b, n_w};
+    const char *names[3] = {"a / log_alpha", "b_pre / b", "w_pre / w"};
+    for (int k = 0; k < 3; ++k) {
+        if (ns[k] == 0) continue;
+        if (!ins[k] != !outs[k]) return fail(GDR2_ERR_INVALID_ARG, "%s: give both or neither", names[k]);
+        if (!ins[k]) continue;
+        if (!aligned16(ins[k]) || !aligned16(outs[k]))
+            return fail(GDR2_ERR_INVALID_ARG, "%s: not 16-byte aligned", names[k]);
+        if (ins[k] == outs[k] && k == 0 && dt == GDR2_BF16)
+            return fail(GDR2_ERR_INVALID_ARG, "log_alpha (fp32) cannot overwrite a (bf16)");
+    }
+    gdr2::ActArgs args{dt == GDR2_BF16, a ? n_alpha : 0, b_pre ? n_b : 0, w_pre ? n_w : 0, a, b_pre, w_pre,
+                       log_alpha, b, w};
+    return launched(gdr2::launch_gate_activations(args, static_cast<cudaStream_t>(stream)), "gdr2_gate_activations");
+}
+
 gdr2_status gdr2_decode_step_gated(int N, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
                                    const void *k, const void *v, const float *log_alpha, const void *b,
                                    const void *w, float *S, void *o, void *stream)

@@ -59,6 +59,29 @@ struct BwdArgs {
     unsigned *status;
 };
 
+// Block prologue (csrc/prologue.cu).
+struct ConvArgs {
+    int N, T, H, d, width;  // sequences (batches when dense), tokens, heads, channels per head, taps
+    bool bf16, l2norm;
+    float eps;
+    const int *cu_seqlens;  // packed sequences, or null (dense [N, T, H, d])
+    const void *x;
+    const float *weight;    // [H * d][width]
+    const void *state_in;   // [N][width - 1][H][d] or null
+    void *state_out;        // same layout, or null
+    void *y;
+};
+
+struct ActArgs {
+    bool bf16;
+    long long n_alpha, n_b, n_w;
+    const void *a, *b_pre, *w_pre;
+    float *log_alpha;
+    void *b, *w;
+};
+
+cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t s);
+cudaError_t launch_gate_activations(const ActArgs &a, cudaStream_t s);
 cudaError_t launch_forward_simt(const FwdArgs &a, cudaStream_t s);
 cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s);
 bool forward_tc_supported(const FwdArgs &a);

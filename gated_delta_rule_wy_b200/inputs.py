@@ -123,3 +123,32 @@ def make_epilogue_inputs(o_shape, dv, dtype=torch.bfloat16, seed=0, gate_scale=1
     g = (torch.randn(tuple(o_shape), generator=gen) * gate_scale).to(dtype)
     weight = 1.0 + 0.1 * torch.randn((dv,), generator=gen)
     return g, weight
+
+
+def make_conv_inputs(x_shape, W, dtype=torch.bfloat16, seed=0):
+    """Short-convolution branch inputs: x ~ N(0, 1) (a projection's output) in x_shape
+    ([N, T, H, d] or [T, H, d]); taps ~ U(-1/sqrt(W), 1/sqrt(W)) fp32 [H * d, W] (the usual
+    initialisation of a depthwise convolution with W inputs per output); a state
+    ~ N(0, 1) [N, W - 1, H, d] in dtype (N = x_shape[0])."""
+    gen = torch.Generator().manual_seed(int(seed) + 130363)
+    H, d = x_shape[-2], x_shape[-1]
+    x = torch.randn(tuple(x_shape), generator=gen).to(dtype)
+    wgt = (torch.rand((H * d, W), generator=gen) * 2 - 1) / W ** 0.5
+    st = torch.randn((x_shape[0], W - 1, H, d), generator=gen).to(dtype)
+    return x, wgt, st
+
+
+def make_prologue_inputs(B, T, H, dk, dv, W, dtype=torch.bfloat16, seed=0, decay_shift=2.0):
+    """Projection outputs for the whole block prologue: xq, xk [B, T, H, dk], xv [B, T, H, dv]
+    ~ N(0, 1); convolution taps as in make_conv_inputs; decay pre-activation a ~ N(0, 1) +
+    shift and gate pre-activations ~ N(0, 1), so that -softplus(a) and sigmoid give the
+    mixer's input laws above."""
+    gen = torch.Generator().manual_seed(int(seed) + 15485863)
+    out = {}
+    for name, dd in (("q", dk), ("k", dk), ("v", dv)):
+        out["x" + name] = torch.randn((B, T, H, dd), generator=gen).to(dtype)
+        out["conv_" + name] = (torch.rand((H * dd, W), generator=gen) * 2 - 1) / W ** 0.5
+    out["a"] = (torch.randn((B, T, H, dk), generator=gen) + decay_shift).to(dtype)
+    out["b"] = torch.randn((B, T, H, dk), generator=gen).to(dtype)
+    out["w"] = torch.randn((B, T, H, dv), generator=gen).to(dtype)
+    return out

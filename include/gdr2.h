@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 5
+#define GDR2_ABI_VERSION 6
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -223,6 +223,46 @@ gdr2_status gdr2_forward_ex(int B, int T, int H, int dk, int dv, gdr2_dtype dt, 
                             const void *out_gate, const float *norm_weight, float norm_eps,
                             void *o, float *S_T, float *saved_states,
                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Block prologue (Gated DeltaNet-2 note sec. 3, block data-flow paragraph: query and
+ * key go linear -> conv -> SiLU -> L2 norm, the value linear -> conv -> SiLU, and three
+ * separate branches give the decay and the erase and write gates). The linear
+ * projections are the caller's; these two calls take their outputs to the mixer's
+ * inputs. The note gives neither the convolution width nor the activation laws; the
+ * readings taken are stated with each call.
+ *
+ * gdr2_short_conv_silu -- y = SiLU(causal depthwise convolution of x), then, with
+ *   l2norm, y / sqrt(sum over the head's d channels of y^2 + l2_eps) per token and head.
+ *   The convolution has the tap layout of a depthwise Conv1d weight [C, 1, W] left-padded
+ *   by W - 1: y[t, c] = sum_i weight[c][i] x[t - (W - 1) + i, c] (the last tap is the
+ *   current token); inputs before a sequence's first token come from state_in, or are 0.
+ * in:  x [N, T, H, d] dt (dense; N sequences of T tokens), or [T, H, d] with cu_seqlens
+ *      ([N + 1] int32 on the device, as for gdr2_forward_varlen; T = all tokens);
+ *      weight [H * d][width] fp32 (channel c = h * d + j); width 1 .. 4;
+ *      state_in [N][width - 1][H][d] dt or NULL: the width - 1 inputs before each
+ *      sequence, oldest first.
+ * out: y in x's layout (must not be x); state_out in state_in's layout or NULL: the last
+ *      width - 1 inputs of [state_in; sequence] (a sequence without tokens keeps its
+ *      state). state_out may be state_in only for T = 1 without cu_seqlens (a decode step,
+ *      updated in place); otherwise the two must not overlap.
+ * d is 64 or 128; dt fp32 or bf16 (arithmetic fp32); l2_eps finite and >= 0.
+ */
+gdr2_status gdr2_short_conv_silu(int N, int T, int H, int d, gdr2_dtype dt, int width, int l2norm, float l2_eps,
+                                 const int *cu_seqlens, const void *x, const float *weight,
+                                 const void *state_in, void *state_out, void *y, void *stream);
+
+/*
+ * gdr2_gate_activations -- the decay and gate branches' activations, element by element
+ * over flat arrays (any layout: vector or scalar gates alike):
+ *   log_alpha = -softplus(a) = -log(1 + e^a)   (so alpha = sigmoid(-a), in (0, 1))
+ *   b = sigmoid(b_pre),  w = sigmoid(w_pre)
+ * in:  a [n_alpha], b_pre [n_b], w_pre [n_w] in dt; any of them NULL (with its output) to
+ *      skip it. out: log_alpha [n_alpha] fp32; b [n_b], w [n_w] in dt. 16-byte aligned.
+ */
+gdr2_status gdr2_gate_activations(gdr2_dtype dt, long long n_alpha, const void *a, float *log_alpha,
+                                  long long n_b, const void *b_pre, void *b,
+                                  long long n_w, const void *w_pre, void *w, void *stream);
 
 /* Bytes of device scratch gdr2_backward needs for this problem. */
 size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt);

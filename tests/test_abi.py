@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 5
+    assert lib.gdr2_abi_version() == 6
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -189,3 +189,39 @@ def test_forward_ex_checks_the_epilogue_on_the_host(lib):
     assert st == binding.GDR2_ERR_INVALID_ARG and b"workspace" in lib.gdr2_last_error()
     st = lib.gdr2_forward_ex(3, 64, 2, 128, 128, 0, 0, *_ex_args(None, None, 0.0, cu=cu))
     assert st == binding.GDR2_ERR_UNSUPPORTED and b"packed" in lib.gdr2_last_error()
+
+
+def test_prologue_entry_points_check_on_the_host(lib):
+    p, q = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    f = ctypes.c_float
+
+    def conv(N=2, T=8, H=2, d=128, dt=1, W=4, l2=1, eps=1e-6, cu=None, x=p, wgt=p, sin=None, sout=None, y=q):
+        return lib.gdr2_short_conv_silu(N, T, H, d, dt, W, l2, f(eps), cu, x, wgt, sin, sout, y, None)
+
+    assert conv(W=5) == binding.GDR2_ERR_UNSUPPORTED and b"width" in lib.gdr2_last_error()
+    assert conv(W=0) == binding.GDR2_ERR_UNSUPPORTED
+    assert conv(d=96) == binding.GDR2_ERR_UNSUPPORTED
+    assert conv(N=-1) == binding.GDR2_ERR_INVALID_ARG
+    assert conv(l2=2) == binding.GDR2_ERR_INVALID_ARG
+    assert conv(eps=-1.0) == binding.GDR2_ERR_INVALID_ARG and b"l2_eps" in lib.gdr2_last_error()
+    assert conv(y=p) == binding.GDR2_ERR_INVALID_ARG and b"y must not be x" in lib.gdr2_last_error()
+    assert conv(x=ctypes.c_void_p(0x10008)) == binding.GDR2_ERR_INVALID_ARG
+    assert conv(wgt=None) == binding.GDR2_ERR_INVALID_ARG and b"weight" in lib.gdr2_last_error()
+    s = ctypes.c_void_p(0x30000)
+    st = conv(sin=s, sout=s)  # in place needs T = 1 without cu_seqlens
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"state_in" in lib.gdr2_last_error()
+    st = conv(T=1, sin=s, sout=s, cu=ctypes.c_void_p(0x40000))
+    assert st == binding.GDR2_ERR_INVALID_ARG
+    assert conv(cu=ctypes.c_void_p(0x40002)) == binding.GDR2_ERR_INVALID_ARG  # cu_seqlens alignment
+    assert conv(N=0, x=None, wgt=None, y=None) == binding.GDR2_OK  # nothing to do
+    assert conv(H=0, x=None, wgt=None, y=None) == binding.GDR2_OK
+
+    def act(dt=1, na=16, a=p, la=q, nb=0, b=None, bo=None, nw=0, w=None, wo=None):
+        return lib.gdr2_gate_activations(dt, na, a, la, nb, b, bo, nw, w, wo, None)
+
+    assert act(dt=5) == binding.GDR2_ERR_INVALID_ARG
+    assert act(na=-1) == binding.GDR2_ERR_INVALID_ARG
+    assert act(la=None) == binding.GDR2_ERR_INVALID_ARG and b"both or neither" in lib.gdr2_last_error()
+    assert act(a=ctypes.c_void_p(0x10004)) == binding.GDR2_ERR_INVALID_ARG and b"aligned" in lib.gdr2_last_error()
+    assert act(la=p) == binding.GDR2_ERR_INVALID_ARG  # bf16 a cannot become fp32 log_alpha in place
+    assert act(na=0, a=None, la=None) == binding.GDR2_OK

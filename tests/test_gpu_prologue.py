@@ -1,0 +1,124 @@
+"""GPU parity of the block prologue (short causal convolution + SiLU + per-head L2 norm,
+and the decay and gate activations) against the fp64 oracle (Gated DeltaNet-2 note,
+sec. 3, block data-flow paragraph), and of the whole block data flow: prologue, mixer
+and output epilogue against the oracle's chain."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import block as OB
+from gated_delta_rule_wy_b200 import (gdr2_block_prologue, gdr2_forward, gdr2_gate_activations,
+                                      gdr2_short_conv_silu, gdr2_sync_status)
+from gated_delta_rule_wy_b200 import inputs as I
+from parity import TOL, assert_close, assert_epilogue_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _expected_state(x, W, state):
+    """The state after the call is a copy of inputs: exact in the input dtype."""
+    return torch.from_numpy(OB.conv_state_after(_np(x), W, None if state is None else _np(state)))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("W", [4, 2, 1])
+@pytest.mark.parametrize("l2", [True, False])
+def test_dense_conv_matches_the_oracle(dtype, d, W, l2):
+    N, T, H = 2, 77, 3  # 77 tokens: two 32-token runs and a ragged one
+    x, wgt, st = I.make_conv_inputs((N, T, H, d), W, dtype, seed=111)
+    y, s_out = gdr2_short_conv_silu(x.cuda(), wgt.cuda(), st.cuda(), l2norm=l2, eps=1e-6, final_state=True)
+    gdr2_sync_status()
+    xr = _np(x).reshape(N, T, H * d)
+    sr = _np(st).reshape(N, W - 1, H * d)
+    y_ref, s_ref = OB.short_conv_silu(xr, _np(wgt), sr, l2norm=l2, eps=1e-6, heads=H)
+    assert_close(y.reshape(N, T, H * d), y_ref, TOL[dtype], f"y (W={W}, d={d}, l2={l2})")
+    assert torch.equal(s_out.cpu(), torch.from_numpy(s_ref.reshape(N, W - 1, H, d)).to(dtype))
+
+
+def test_without_a_state_the_past_is_zero():
+    x, wgt, _ = I.make_conv_inputs((1, 40, 2, 128), 4, torch.bfloat16, seed=112)
+    y, _ = gdr2_short_conv_silu(x.cuda(), wgt.cuda(), None)
+    gdr2_sync_status()
+    y_ref, _ = OB.short_conv_silu(_np(x).reshape(1, 40, 256), _np(wgt))
+    assert_close(y.reshape(1, 40, 256), y_ref, TOL[torch.bfloat16], "y without a state")
+
+
+@pytest.mark.parametrize("l2", [True, False])
+def test_packed_sequences_convolve_on_their_own(l2):
+    lens = [0, 5, 1, 70, 2, 0, 40]  # empty, short (< W - 1), across 32-token runs
+    T, H, d, W = sum(lens), 2, 128, 4
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    x, wgt, _ = I.make_conv_inputs((T, H, d), W, torch.bfloat16, seed=113)
+    _, _, sts = I.make_conv_inputs((len(lens), 1, H, d), W, torch.bfloat16, seed=114)
+    y, s_out = gdr2_short_conv_silu(x.cuda(), wgt.cuda(), sts.cuda(), l2norm=l2,
+                                    cu_seqlens=torch.tensor(cu, dtype=torch.int32, device="cuda"), final_state=True)
+    gdr2_sync_status()
+    y_ref, s_ref = OB.short_conv_silu(_np(x).reshape(1, T, H * d), _np(wgt), l2norm=l2, heads=H, cu_seqlens=cu,
+                                      states=_np(sts).reshape(len(lens), W - 1, H * d))
+    assert_close(y.reshape(1, T, H * d), y_ref, TOL[torch.bfloat16], "packed y")
+    assert torch.equal(s_out.cpu(), torch.from_numpy(s_ref.reshape(len(lens), W - 1, H, d)).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_steps_in_place_equal_one_call(dtype):
+    """Ten one-token calls, the state updated in place, give the bits of one ten-token call."""
+    N, T, H, d, W = 4, 10, 2, 128, 4
+    x, wgt, st = I.make_conv_inputs((N, T, H, d), W, dtype, seed=115)
+    xc, wc = x.cuda(), wgt.cuda()
+    y_all, s_all = gdr2_short_conv_silu(xc, wc, st.cuda(), l2norm=True, final_state=True)
+    s = st.cuda().clone()
+    ys = []
+    for t in range(T):
+        yt, _ = gdr2_short_conv_silu(xc[:, t:t + 1].contiguous(), wc, s, l2norm=True, state_out=s)
+        ys.append(yt)
+    gdr2_sync_status()
+    assert torch.equal(torch.cat(ys, 1), y_all) and torch.equal(s, s_all)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("shape", [(2, 100, 3, 128), (2, 101, 3)])  # vector gates; scalar gates (ragged count)
+def test_gate_activations_match_the_oracle(dtype, shape):
+    g = torch.Generator().manual_seed(116)
+    a = (torch.randn(shape, generator=g) * 4 + 2).to(dtype)
+    b = (torch.randn(shape, generator=g) * 4).to(dtype)
+    w = (torch.randn(shape, generator=g) * 4).to(dtype)
+    la, bo, wo = gdr2_gate_activations(a.cuda(), b.cuda(), w.cuda())
+    gdr2_sync_status()
+    assert la.dtype == torch.float32 and bo.dtype == dtype
+    assert_close(la, OB.neg_softplus(_np(a)), 1e-5, "log alpha")
+    assert_close(bo, OB.sigmoid(_np(b)), TOL[dtype] / 4, "b")
+    assert_close(wo, OB.sigmoid(_np(w)), TOL[dtype] / 4, "w")
+    la2, _, _ = gdr2_gate_activations(a.cuda())  # one branch alone
+    gdr2_sync_status()
+    assert torch.equal(la2, la)
+
+
+def test_block_data_flow_end_to_end():
+    """Prologue -> mixer -> output epilogue on the GPU against the oracle's same chain from
+    the same projections (B=1, H=2, T=200, d=128, bf16)."""
+    B, T, H, d, W = 1, 200, 2, 128, 4
+    p = I.make_prologue_inputs(B, T, H, d, d, W, torch.bfloat16, seed=117)
+    g, wt = I.make_epilogue_inputs((B, T, H, d), d, seed=118)
+    dv = {k: v.cuda() for k, v in p.items()}
+    q, k, v, la, b, w, _ = gdr2_block_prologue(dv["xq"], dv["xk"], dv["xv"], dv["conv_q"], dv["conv_k"],
+                                               dv["conv_v"], dv["a"], dv["b"], dv["w"])
+    y, S_T, _ = gdr2_forward(q, k, v, la, b, w, None, out_gate=g.cuda(), norm_weight=wt.cuda())
+    gdr2_sync_status()
+    n = {kk: _np(vv) for kk, vv in p.items()}
+    rs = lambda a_: a_.reshape(B, T, H * d)  # noqa: E731
+    back = lambda a_: a_.reshape(B, T, H, d)  # noqa: E731
+    qr, _ = OB.short_conv_silu(rs(n["xq"]), n["conv_q"], l2norm=True, heads=H)
+    kr, _ = OB.short_conv_silu(rs(n["xk"]), n["conv_k"], l2norm=True, heads=H)
+    vr, _ = OB.short_conv_silu(rs(n["xv"]), n["conv_v"], heads=H)
+    o_ref, S_ref = oracle.forward(back(qr), back(kr), back(vr), OB.neg_softplus(n["a"]), OB.sigmoid(n["b"]),
+                                  OB.sigmoid(n["w"]))
+    gn, wn = _np(g), _np(wt)
+    y_ref = OB.output_norm_gate(o_ref, gn, wn, 1e-6)
+    assert_epilogue_close(y, y_ref, o_ref, gn, wn, 1e-6, TOL[torch.bfloat16], "block y")
+    assert_close(S_T, S_ref, TOL[torch.bfloat16], "block S_T")
