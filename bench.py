@@ -203,6 +203,14 @@ def time_steps(fn, steps: int, stream) -> list:
     return [s.elapsed_time(e) for s, e in evs]
 
 
+def time_steps_queued(fn, steps: int, stream) -> list:
+    """time_steps for calls whose host-side work (argument checks, output allocation) can
+    outlast their kernels: the stream first spins on the device long enough for every step
+    to be enqueued, so the events see the kernels back to back, not the host's pace."""
+    torch.cuda._sleep(200_000_000)  # about 0.1 s at the B200's clock
+    return time_steps(fn, steps, stream)
+
+
 # ----------------------------------------------------------------------------- the oracle (CPU baseline)
 def oracle_tokens_per_s(x: I.FwdInputs, heads, nthreads):
     """Time the fp64 oracle on the listed (batch, head) recurrences over the full T."""
@@ -267,7 +275,7 @@ def bench_components(dev, stream, peaks):
 
     for _ in range(5):
         dec()
-    ms = time_steps(dec, 200, stream)
+    ms = time_steps_queued(dec, 200, stream)
     us = 1e3 * statistics.median(ms)
     state_bytes = 2 * N * H * dk * dv * 4
     tok_bytes = N * H * (3 * dk * 2 + dk * 4 + 2 * dv * 2 + dv * 2)  # q,k,b bf16 + log_alpha + v,w + o
@@ -305,7 +313,7 @@ def bench_components(dev, stream, peaks):
 
         for _ in range(3):
             fwd()
-        ms = statistics.median(time_steps(fwd, 10, stream))
+        ms = statistics.median(time_steps_queued(fwd, 10, stream))
         tokens = c["B"] * T
         alg = tokens * c["H"] * BYTES_PER_TOKEN_HEAD + c["B"] * c["H"] * c["dk"] * c["dv"] * 4
         sweep.append({"T": T, "B": c["B"], "ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3),
@@ -332,7 +340,7 @@ def bench_components(dev, stream, peaks):
 
     for _ in range(3):
         fwd_packed()
-    ms = statistics.median(time_steps(fwd_packed, 10, stream))
+    ms = statistics.median(time_steps_queued(fwd_packed, 10, stream))
     gdr2_sync_status()
     out["packed"] = {"workload": f"{Tt} tokens as {len(lens)} packed sequences (random cuts; lengths "
                                  f"{int(lens.min())} .. {int(lens.max())}), H=16, d=128, bf16",
@@ -352,7 +360,7 @@ def bench_components(dev, stream, peaks):
 
     for _ in range(3):
         fwd_kda()
-    ms = statistics.median(time_steps(fwd_kda, 20, stream))
+    ms = statistics.median(time_steps_queued(fwd_kda, 20, stream))
     gdr2_sync_status()
     tokens = c["B"] * c["T"]
     alg = tokens * c["H"] * (BYTES_PER_TOKEN_HEAD - 2 * 256 + 2 * 2) + c["B"] * c["H"] * c["dk"] * c["dv"] * 4
@@ -374,7 +382,7 @@ def bench_components(dev, stream, peaks):
 
     for _ in range(3):
         fwd_epi()
-    ms = statistics.median(time_steps(fwd_epi, 20, stream))
+    ms = statistics.median(time_steps_queued(fwd_epi, 20, stream))
     gdr2_sync_status()
     alg = tokens * c["H"] * (BYTES_PER_TOKEN_HEAD + 2 * c["dv"]) + c["B"] * c["H"] * c["dk"] * c["dv"] * 4
     out["epilogue"] = {"workload": "B=4 H=16 T=4096 d=128 bf16, output RMSNorm x weight x SiLU(gate) fused "
@@ -394,7 +402,7 @@ def bench_components(dev, stream, peaks):
 
     for _ in range(3):
         prologue()
-    ms = statistics.median(time_steps(prologue, 20, stream))
+    ms = statistics.median(time_steps_queued(prologue, 20, stream))
     gdr2_sync_status()
     th = tokens * c["H"]
     # per token-head: q, k, v read and written in bf16; a read in bf16, log alpha written in fp32;

@@ -282,7 +282,8 @@ gdr2_status gdr2_short_conv_silu(int N, int T, int H, int d, gdr2_dtype dt, int 
         return GDR2_OK;
     }
     gdr2::ConvArgs a{N, T, H, d, width, dt == GDR2_BF16, l2norm != 0, l2_eps, cu_seqlens, x, weight,
-                     width > 1 ? state_in : nullptr, width > 1 ? state_out : nullptr, y};
+                     width > 1 ? state_in : nullptr, width > 1 ? state_out : nullptr, y, nullptr};
+    GDR2_TRY(device_status(&a.status));
     return launched(gdr2::launch_short_conv(a, s), "gdr2_short_conv_silu");
 }
 

@@ -70,6 +70,7 @@ struct ConvArgs {
     const void *state_in;   // [N][width - 1][H][d] or null
     void *state_out;        // same layout, or null
     void *y;
+    unsigned *status;       // device status word
 };
 
 struct ActArgs {

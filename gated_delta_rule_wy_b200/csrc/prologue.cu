@@ -19,13 +19,17 @@
 
 #include "gdr2_common.cuh"
 #include "gdr2_launch.h"
+#include "sm100_ptx.cuh"
 
 namespace gdr2 {
 namespace {
 
+using namespace sm100;
+
 constexpr int kMaxWidth = 4;    // taps; the window keeps the kMaxWidth - 1 previous rows
 constexpr int kRun = 32;        // tokens per warp task
 constexpr int kConvWarps = 8;
+constexpr uint64_t kConvWaitNs = 2000000000ull;  // bounded wait for a run's rows (2 s)
 
 template <typename TIn> struct Vec;
 template <> struct Vec<float> {
@@ -85,9 +89,11 @@ struct ConvParams {
     void *state_out;         // [N][W - 1][H][D] or null
     void *y;                 // [Bm, T, H, D]
     float eps;
+    unsigned *status;        // device status word (a wait given up)
 };
 
-__device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
+// silu(v) = v / (1 + e^-v); below v = -87 the denominator overflows and the quotient is 0
+__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
 // The sequence that token t of a packed stream belongs to: the s with cu[s] <= t < cu[s+1].
 __device__ __forceinline__ int find_sequence(const int *cu, int N, int t)
@@ -101,16 +107,30 @@ __device__ __forceinline__ int find_sequence(const int *cu, int N, int t)
     return lo;
 }
 
+// Shared memory of one warp's task: its mbarrier, then the run's rows from kMaxWidth - 1
+// tokens before it (kRun + kMaxWidth - 1 rows of D values).
+template <typename TIn, int D>
+constexpr uint32_t conv_rows_bytes() { return (uint32_t)((kRun + kMaxWidth - 1) * D * sizeof(TIn)); }
+template <typename TIn, int D>
+constexpr uint32_t conv_smem_bytes() { return kConvWarps * (128 + conv_rows_bytes<TIn, D>()); }
+
 template <typename TIn, int D, bool L2>
 __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams p)
 {
     constexpr int V = D / 32;  // channels per lane
-    const int lane = threadIdx.x & 31;
-    const long long task = (long long)blockIdx.x * kConvWarps + (threadIdx.x >> 5);
+    constexpr uint32_t kRowBytes = D * sizeof(TIn);
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char *wsm = smem_raw + warp * (128 + conv_rows_bytes<TIn, D>());
+    uint64_t *bar = reinterpret_cast<uint64_t *>(wsm);
+    const TIn *rows = reinterpret_cast<const TIn *>(wsm + 128);  // row r = token t0 - (kMaxWidth - 1) + r
+
+    const long long task = (long long)blockIdx.x * kConvWarps + warp;
     const long long ntasks = (long long)p.Bm * p.H * p.runs;
     if (task >= ntasks) return;
-    const int run = (int)(task % p.runs);
-    const int h = (int)((task / p.runs) % p.H);
+    // heads fastest: the warps of a block read and write neighbouring slices of the same rows
+    const int h = (int)(task % p.H);
+    const int run = (int)((task / p.H) % p.runs);
     const int bs = (int)(task / ((long long)p.runs * p.H));  // token stream
     const int t0 = run * kRun, t1 = min(p.T, t0 + kRun);
     const int c0 = lane * V;
@@ -119,7 +139,19 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
     const TIn *sin = static_cast<const TIn *>(p.state_in);
     TIn *sout = static_cast<TIn *>(p.state_out);
     const size_t HD = (size_t)p.H * D;
-    auto row = [&](int t) -> size_t { return ((size_t)bs * p.T + t) * HD + (size_t)h * D + c0; };
+    auto grow = [&](int t) -> size_t { return ((size_t)bs * p.T + t) * HD + (size_t)h * D; };
+
+    // the run's rows (and the halo before it) into shared memory, all copies in flight at
+    // once; rows before the stream's start are never read
+    const int r_lo = max(0, (kMaxWidth - 1) - t0), r_hi = t1 - t0 + (kMaxWidth - 1);
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar, (uint32_t)(r_hi - r_lo) * kRowBytes);
+    }
+    __syncwarp();
+    for (int r = r_lo + lane; r < r_hi; r += 32)
+        bulk_load(wsm + 128 + r * kRowBytes, x + grow(t0 - (kMaxWidth - 1) + r), kRowBytes, bar);
 
     // taps, right-aligned in kMaxWidth: wt[i] multiplies the input kMaxWidth - 1 - i back
     float wt[kMaxWidth][V];
@@ -130,7 +162,6 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
             const int j = i - (kMaxWidth - p.W);
             wt[i][v] = j >= 0 ? __ldg(p.weight + ((size_t)h * D + c0 + v) * p.W + j) : 0.f;
         }
-
     // the sequence of t0, its first token and one past its last
     int s = bs, sbeg = 0, send = p.T;
     if (p.cu_seqlens) {
@@ -138,34 +169,41 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
         sbeg = __ldg(p.cu_seqlens + s);
         send = __ldg(p.cu_seqlens + s + 1);
     }
-    // window: win[i] = input at t - (kMaxWidth - 1) + i, from the stream, the state or zero
-    float win[kMaxWidth - 1][V];
-    auto fill_window = [&](int t) {
+    if (!mbar_wait_bounded(bar, 0, kConvWaitNs)) {
+        if (lane == 0) atomicOr(p.status, kStatusTimeout);
+        mbar_wait_bounded(bar, 0, kConvWaitNs);  // let the copies land before the block's memory goes
+        return;
+    }
+    // input tau of this lane's channels: the sequence's own token, its state, or zero
+    auto input = [&](int tau, float (&v)[V]) {
+        if (tau >= sbeg) {
+            Vec<TIn>::template load<V>(rows + (tau - t0 + (kMaxWidth - 1)) * D + c0, v);
+        } else {
+            const int js = (p.W - 1) - (sbeg - tau);  // state row (oldest first), if it has one
+            if (sin && js >= 0)
+                Vec<TIn>::template load<V>(sin + (((size_t)s * (p.W - 1) + js) * p.H + h) * D + c0, v);
+            else
 #pragma unroll
-        for (int i = 0; i < kMaxWidth - 1; ++i) {
-            const int tau = t - (kMaxWidth - 1) + i;
-            if (tau >= sbeg) {
-                Vec<TIn>::template load<V>(x + row(tau), win[i]);
-            } else {
-                const int js = (p.W - 1) - (sbeg - tau);  // state row (oldest first), if it has one
-                if (sin && js >= 0)
-                    Vec<TIn>::template load<V>(sin + (((size_t)s * (p.W - 1) + js) * p.H + h) * D + c0, win[i]);
-                else
-#pragma unroll
-                    for (int v = 0; v < V; ++v) win[i][v] = 0.f;
-            }
+                for (int k = 0; k < V; ++k) v[k] = 0.f;
         }
     };
-    fill_window(t0);
+    // window: win[i] = input t - (kMaxWidth - 1) + i for the next token t, refilled through
+    // the general path only where a sequence starts; each token then reads one row
+    float win[kMaxWidth - 1][V];
+    auto refill = [&](int t) {
+#pragma unroll
+        for (int i = 0; i < kMaxWidth - 1; ++i) input(t - (kMaxWidth - 1) + i, win[i]);
+    };
+    refill(t0);
     for (int t = t0; t < t1; ++t) {
         if (t >= send) {  // the next non-empty sequence starts here
-            while (__ldg(p.cu_seqlens + s + 1) <= t) ++s;
+            while (s + 1 < p.N && __ldg(p.cu_seqlens + s + 1) <= t) ++s;  // stays in [0, N) for any array
             sbeg = __ldg(p.cu_seqlens + s);
             send = __ldg(p.cu_seqlens + s + 1);
-            fill_window(t);
+            refill(t);
         }
         float xt[V], o[V];
-        Vec<TIn>::template load<V>(x + row(t), xt);
+        Vec<TIn>::template load<V>(rows + (t - t0 + (kMaxWidth - 1)) * D + c0, xt);
 #pragma unroll
         for (int v = 0; v < V; ++v) {
             float a = wt[kMaxWidth - 1][v] * xt[v];
@@ -183,7 +221,7 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
 #pragma unroll
             for (int v = 0; v < V; ++v) o[v] *= inv;
         }
-        Vec<TIn>::template store<V>(y + row(t), o);
+        Vec<TIn>::template store<V>(y + grow(t) + c0, o);
 #pragma unroll
         for (int v = 0; v < V; ++v) {
 #pragma unroll
@@ -191,9 +229,10 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
             win[kMaxWidth - 2][v] = xt[v];
         }
         if (sout && t == send - 1) {
-            // the sequence's last token: its state is the last W - 1 inputs, oldest first
-            // (window slot i holds state row i - (kMaxWidth - W); static slots keep the window
-            // in registers)
+            // the sequence's last token: its state is the last W - 1 inputs, oldest first;
+            // after the shift win[i] is input t - (kMaxWidth - 2) + i, so state row
+            // j = i - (kMaxWidth - W), 0 <= j <= W - 2; every read of the old state above
+            // precedes these writes in this lane
 #pragma unroll
             for (int i = 0; i < kMaxWidth - 1; ++i) {
                 const int j = i - (kMaxWidth - p.W);
@@ -223,9 +262,12 @@ cudaError_t launch_conv(const ConvParams &p, bool l2, cudaStream_t st)
     const long long ntasks = (long long)p.Bm * p.H * p.runs;
     const unsigned blocks = (unsigned)((ntasks + kConvWarps - 1) / kConvWarps);
     if (blocks > 0) {
-        if (l2) short_conv_kernel<TIn, D, true><<<blocks, kConvWarps * 32, 0, st>>>(p);
-        else short_conv_kernel<TIn, D, false><<<blocks, kConvWarps * 32, 0, st>>>(p);
-        const cudaError_t e = cudaGetLastError();
+        auto kern = l2 ? short_conv_kernel<TIn, D, true> : short_conv_kernel<TIn, D, false>;
+        constexpr uint32_t smem = conv_smem_bytes<TIn, D>();
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<blocks, kConvWarps * 32, smem, st>>>(p);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (p.cu_seqlens && p.state_out && p.W > 1 && p.N > 0) {
@@ -236,8 +278,17 @@ cudaError_t launch_conv(const ConvParams &p, bool l2, cudaStream_t st)
 }
 
 // ---------------------------------------------------------------- activations
-__device__ __forceinline__ float neg_softplus(float a) { return -(fmaxf(a, 0.f) + log1pf(__expf(-fabsf(a)))); }
-__device__ __forceinline__ float sigmoid(float a) { return 1.f / (1.f + __expf(-a)); }
+// -softplus(a) = -(max(a, 0) + log(1 + e)) with e = exp(-|a|) in (0, 1]: log(1 + e) by its
+// Taylor series e - e^2/2 + e^3/3 below e = 1/32 (truncation below e^4/4, 7e-6 of the value),
+// else from the logarithm intrinsic (absolute error below 4e-7 on [1, 2], 1.2e-5 of the value)
+__device__ __forceinline__ float neg_softplus(float a)
+{
+    const float e = __expf(-fabsf(a));
+    const float l = e < 0.03125f ? e * fmaf(e, fmaf(e, 1.f / 3.f, -0.5f), 1.f) : __logf(1.f + e);
+    return -(fmaxf(a, 0.f) + l);
+}
+// 1 / (1 + e^-a); below a = -87 the denominator overflows and the quotient is 0
+__device__ __forceinline__ float sigmoid(float a) { return __fdividef(1.f, 1.f + __expf(-a)); }
 
 template <typename TIn>
 __device__ __forceinline__ float ld1(const TIn *p, long long i)
@@ -246,52 +297,70 @@ __device__ __forceinline__ float ld1(const TIn *p, long long i)
     else return p[i];
 }
 
-// kind 0: log_alpha = -softplus(a) (fp32 out); kinds 1, 2: sigmoid, in the input dtype.
-// 8 elements per thread per step; the ragged tail element by element.
+// Eight consecutive elements i * 8 .. i * 8 + 7 of a 16-byte aligned array, as fp32.
+template <typename TIn>
+__device__ __forceinline__ void load8(const TIn *in, long long i, float (&v)[8])
+{
+    if constexpr (sizeof(TIn) == 2) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(in + 8 * i);
+        const uint32_t u[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[k]));
+            v[2 * k] = f.x;
+            v[2 * k + 1] = f.y;
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4 *>(in + 8 * i);
+        const float4 b = *reinterpret_cast<const float4 *>(in + 8 * i + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+// kind 0: log_alpha = -softplus(v) to fp32; kinds 1, 2: sigmoid(v) in the input dtype.
+template <typename TIn>
+__device__ __forceinline__ void act8(float (&v)[8], void *out, long long i, int kind)
+{
+    if (kind == 0) {
+        float *o = static_cast<float *>(out) + 8 * i;
+        *reinterpret_cast<float4 *>(o) =
+            make_float4(neg_softplus(v[0]), neg_softplus(v[1]), neg_softplus(v[2]), neg_softplus(v[3]));
+        *reinterpret_cast<float4 *>(o + 4) =
+            make_float4(neg_softplus(v[4]), neg_softplus(v[5]), neg_softplus(v[6]), neg_softplus(v[7]));
+        return;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = sigmoid(v[k]);
+    TIn *o = static_cast<TIn *>(out) + 8 * i;
+    if constexpr (sizeof(TIn) == 2) {
+        uint32_t u[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+            u[k] = *reinterpret_cast<const uint32_t *>(&hv);
+        }
+        *reinterpret_cast<uint4 *>(o) = make_uint4(u[0], u[1], u[2], u[3]);
+    } else {
+        *reinterpret_cast<float4 *>(o) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(o + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
+// One activation over a flat array: 8-element vectors, two per thread per step (both
+// loads in flight), then the ragged tail element by element.
 template <typename TIn>
 __global__ void __launch_bounds__(256) gate_act_kernel(long long n, const TIn *in, void *out, int kind)
 {
     const long long nv = n / 8;
     const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride) {
-        float v[8];
-        if constexpr (sizeof(TIn) == 2) {
-            const uint4 a = *reinterpret_cast<const uint4 *>(in + 8 * i);
-            const uint32_t u[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[k]));
-                v[2 * k] = f.x;
-                v[2 * k + 1] = f.y;
-            }
-        } else {
-            const float4 a = *reinterpret_cast<const float4 *>(in + 8 * i);
-            const float4 b = *reinterpret_cast<const float4 *>(in + 8 * i + 4);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-        }
-        if (kind == 0) {
-            float *o = static_cast<float *>(out) + 8 * i;
-            *reinterpret_cast<float4 *>(o) =
-                make_float4(neg_softplus(v[0]), neg_softplus(v[1]), neg_softplus(v[2]), neg_softplus(v[3]));
-            *reinterpret_cast<float4 *>(o + 4) =
-                make_float4(neg_softplus(v[4]), neg_softplus(v[5]), neg_softplus(v[6]), neg_softplus(v[7]));
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = sigmoid(v[k]);
-            TIn *o = static_cast<TIn *>(out) + 8 * i;
-            if constexpr (sizeof(TIn) == 2) {
-                uint32_t u[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-                    u[k] = *reinterpret_cast<const uint32_t *>(&hv);
-                }
-                *reinterpret_cast<uint4 *>(o) = make_uint4(u[0], u[1], u[2], u[3]);
-            } else {
-                *reinterpret_cast<float4 *>(o) = make_float4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<float4 *>(o + 4) = make_float4(v[4], v[5], v[6], v[7]);
-            }
-        }
+    const long long half = (nv + 1) / 2;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < half; i += stride) {
+        const long long j = i + half;
+        float va[8], vb[8];
+        load8(in, i, va);
+        if (j < nv) load8(in, j, vb);
+        act8<TIn>(va, out, i, kind);
+        if (j < nv) act8<TIn>(vb, out, j, kind);
     }
     for (long long i = 8 * nv + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const float a = ld1(in, i);
@@ -305,7 +374,7 @@ template <typename TIn>
 cudaError_t launch_act(long long n, const void *in, void *out, int kind, int nsm, cudaStream_t st)
 {
     if (n <= 0) return cudaSuccess;
-    const long long want = (n / 8 + 255) / 256 + 1;
+    const long long want = (n / 16 + 255) / 256 + 1;
     const int blocks = (int)(want < 8LL * nsm ? want : 8LL * nsm);
     gate_act_kernel<TIn><<<blocks, 256, 0, st>>>(n, static_cast<const TIn *>(in), out, kind);
     return cudaGetLastError();
@@ -329,6 +398,7 @@ cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t st)
     p.state_out = a.state_out;
     p.y = a.y;
     p.eps = a.eps;
+    p.status = a.status;
     if (a.bf16)
         return a.d == 128 ? launch_conv<__nv_bfloat16, 128>(p, a.l2norm, st) : launch_conv<__nv_bfloat16, 64>(p, a.l2norm, st);
     return a.d == 128 ? launch_conv<float, 128>(p, a.l2norm, st) : launch_conv<float, 64>(p, a.l2norm, st);

@@ -1,10 +1,11 @@
 """Run one libgdr2.so kernel on its benchmark workload, for profilers.
 
-    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd} [--launches N] [--batch B] [--epilogue]
+    python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd,prologue} [--launches N] [--batch B] [--epilogue]
 
 fwd     gdr2_forward   B=4 H=16 T=4096 d=128 bf16 (the 1.3B-model layer)
 decode  gdr2_decode_step  256 sequences x 16 heads, d=128, fp32 state (256 MiB)
 bwd     gdr2_backward  B=2 H=16 T=4096 d=128 bf16 with saved chunk states
+prologue  gdr2_block_prologue  B=4 H=16 T=4096 d=128 bf16, width-4 convolutions
 
 Inputs are drawn once (seeded) and stay on the device; the kernel is then
 launched N times back to back (use ncu -s/-c to pick one launch). --batch
@@ -24,7 +25,7 @@ from .binding import gdr2_backward, gdr2_decode_step, gdr2_forward, gdr2_forward
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=("fwd", "decode", "bwd"))
+    ap.add_argument("kernel", choices=("fwd", "decode", "bwd", "prologue"))
     ap.add_argument("--launches", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--epilogue", action="store_true")
@@ -53,6 +54,17 @@ def main():
                                   c["decay_shift"], gen)
         for _ in range(args.launches):
             gdr2_decode_step(*tok, S)
+    elif args.kernel == "prologue":
+        from .binding import gdr2_block_prologue
+
+        c = dict(I.FWD_1P3B_BF16)
+        if args.batch:
+            c["B"] = args.batch
+        pin = {k: v.to("cuda") for k, v in I.make_prologue_inputs(c["B"], c["T"], c["H"], c["dk"], c["dv"], 4,
+                                                                   c["dtype"], seed=1010).items()}
+        for _ in range(args.launches):
+            gdr2_block_prologue(pin["xq"], pin["xk"], pin["xv"], pin["conv_q"], pin["conv_k"], pin["conv_v"],
+                                pin["a"], pin["b"], pin["w"])
     else:
         c = dict(I.BWD_1P3B_BF16)
         if args.batch:

@@ -247,6 +247,9 @@ gdr2_status gdr2_forward_ex(int B, int T, int H, int dk, int dv, gdr2_dtype dt, 
  *      state). state_out may be state_in only for T = 1 without cu_seqlens (a decode step,
  *      updated in place); otherwise the two must not overlap.
  * d is 64 or 128; dt fp32 or bf16 (arithmetic fp32); l2_eps finite and >= 0.
+ * cu_seqlens is not checked here (gdr2_forward_varlen checks it): an array that breaks
+ * the rule gives unspecified outputs, but every access stays inside the buffers above.
+ * A bounded device wait that gives up is reported by gdr2_sync_status (TIMEOUT).
  */
 gdr2_status gdr2_short_conv_silu(int N, int T, int H, int d, gdr2_dtype dt, int width, int l2norm, float l2_eps,
                                  const int *cu_seqlens, const void *x, const float *weight,
