@@ -195,7 +195,10 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
         for (int i = 0; i < kMaxWidth - 1; ++i) input(t - (kMaxWidth - 1) + i, win[i]);
     };
     refill(t0);
-    for (int t = t0; t < t1; ++t) {
+    const TIn *xr = rows + (kMaxWidth - 1) * D + c0;  // token t's row in shared memory
+    TIn *yr = y + grow(t0) + c0;                      // token t's output row
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t, xr += D, yr += HD) {
         if (t >= send) {  // the next non-empty sequence starts here
             while (s + 1 < p.N && __ldg(p.cu_seqlens + s + 1) <= t) ++s;  // stays in [0, N) for any array
             sbeg = __ldg(p.cu_seqlens + s);
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
             refill(t);
         }
         float xt[V], o[V];
-        Vec<TIn>::template load<V>(rows + (t - t0 + (kMaxWidth - 1)) * D + c0, xt);
+        Vec<TIn>::template load<V>(xr, xt);
 #pragma unroll
         for (int v = 0; v < V; ++v) {
             float a = wt[kMaxWidth - 1][v] * xt[v];
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(kConvWarps * 32) short_conv_kernel(ConvParams 
 #pragma unroll
             for (int v = 0; v < V; ++v) o[v] *= inv;
         }
-        Vec<TIn>::template store<V>(y + grow(t) + c0, o);
+        Vec<TIn>::template store<V>(yr, o);
 #pragma unroll
         for (int v = 0; v < V; ++v) {
 #pragma unroll
