@@ -122,3 +122,23 @@ def test_block_data_flow_end_to_end():
     y_ref = OB.output_norm_gate(o_ref, gn, wn, 1e-6)
     assert_epilogue_close(y, y_ref, o_ref, gn, wn, 1e-6, TOL[torch.bfloat16], "block y")
     assert_close(S_T, S_ref, TOL[torch.bfloat16], "block S_T")
+
+
+@pytest.mark.slow
+def test_full_size_1p3b_layer_prologue_sampled_heads():
+    """B=4 H=16 T=4096 d=128 bf16 width 4, the benchmarked launch; oracle on sampled (b, h)."""
+    B, T, H, d, W = 4, 4096, 16, 128, 4
+    p = I.make_prologue_inputs(B, T, H, d, d, W, torch.bfloat16, seed=1010)
+    dv = {k: v.cuda() for k, v in p.items()}
+    q, k, v, la, b, w, _ = gdr2_block_prologue(dv["xq"], dv["xk"], dv["xv"], dv["conv_q"], dv["conv_k"],
+                                               dv["conv_v"], dv["a"], dv["b"], dv["w"])
+    gdr2_sync_status()
+    for (bb, h) in [(0, 0), (1, 9), (3, 15)]:
+        for name, y, l2 in (("q", q, True), ("k", k, True), ("v", v, False)):
+            xs = _np(p["x" + name][bb:bb + 1, :, h])                       # [1, T, d]
+            ws = _np(p["conv_" + name].reshape(H, d, W)[h])               # [d, W]
+            y_ref, _ = OB.short_conv_silu(xs, ws, l2norm=l2, heads=1)
+            assert_close(y[bb:bb + 1, :, h], y_ref, TOL[torch.bfloat16], f"{name}[b={bb},h={h}]")
+        assert_close(la[bb, :, h], OB.neg_softplus(_np(p["a"][bb, :, h])), 1e-5, f"log alpha[b={bb},h={h}]")
+        assert_close(b[bb, :, h], OB.sigmoid(_np(p["b"][bb, :, h])), TOL[torch.bfloat16] / 4, f"b[b={bb},h={h}]")
+        assert_close(w[bb, :, h], OB.sigmoid(_np(p["w"][bb, :, h])), TOL[torch.bfloat16] / 4, f"w[b={bb},h={h}]")
