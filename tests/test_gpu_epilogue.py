@@ -160,3 +160,19 @@ def test_full_size_1p3b_layer_with_epilogue_sampled_heads():
         assert_epilogue_close(y[b:b + 1, :, h:h + 1], y_ref, o_ref, gi, wn, 1e-6, TOL[torch.bfloat16],
                               f"y[b={b},h={h}]")
         assert_close(S_T[b:b + 1, h:h + 1], S_ref, TOL[torch.bfloat16], f"S_T[b={b},h={h}]")
+
+
+def test_one_token_with_the_epilogue():
+    """T = 1: one partial chunk, its gate tile clipped to one row."""
+    x = I.make_forward_inputs(B=3, H=2, T=1, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=2.0, seed=104,
+                              with_S0=True)
+    g, _ = I.make_epilogue_inputs((3, 1, 2, 128), 128, seed=105)
+    wt = torch.randn(128, generator=torch.Generator().manual_seed(106))
+    d = x.to("cuda")
+    y, _, _ = gdr2_forward(d.q, d.k, d.v, d.log_alpha, d.b, d.w, d.S0, out_gate=g.cuda(), norm_weight=wt.cuda(),
+                           norm_eps=1e-2)
+    gdr2_sync_status()
+    n = x.as_numpy64()
+    o_ref, _ = oracle.forward(n["q"], n["k"], n["v"], n["log_alpha"], n["b"], n["w"], S0=n["S0"])
+    y_ref = output_norm_gate(o_ref, g.double().numpy(), wt.double().numpy(), 1e-2)
+    assert_epilogue_close(y, y_ref, o_ref, g.double().numpy(), wt.double().numpy(), 1e-2, TOL[torch.bfloat16], "T=1 y")

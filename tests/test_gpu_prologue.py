@@ -142,3 +142,40 @@ def test_full_size_1p3b_layer_prologue_sampled_heads():
         assert_close(la[bb, :, h], OB.neg_softplus(_np(p["a"][bb, :, h])), 1e-5, f"log alpha[b={bb},h={h}]")
         assert_close(b[bb, :, h], OB.sigmoid(_np(p["b"][bb, :, h])), TOL[torch.bfloat16] / 4, f"b[b={bb},h={h}]")
         assert_close(w[bb, :, h], OB.sigmoid(_np(p["w"][bb, :, h])), TOL[torch.bfloat16] / 4, f"w[b={bb},h={h}]")
+
+
+def test_width_three_and_fp32_packed():
+    x, wgt, st = I.make_conv_inputs((2, 45, 2, 64), 3, torch.bfloat16, seed=120)
+    y, s_out = gdr2_short_conv_silu(x.cuda(), wgt.cuda(), st.cuda(), l2norm=True, final_state=True)
+    gdr2_sync_status()
+    y_ref, s_ref = OB.short_conv_silu(_np(x).reshape(2, 45, 128), _np(wgt), _np(st).reshape(2, 2, 128), l2norm=True,
+                                      heads=2)
+    assert_close(y.reshape(2, 45, 128), y_ref, TOL[torch.bfloat16], "W=3 y")
+    assert torch.equal(s_out.cpu(), torch.from_numpy(s_ref.reshape(2, 2, 2, 64)).to(torch.bfloat16))
+    lens = [33, 0, 2, 40]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    xp, wp, _ = I.make_conv_inputs((sum(lens), 2, 128), 4, torch.float32, seed=121)
+    _, _, sp = I.make_conv_inputs((len(lens), 1, 2, 128), 4, torch.float32, seed=122)
+    y, s_out = gdr2_short_conv_silu(xp.cuda(), wp.cuda(), sp.cuda(), cu_seqlens=torch.tensor(cu, dtype=torch.int32,
+                                    device="cuda"), final_state=True)
+    gdr2_sync_status()
+    y_ref, s_ref = OB.short_conv_silu(_np(xp).reshape(1, -1, 256), _np(wp), cu_seqlens=cu,
+                                      states=_np(sp).reshape(len(lens), 3, 256))
+    assert_close(y.reshape(1, -1, 256), y_ref, TOL[torch.float32], "fp32 packed y")
+    assert torch.equal(s_out.cpu(), torch.from_numpy(s_ref.reshape(len(lens), 3, 2, 128)).float())
+
+
+def test_no_tokens_pass_the_state_through():
+    _, wgt, st = I.make_conv_inputs((2, 1, 2, 128), 4, torch.bfloat16, seed=123)
+    x = torch.empty((2, 0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    y, s_out = gdr2_short_conv_silu(x, wgt.cuda(), st.cuda(), final_state=True)  # dense, T = 0
+    gdr2_sync_status()
+    assert y.numel() == 0 and torch.equal(s_out.cpu(), st)
+    xp = torch.empty((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")  # two empty packed sequences
+    _, s_out = gdr2_short_conv_silu(xp, wgt.cuda(), st.cuda(), cu_seqlens=cu, final_state=True)
+    gdr2_sync_status()
+    assert torch.equal(s_out.cpu(), st)
+    _, s_zero = gdr2_short_conv_silu(xp, wgt.cuda(), None, cu_seqlens=cu, final_state=True)
+    gdr2_sync_status()
+    assert torch.count_nonzero(s_zero) == 0
