@@ -25,7 +25,7 @@ _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIM
 # Every symbol include/gdr2.h declares (the ABI tests check the exports).
 EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspace_bytes", "gdr2_forward",
                     "gdr2_forward_gated", "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen",
-                    "gdr2_forward_ex", "gdr2_short_conv_silu", "gdr2_gate_activations",
+                    "gdr2_forward_ex", "gdr2_short_conv_silu", "gdr2_gate_activations", "gdr2_segment_states",
                     "gdr2_decode_step", "gdr2_decode_step_gated",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
                     "gdr2_sync_status")
@@ -73,6 +73,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_short_conv_silu.argtypes = [I] * 7 + [ctypes.c_float] + [P] * 7
         lib.gdr2_gate_activations.restype = I
         lib.gdr2_gate_activations.argtypes = [I] + [ctypes.c_longlong, P, P] * 3 + [P]
+        lib.gdr2_segment_states.restype = I
+        lib.gdr2_segment_states.argtypes = [I] * 5 + [P] * 6
         lib.gdr2_forward_gated.restype = I
         lib.gdr2_forward_gated.argtypes = [I, I, I, I, I, I, I] + [P] * 11 + [Z, P]
         lib.gdr2_decode_step_gated.restype = I
@@ -348,6 +350,25 @@ def gdr2_block_prologue(xq, xk, xv, conv_q, conv_k, conv_v, a, b, w, *, states=N
     v, nv = gdr2_short_conv_silu(xv, conv_v, sv, l2norm=False, **kw)
     la, bo, wo = gdr2_gate_activations(a, b, w, stream=stream)
     return q, k, v, la, bo, wo, ((nq, nk, nv) if final_state else None)
+
+
+def gdr2_segment_states(A, Bst, S0=None, *, final_state=True, stream=None):
+    """States entering the segments of split sequences (see include/gdr2.h).
+
+    A: [B, G, H, dk, dk] fp32 segment transitions; Bst: [B, G, H, dk, dv] fp32 segment
+    offsets; S0: [B, H, dk, dv] fp32 or None. Returns (S_starts [B, G, H, dk, dv], S_T or None).
+    """
+    lib = load_library()
+    B, G, H, dk, dv = Bst.shape
+    _check(A, "A", (B, G, H, dk, dk), torch.float32)
+    _check(Bst, "Bst", (B, G, H, dk, dv), torch.float32)
+    _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    S_starts = torch.empty_like(Bst)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=Bst.device) if final_state else None
+    st = lib.gdr2_segment_states(B, G, H, dk, dv, _ptr(A), _ptr(Bst), _ptr(S0), _ptr(S_starts), _ptr(S_T),
+                                 _stream(stream))
+    _raise(lib, st)
+    return S_starts, S_T
 
 
 def gdr2_decode_step(q, k, v, log_alpha, b, w, S, *, out=None, stream=None):

@@ -311,6 +311,24 @@ gdr2_status gdr2_gate_activations(gdr2_dtype dt, long long n_alpha, const void *
     return launched(gdr2::launch_gate_activations(args, static_cast<cudaStream_t>(stream)), "gdr2_gate_activations");
 }
 
+gdr2_status gdr2_segment_states(int B, int G, int H, int dk, int dv, const float *A, const float *Bst,
+                                const float *S0, float *S_starts, float *S_T, void *stream)
+{
+    if (B < 0 || G < 0 || H < 0) return fail(GDR2_ERR_INVALID_ARG, "negative size (B=%d G=%d H=%d)", B, G, H);
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(GDR2_ERR_UNSUPPORTED, "dk and dv must be 64 or 128 (dk=%d dv=%d)", dk, dv);
+    if ((long long)B * G * H * dk * (dk > dv ? dk : dv) > (1ll << 40)) return fail(GDR2_ERR_INVALID_ARG, "problem too large");
+    if ((long long)B * H == 0) return GDR2_OK;
+    const bool segs = G > 0;
+    GDR2_TRY(check_ptr(A, "A", !segs));
+    GDR2_TRY(check_ptr(Bst, "Bst", !segs));
+    GDR2_TRY(check_ptr(S_starts, "S_starts", !segs));
+    GDR2_TRY(check_ptr(S0, "S0", true));
+    GDR2_TRY(check_ptr(S_T, "S_T", true));
+    gdr2::SegArgs a{B, G, H, dk, dv, A, Bst, S0, S_starts, S_T};
+    return launched(gdr2::launch_segment_states(a, static_cast<cudaStream_t>(stream)), "gdr2_segment_states");
+}
+
 gdr2_status gdr2_decode_step_gated(int N, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
                                    const void *k, const void *v, const float *log_alpha, const void *b,
                                    const void *w, float *S, void *o, void *stream)

@@ -81,6 +81,17 @@ struct ActArgs {
     void *b, *w;
 };
 
+// States entering the segments of split sequences (csrc/segments.cu).
+struct SegArgs {
+    int B, G, H, dk, dv;   // batch, segments, heads, state rows and columns
+    const float *A;        // [B][G][H][dk][dk] segment transitions
+    const float *Bst;      // [B][G][H][dk][dv] segment offsets (final states from zero)
+    const float *S0;       // [B][H][dk][dv] or null (zeros)
+    float *S_starts;       // [B][G][H][dk][dv] out: the state entering each segment
+    float *S_T;            // [B][H][dk][dv] or null: the state after the last segment
+};
+
+cudaError_t launch_segment_states(const SegArgs &a, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t s);
 cudaError_t launch_gate_activations(const ActArgs &a, cudaStream_t s);
 cudaError_t launch_forward_simt(const FwdArgs &a, cudaStream_t s);

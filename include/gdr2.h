@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 6
+#define GDR2_ABI_VERSION 7
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -266,6 +266,23 @@ gdr2_status gdr2_short_conv_silu(int N, int T, int H, int d, gdr2_dtype dt, int 
 gdr2_status gdr2_gate_activations(gdr2_dtype dt, long long n_alpha, const void *a, float *log_alpha,
                                   long long n_b, const void *b_pre, void *b,
                                   long long n_w, const void *w_pre, void *w, void *stream);
+
+/*
+ * gdr2_segment_states -- the states entering the G segments of split sequences, for a
+ * forward whose segments run at the same time (on one GPU as a batch, or one segment per
+ * GPU). Across a segment the recurrence is affine in the entering state:
+ * S_out = A_g S_in + B_g, with A_g the product of the segment's (I - k e^T) Diag(alpha)
+ * factors -- the segment's final state from S0 = I with the write gate w = 0 -- and B_g its
+ * final state from S0 = 0 (both from gdr2_forward). This call scans them in order:
+ *   S_starts[g = 0] = S0,  S_starts[g + 1] = A_g S_starts[g] + B_g,  S_T = after the last.
+ * in:  A [B][G][H][dk][dk] fp32, Bst [B][G][H][dk][dv] fp32 (the layout of a batched
+ *      forward's S_T over B * G segments, segment index inside the batch index);
+ *      S0 [B][H][dk][dv] fp32 or NULL (zeros).
+ * out: S_starts [B][G][H][dk][dv] fp32; S_T [B][H][dk][dv] fp32 or NULL.
+ * dk and dv are 64 or 128; fp32 arithmetic; buffers must not overlap.
+ */
+gdr2_status gdr2_segment_states(int B, int G, int H, int dk, int dv, const float *A, const float *Bst,
+                                const float *S0, float *S_starts, float *S_T, void *stream);
 
 /* Bytes of device scratch gdr2_backward needs for this problem. */
 size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dtype dt);

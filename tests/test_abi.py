@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 6
+    assert lib.gdr2_abi_version() == 7
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -225,3 +225,14 @@ def test_prologue_entry_points_check_on_the_host(lib):
     assert act(a=ctypes.c_void_p(0x10004)) == binding.GDR2_ERR_INVALID_ARG and b"aligned" in lib.gdr2_last_error()
     assert act(la=p) == binding.GDR2_ERR_INVALID_ARG  # bf16 a cannot become fp32 log_alpha in place
     assert act(na=0, a=None, la=None) == binding.GDR2_OK
+
+
+def test_segment_states_checks_on_the_host(lib):
+    p = ctypes.c_void_p(0x10000)
+    assert lib.gdr2_segment_states(2, 3, 2, 96, 128, p, p, None, p, None, None) == binding.GDR2_ERR_UNSUPPORTED
+    assert lib.gdr2_segment_states(-1, 3, 2, 128, 128, p, p, None, p, None, None) == binding.GDR2_ERR_INVALID_ARG
+    st = lib.gdr2_segment_states(2, 3, 2, 128, 128, None, p, None, p, None, None)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"A is NULL" in lib.gdr2_last_error()
+    st = lib.gdr2_segment_states(2, 3, 2, 128, 128, p, p, ctypes.c_void_p(0x10004), p, None, None)
+    assert st == binding.GDR2_ERR_INVALID_ARG and b"S0" in lib.gdr2_last_error()
+    assert lib.gdr2_segment_states(0, 3, 2, 128, 128, None, None, None, None, None, None) == binding.GDR2_OK
