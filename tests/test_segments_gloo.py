@@ -72,3 +72,17 @@ def test_two_ranks_reproduce_the_whole_sequence(tmp_path):
         res = json.loads((tmp_path / f"rank{r}.json").read_text())
         assert res["o_err"] <= 1e-12 * max(1.0, res["o_scale"]), res
         assert res["S_err"] <= 1e-12, res
+
+
+def test_the_oracle_is_affine_in_the_entering_state():
+    """What the segments rest on, checked on the fp64 oracle: the final state from any S0 is
+    A S0 + B, A the final state from the identity with the write gate off, B from zero."""
+    x = I.make_forward_inputs(B=1, H=2, T=9, dk=5, dv=3, dtype=torch.float32, decay_shift=0.0, seed=132)
+    n = x.as_numpy64()
+    _, B_ = oracle.forward(n["q"], n["k"], n["v"], n["log_alpha"], n["b"], n["w"])
+    eye = np.broadcast_to(np.eye(5), (1, 2, 5, 5)).copy()
+    _, A_ = oracle.forward(n["q"], n["k"], np.zeros(n["k"].shape), n["log_alpha"], n["b"], np.zeros(n["k"].shape),
+                           S0=eye)
+    S0 = np.random.default_rng(133).standard_normal((1, 2, 5, 3))
+    _, S_T = oracle.forward(n["q"], n["k"], n["v"], n["log_alpha"], n["b"], n["w"], S0=S0)
+    np.testing.assert_allclose(S_T, A_ @ S0 + B_, rtol=0, atol=1e-12)
