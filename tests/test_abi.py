@@ -236,3 +236,17 @@ def test_segment_states_checks_on_the_host(lib):
     st = lib.gdr2_segment_states(2, 3, 2, 128, 128, p, p, ctypes.c_void_p(0x10004), p, None, None)
     assert st == binding.GDR2_ERR_INVALID_ARG and b"S0" in lib.gdr2_last_error()
     assert lib.gdr2_segment_states(0, 3, 2, 128, 128, None, None, None, None, None, None) == binding.GDR2_OK
+
+
+def test_new_binding_functions_validate_before_calling():
+    import torch
+
+    x = torch.zeros(1, 8, 2, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdr2_short_conv_silu(x, torch.zeros(128, 4))
+    with pytest.raises(ValueError, match="multiple of segments"):
+        g.gdr2_forward_segmented(x, x, x, x, x, x, segments=3)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdr2_segment_states(torch.zeros(1, 2, 2, 64, 64), torch.zeros(1, 2, 2, 64, 64))
+    with pytest.raises(ValueError, match="CUDA"):
+        g.gdr2_gate_activations(torch.zeros(16))
