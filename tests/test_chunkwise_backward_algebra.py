@@ -1,0 +1,141 @@
+"""The chunkwise backward's equations, checked on the CPU before any kernel implements them.
+
+A numpy fp64 restatement of the gradient of the decay-normalised WY chunk form (Gated
+DeltaNet-2 note, sec. 3, chunkwise and gate-aware backward paragraphs), against the
+oracle's token-level reverse mode. Per chunk of C tokens entering with state S0, with G
+the cumulative log-decay inside the chunk (G_C its last value):
+
+    e = b k, z = w v, e^ = e exp(G), k^ = k exp(-G), q^ = q exp(G), k~ = k exp(G_C - G)
+    A = strict_lower(E^ K^^T),  P = lower(Q^ K^^T),  T = (I + A)^-1,  W = T E^,  U~ = T Z
+    Q' = Q^ - P W,  M = -K~^T W
+    O = Q' S0 + P U~,   S_C = (Diag(exp G_C) + M) S0 + K~^T U~
+
+and its reverse, chunk by chunk from the last: dS0 = Q'^T dO + (Diag(exp G_C) + M)^T dS_C,
+then through P, T, W, U~ and the decay factors to dq, dk, dv, db, dw and dlog alpha (a
+reverse cumulative sum of dG). This is the plan of the tensor-core backward; the
+token-level kernel stays the path the library runs.
+"""
+import numpy as np
+
+import oracle
+
+
+def _chunk_forward(q, k, v, la, b, w, S0):
+    """One chunk's forward in the WY form; returns O, S_C and what the reverse needs."""
+    C = q.shape[0]
+    G = np.cumsum(la, axis=0)
+    GC = G[-1]
+    e = b * k
+    z = w * v
+    eh, kh, qh = e * np.exp(G), k * np.exp(-G), q * np.exp(G)
+    kt = k * np.exp(GC - G)
+    A = np.tril(eh @ kh.T, -1)
+    P = np.tril(qh @ kh.T)
+    T = np.linalg.inv(np.eye(C) + A)
+    W = T @ eh
+    Ut = T @ z
+    Qp = qh - P @ W
+    M = -kt.T @ W
+    O = Qp @ S0 + P @ Ut
+    SC = (np.diag(np.exp(GC)) + M) @ S0 + kt.T @ Ut
+    return O, SC, dict(G=G, GC=GC, e=e, z=z, eh=eh, kh=kh, qh=qh, kt=kt, P=P, T=T, W=W, Ut=Ut, Qp=Qp, M=M)
+
+
+def _chunk_backward(q, k, v, la, b, w, S0, dO, dSC, f):
+    """Reverse of _chunk_forward: gradients of <dO, O> + <dSC, S_C>."""
+    G, GC, P, T, W, Ut, Qp, M = f["G"], f["GC"], f["P"], f["T"], f["W"], f["Ut"], f["Qp"], f["M"]
+    eh, kh, qh, kt, e, z = f["eh"], f["kh"], f["qh"], f["kt"], f["e"], f["z"]
+    dS0 = Qp.T @ dO + (np.diag(np.exp(GC)) + M).T @ dSC
+    dQp = dO @ S0.T
+    dP = dO @ Ut.T - dQp @ W.T
+    dUt = P.T @ dO + kt @ dSC
+    dM = dSC @ S0.T
+    dGC = np.sum(dSC * S0, axis=1) * np.exp(GC)
+    dkt = Ut @ dSC.T - W @ dM.T
+    dW = -P.T @ dQp - kt @ dM
+    dqh = dQp.copy()
+    dT = dW @ eh.T + dUt @ z.T
+    deh = T.T @ dW
+    dz = T.T @ dUt
+    dA = np.tril(-T.T @ dT @ T.T, -1)
+    deh += dA @ kh
+    dkh = dA.T @ eh
+    dPm = np.tril(dP)
+    dqh += dPm @ kh
+    dkh += dPm.T @ qh
+    # raw inputs and the cumulative decay
+    de = deh * np.exp(G)
+    dG = deh * eh - dkh * kh + dqh * qh - dkt * kt
+    dk = dkh * np.exp(-G) + dkt * np.exp(GC - G)
+    dGC = dGC + np.sum(dkt * kt, axis=0)
+    dq = dqh * np.exp(G)
+    db = de * k
+    dk = dk + de * b
+    dw = dz * v
+    dv = dz * w
+    dG[-1] += dGC
+    dla = np.cumsum(dG[::-1], axis=0)[::-1]
+    return dq, dk, dv, dla, db, dw, dS0
+
+
+def chunkwise_backward(q, k, v, la, b, w, S0, dO, dS_T, C):
+    """[T, d] arrays of one (batch, head); chunks of C tokens (the last one ragged)."""
+    T_ = q.shape[0]
+    bounds = [(s, min(T_, s + C)) for s in range(0, T_, C)]
+    states, feats = [], []
+    S = S0.copy()
+    for s, t in bounds:
+        states.append(S)
+        _, S, f = _chunk_forward(q[s:t], k[s:t], v[s:t], la[s:t], b[s:t], w[s:t], S)
+        feats.append(f)
+    grads = [np.zeros_like(x) for x in (q, k, v, la, b, w)]
+    dS = dS_T.copy()
+    for (s, t), S_in, f in zip(reversed(bounds), reversed(states), reversed(feats)):
+        *g, dS = _chunk_backward(q[s:t], k[s:t], v[s:t], la[s:t], b[s:t], w[s:t], S_in, dO[s:t], dS, f)
+        for acc, gi in zip(grads, g):
+            acc[s:t] = gi
+    return (*grads, dS)
+
+
+def test_chunkwise_backward_equations_match_the_token_level_oracle():
+    rng = np.random.default_rng(151)
+    B, H, T, dk, dv, C = 1, 2, 45, 6, 5, 16  # two full chunks and a ragged one
+    q = rng.standard_normal((B, T, H, dk)) * 0.5
+    k = rng.standard_normal((B, T, H, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((B, T, H, dk)) + 1.0))
+    b = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, H, dk))))
+    w = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, H, dv))))
+    S0 = rng.standard_normal((B, H, dk, dv)) * 0.3
+    dO = rng.standard_normal((B, T, H, dv))
+    dS_T = rng.standard_normal((B, H, dk, dv))
+    ref = oracle.backward(q, k, v, la, b, w, dO, S0=S0, dS_T=dS_T)
+    names = ("dq", "dk", "dv", "dlog_alpha", "db", "dw")
+    for h in range(H):
+        sl = lambda x: x[0, :, h]  # noqa: E731
+        got = chunkwise_backward(*(sl(x) for x in (q, k, v, la, b, w)), S0[0, h], sl(dO), dS_T[0, h], C)
+        for name, g_ in zip(names, got[:6]):
+            r = ref[name][0, :, h]
+            assert np.max(np.abs(g_ - r)) <= 1e-10 * max(1.0, np.max(np.abs(r))), f"{name} head {h}"
+        assert np.max(np.abs(got[6] - ref["dS0"][0, h])) <= 1e-10 * max(1.0, np.max(np.abs(ref["dS0"][0, h])))
+
+
+def test_chunkwise_forward_equations_match_the_oracle():
+    """The forward half of the same restatement, for completeness."""
+    rng = np.random.default_rng(152)
+    T, dk, dv, C = 40, 6, 5, 16
+    q, k = rng.standard_normal((T, dk)), rng.standard_normal((T, dk)) / 2
+    v = rng.standard_normal((T, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((T, dk))))
+    b, w = rng.uniform(0, 1, (T, dk)), rng.uniform(0, 1, (T, dv))
+    S0 = rng.standard_normal((dk, dv))
+    S = S0
+    outs = []
+    for s in range(0, T, C):
+        t = min(T, s + C)
+        O, S, _ = _chunk_forward(q[s:t], k[s:t], v[s:t], la[s:t], b[s:t], w[s:t], S)
+        outs.append(O)
+    o_ref, S_ref = oracle.forward(*(x[None, :, None] for x in (q, k, v, la, b, w)), S0=S0[None, None])
+    assert np.allclose(np.concatenate(outs), o_ref[0, :, 0], rtol=0, atol=1e-11)
+    assert np.allclose(S, S_ref[0, 0], rtol=0, atol=1e-11)
