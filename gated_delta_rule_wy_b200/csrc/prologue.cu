@@ -10,8 +10,9 @@
 // before a sequence's first token; the L2 norm is x / sqrt(sum_head x^2 + eps);
 // log alpha = -softplus(a), b = sigmoid(b'), w = sigmoid(w').
 //
-// Both kernels are HBM streams (one read and one write per element; the convolution's
-// W - 1 halo rows per 32-token run come from L2).
+// Both kernels are HBM streams (one read and one write per element). The convolution
+// stages each 32-token run's rows, and the rows before it that the taps reach (mostly
+// L2 hits), in shared memory by bulk asynchronous copies, all in flight at once.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
