@@ -176,3 +176,32 @@ def test_one_token_with_the_epilogue():
     o_ref, _ = oracle.forward(n["q"], n["k"], n["v"], n["log_alpha"], n["b"], n["w"], S0=n["S0"])
     y_ref = output_norm_gate(o_ref, g.double().numpy(), wt.double().numpy(), 1e-2)
     assert_epilogue_close(y, y_ref, o_ref, g.double().numpy(), wt.double().numpy(), 1e-2, TOL[torch.bfloat16], "T=1 y")
+
+
+def test_packed_scalar_gates_with_the_epilogue():
+    """Packed sequences, b = w = beta per token-head and the output norm and gate, all in one
+    gdr2_forward_ex call, against the oracle sequence by sequence."""
+    lens = [50, 0, 129, 7]
+    T, H = sum(lens), 2
+    x = I.make_forward_inputs(B=1, H=H, T=T, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=2.0, seed=107)
+    beta = torch.sigmoid(torch.randn((T, H), generator=torch.Generator().manual_seed(108))).to(torch.bfloat16)
+    g, wt = I.make_epilogue_inputs((T, H, 128), 128, seed=109)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    d = x.to("cuda")
+    y, S_T, _ = gdr2_forward_varlen(d.q, d.k, d.v, d.log_alpha, beta.cuda(), beta.cuda(),
+                                    torch.tensor(cu, dtype=torch.int32, device="cuda"), out_gate=g.cuda(),
+                                    norm_weight=wt.cuda())
+    gdr2_sync_status()
+    n = x.as_numpy64()
+    bv = np.repeat(beta.double().numpy()[None, ..., None], 128, axis=-1)
+    gn, wn = g.double().numpy(), wt.double().numpy()
+    for i in range(len(lens)):
+        s, e = int(cu[i]), int(cu[i + 1])
+        if e == s:
+            assert torch.count_nonzero(S_T[i]) == 0
+            continue
+        o_ref, S_ref = oracle.forward(n["q"][:, s:e], n["k"][:, s:e], n["v"][:, s:e], n["log_alpha"][:, s:e],
+                                      bv[:, s:e], bv[:, s:e])
+        y_ref = output_norm_gate(o_ref, gn[None, s:e], wn, 1e-6)
+        assert_epilogue_close(y[s:e][None], y_ref, o_ref, gn[None, s:e], wn, 1e-6, TOL[torch.bfloat16], f"seq {i}")
+        assert_close(S_T[i:i + 1], S_ref, TOL[torch.bfloat16], f"seq {i} S_T")
