@@ -154,10 +154,12 @@ def _raise(lib, st):
 
 
 def gdr2_abi_version() -> int:
+    """GDR2_ABI_VERSION of the loaded libgdr2.so."""
     return load_library().gdr2_abi_version()
 
 
 def gdr2_last_error() -> str:
+    """Description of the calling thread's last non-OK status ('' if none)."""
     return load_library().gdr2_last_error().decode(errors="replace")
 
 
@@ -168,6 +170,7 @@ def gdr2_sync_status(stream=None) -> None:
 
 
 def gdr2_forward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Device scratch gdr2_forward needs (0 on the CUDA-core path: fp32, or d other than 128)."""
     lib = load_library()
     return int(lib.gdr2_forward_workspace_bytes(B, T, H, dk, dv, GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
 
@@ -217,6 +220,7 @@ def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_st
 
 
 def gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Device scratch gdr2_forward_varlen needs for N sequences of T tokens in all."""
     lib = load_library()
     return int(lib.gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv,
                                                        GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
@@ -396,6 +400,7 @@ def gdr2_decode_step(q, k, v, log_alpha, b, w, S, *, out=None, stream=None):
 
 
 def gdr2_backward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Device scratch gdr2_backward needs for this problem."""
     lib = load_library()
     return int(lib.gdr2_backward_workspace_bytes(B, T, H, dk, dv, GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
 
