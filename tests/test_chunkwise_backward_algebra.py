@@ -12,8 +12,8 @@ the cumulative log-decay inside the chunk (G_C its last value):
 
 and its reverse, chunk by chunk from the last: dS0 = Q'^T dO + (Diag(exp G_C) + M)^T dS_C,
 then through P, T, W, U~ and the decay factors to dq, dk, dv, db, dw and dlog alpha (a
-reverse cumulative sum of dG). This is the plan of the tensor-core backward; the
-token-level kernel stays the path the library runs.
+reverse cumulative sum of dG). _regrouped_backward below is the form the tensor-core
+backward kernels compute, with its operand precision.
 """
 import numpy as np
 
@@ -22,7 +22,7 @@ import oracle
 
 def _round_significand(x, bits):
     """x with its significand rounded to `bits` bits (half to even) at any exponent: bf16 has
-    8, tf32 11. The exponent range is left alone (the kernels keep factors in range with
+    8. The exponent range is left alone (the kernels keep factors in range with
     half-chunk references; the relative rounding is the same)."""
     m, e = np.frexp(np.asarray(x, dtype=np.float64))
     scale = float(1 << bits)
@@ -31,13 +31,6 @@ def _round_significand(x, bits):
 
 def _exact(a, b, tag=None):
     return a @ b
-
-
-def _tensor_core_plan(a, b, tag=None):
-    """The products of a tensor-core backward: bf16 operands with wide accumulation, except
-    the two P-gradient products (tagged "p_grad"), whose operands are tf32."""
-    bits = 11 if tag == "p_grad" else 8
-    return _round_significand(a, bits) @ _round_significand(b, bits)
 
 
 def _chunk_forward(q, k, v, la, b, w, S0, mm=_exact):
@@ -81,10 +74,8 @@ def _chunk_backward(q, k, v, la, b, w, S0, dO, dSC, f, mm=_exact):
     deh += mm(dA, kh)
     dkh = mm(dA.T, eh)
     dPm = np.tril(dP)
-    # the decay gradient subtracts the large dq^ q^ and dk^ k^ terms below: these two
-    # products carry it, and bf16 operands here alone cost dlog alpha a factor of 7
-    dqh += mm(dPm, kh, "p_grad")
-    dkh += mm(dPm.T, qh, "p_grad")
+    dqh += mm(dPm, kh)
+    dkh += mm(dPm.T, qh)
     # raw inputs and the cumulative decay
     de = deh * np.exp(G)
     dG = deh * eh - dkh * kh + dqh * qh - dkt * kt
@@ -163,11 +154,120 @@ def test_chunkwise_forward_equations_match_the_oracle():
     assert np.allclose(S, S_ref[0, 0], rtol=0, atol=1e-11)
 
 
+def _regrouped_backward(q, k, v, la, b, w, S0, dO, dS_T, C, bf=None, diag_split=True):
+    """The tensor-core backward as its kernels take it, for one (batch, head).
+
+    With U = U~ - W S0 = T (Z - E^ S0) (the pseudo-values that enter the state), the
+    S0-dependent products of the chunk gradient collapse:
+        dU~ = P^T dO + K~ dS_C                 dz = T^T dU~
+        dP  = dO U^T          (lower)          dA = -(dz U^T)   (strictly lower)
+        dK~ = U dS_C^T                         dQ^ = dO S0^T + dP K^
+        dE^ = -dz S0^T + dA K^                 dK^ = dA^T E^ + dP^T Q^
+    and the state gradient between chunks is dS0 = (Diag(exp G_C) + M)^T dS_C + Q'^T dO
+    (the reverse scan). `bf` rounds a product operand (the kernels use bf16 operands with
+    fp32 accumulation); None keeps fp64 throughout. With diag_split, the diagonal of dP
+    stays out of the two decay products (fp32 terms dP_tt k_t and dP_tt q_t instead) and
+    out of dG, where its two contributions cancel exactly.
+    """
+    r = bf if bf is not None else (lambda x: x)
+    T_ = q.shape[0]
+    bounds = [(s, min(T_, s + C)) for s in range(0, T_, C)]
+    states, feats = [], []
+    S = S0.copy()
+    for s, t in bounds:
+        qq, kk, vv, ll, bb, ww = q[s:t], k[s:t], v[s:t], la[s:t], b[s:t], w[s:t]
+        G = np.cumsum(ll, axis=0)
+        GC = G[-1]
+        e = bb * kk
+        z = r(ww * vv)
+        eh, kh, qh = e * np.exp(G), kk * np.exp(-G), qq * np.exp(G)
+        kt = r(kk * np.exp(GC - G))
+        A = np.tril(r(eh) @ r(kh).T, -1)
+        P = r(np.tril(r(qh) @ r(kh).T))
+        Tm = r(np.linalg.inv(np.eye(t - s) + A))
+        W = r(Tm @ r(eh))
+        Ut = r(Tm @ z)
+        Qp = r(qh - P @ W)
+        M = r(-(kt.T @ W))
+        states.append(S)
+        S = np.exp(GC)[:, None] * S + M @ r(S) + kt.T @ Ut
+        feats.append(dict(G=G, GC=GC, e=e, T=Tm, W=W, Ut=Ut, P=P, kt=kt, Qp=Qp, M=M))
+    # reverse scan: the state gradient entering each chunk from its end
+    dSC = [None] * len(bounds)
+    dS = dS_T.copy()
+    for n in range(len(bounds) - 1, -1, -1):
+        s, t = bounds[n]
+        f = feats[n]
+        dSC[n] = dS
+        dS = np.exp(f["GC"])[:, None] * dS + f["M"].T @ r(dS) + f["Qp"].T @ r(dO[s:t])
+    grads = [np.zeros_like(x) for x in (q, k, v, la, b, w)]
+    for n, (s, t) in enumerate(bounds):
+        f = feats[n]
+        qq, kk, vv, bb, ww = q[s:t], k[s:t], v[s:t], b[s:t], w[s:t]
+        G, GC, e = f["G"], f["GC"], f["e"]
+        S0n, dSn, dOn = r(states[n]), r(dSC[n]), r(dO[s:t])
+        # value side
+        U = r(f["Ut"] - f["W"] @ S0n)
+        dUt = r(f["P"].T @ dOn + f["kt"] @ dSn)
+        dz = f["T"].T @ dUt
+        dzb = r(dz)
+        dP = dOn @ U.T
+        dA = -np.tril(dzb @ U.T, -1)
+        dPd = np.diag(dP).copy() if diag_split else np.zeros(t - s)
+        dPs = np.tril(dP, -1) if diag_split else np.tril(dP)
+        dPb, dAb = r(dPs), r(dA)
+        XdqS = r((S0n @ dOn.T).T)
+        XdeS = r((S0n @ dzb.T).T)
+        Xdkt = r((dSn @ U.T).T)
+        rowsum = np.sum(dSn * S0n, axis=1)
+        # key side: the decay products (in the kernels through per-half references)
+        qh, kh, eh = qq * np.exp(G), kk * np.exp(-G), e * np.exp(G)
+        eG, kcf = np.exp(G), np.exp(GC - G)
+        dq = XdqS * eG + (dPb @ r(kh)) * eG
+        de = -XdeS * eG + (dAb @ r(kh)) * eG
+        dkAP = (dAb.T @ r(eh) + dPb.T @ r(qh)) * np.exp(-G)
+        dG = de * e - dkAP * kk + dq * qq - Xdkt * kk * kcf
+        dG[-1] += rowsum * np.exp(GC) + np.sum(Xdkt * kk * kcf, axis=0)
+        out = (dq + dPd[:, None] * kk, dkAP + dPd[:, None] * qq + Xdkt * kcf + de * bb,
+               dz * ww, np.cumsum(dG[::-1], axis=0)[::-1], de * kk, dz * vv)
+        for acc, g in zip(grads, out):
+            acc[s:t] = g
+    return (*grads, dS)
+
+
+def test_regrouped_backward_equations_match_the_token_level_oracle():
+    rng = np.random.default_rng(153)
+    T, dk, dv, C = 45, 6, 5, 16
+    q = rng.standard_normal((T, dk)) * 0.5
+    k = rng.standard_normal((T, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((T, dk)) + 1.0))
+    b = rng.uniform(0, 2, (T, dk))
+    w = rng.uniform(0, 1, (T, dv))
+    S0 = rng.standard_normal((dk, dv)) * 0.3
+    dO = rng.standard_normal((T, dv))
+    dS_T = rng.standard_normal((dk, dv))
+    ref = oracle.backward(*(x[None, :, None] for x in (q, k, v, la, b, w)), dO[None, :, None],
+                          S0=S0[None, None], dS_T=dS_T[None, None])
+    names = ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0")
+    for split in (False, True):
+        got = _regrouped_backward(q, k, v, la, b, w, S0, dO, dS_T, C, diag_split=split)
+        for name, g_ in zip(names, got):
+            r = ref[name][0, :, 0] if name != "dS0" else ref["dS0"][0, 0]
+            assert np.max(np.abs(g_ - r)) <= 1e-10 * max(1.0, np.max(np.abs(r))), f"{name} split={split}"
+
+
+def _bf16_operand(x):
+    return _round_significand(x, 8)
+
+
 def test_precision_plan_of_the_tensor_core_backward():
-    """The operand precision a tensor-core backward can use, on the benchmark's input laws
-    (d = 128, T = 256, C = 64, bf16 inputs): bf16 operands everywhere except the two
-    P-gradient products in tf32 keep all seven gradients within the 2e-2 bf16 bound (about
-    3e-3 to 7e-3 here). With those two in bf16 as well, dlog alpha reached 2.5e-2."""
+    """bf16 product operands with wide accumulation, on the benchmark's input laws (d = 128,
+    T = 256, C = 64, bf16 inputs): all seven gradients stay within 1e-2 of the oracle (3e-3
+    to 7e-3 here) when the diagonal of dP is kept out of the decay products. Left in, its
+    contributions to dq^ q^ and dk^ k^ cancel in dG only after bf16 rounding, and dlog alpha
+    reaches 2.5e-2, above the 2e-2 bound: that is what the split is for."""
     import torch
 
     from gated_delta_rule_wy_b200 import inputs as I
@@ -178,11 +278,18 @@ def test_precision_plan_of_the_tensor_core_backward():
     dO = I.make_upstream_grad(1, 256, 2, 128, 161, dtype=torch.bfloat16).double().numpy()
     ref = oracle.backward(n["q"], n["k"], n["v"], n["log_alpha"], n["b"], n["w"], dO, S0=n["S0"])
     names = ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0")
+    worst_unsplit = 0.0
     for h in range(2):
         sl = lambda a: a[0, :, h]  # noqa: E731
-        got = chunkwise_backward(*(sl(n[f]) for f in ("q", "k", "v", "log_alpha", "b", "w")), n["S0"][0, h],
-                                 sl(dO), np.zeros((128, 128)), 64, mm=_tensor_core_plan)
-        for name, g_ in zip(names, got):
-            r = ref[name][0, :, h] if name != "dS0" else ref["dS0"][0, h]
-            err = np.max(np.abs(g_ - r)) / np.max(np.abs(r))
-            assert err <= 1e-2, f"{name} head {h}: {err:.2e}"
+        args = [sl(n[f]) for f in ("q", "k", "v", "log_alpha", "b", "w")]
+        for split in (True, False):
+            got = _regrouped_backward(*args, n["S0"][0, h], sl(dO), np.zeros((128, 128)), 64, bf=_bf16_operand,
+                                      diag_split=split)
+            for name, g_ in zip(names, got):
+                r = ref[name][0, :, h] if name != "dS0" else ref["dS0"][0, h]
+                err = np.max(np.abs(g_ - r)) / np.max(np.abs(r))
+                if split:
+                    assert err <= 1e-2, f"{name} head {h}: {err:.2e}"
+                elif name == "dlog_alpha":
+                    worst_unsplit = max(worst_unsplit, err)
+    assert worst_unsplit > 2e-2
