@@ -313,36 +313,52 @@ cudaError_t launch_dt(const BwdArgs &a, cudaStream_t s)
 
 }  // namespace
 
-size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool /*bf16*/)
+// The token-level path (any supported dk, dv and dtype).
+static cudaError_t launch_backward_simt(const BwdArgs &a, cudaStream_t s)
 {
-    return bwd_layout(B, T, H, dk, dv, true).total;
+    if (a.B * a.H == 0) return cudaSuccess;
+    return a.bf16 ? launch_dt<__nv_bfloat16>(a, s) : launch_dt<float>(a, s);
+}
+
+// bf16 at dk = dv = 128 takes the chunkwise tensor-core path (bwd_tc.cu); its workspace is
+// the larger, so the size covers either path.
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf16)
+{
+    const size_t simt = bwd_layout(B, T, H, dk, dv, true).total;
+    if (bf16 && dk == 128 && dv == 128 && T > 0) {
+        const size_t tcb = backward_tc_workspace_bytes(B, T, H);
+        return tcb > simt ? tcb : simt;
+    }
+    return simt;
 }
 
 cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s)
 {
     if (a.B * a.H == 0) return cudaSuccess;
-    return a.bf16 ? launch_dt<__nv_bfloat16>(a, s) : launch_dt<float>(a, s);
+    if (backward_tc_supported(a)) return launch_backward_tc(a, s);
+    return launch_backward_simt(a, s);
 }
 
 }  // namespace gdr2
 
 // ---------------------------------------------------------------------------
 // Variant for callers that may not allocate device memory: the workspace is a
-// file-scope device array of GDR2_NOALLOC_SCRATCH_BYTES. Host code must not
-// use the array's name as a device address (it is a host-side stand-in): the
-// address is looked up once per device with cudaGetSymbolAddress, with that
-// device current, and passed to the same kernel. The kernel writes every
-// scratch word before reading it, so stale contents from the previous call
-// do no harm; concurrent calls on one device share the array and race.
+// file-scope device array of GDR2_NOALLOC_SCRATCH_BYTES, used by the token-level
+// kernels (whose scratch the array is sized for). Host code must not use the
+// array's name as a device address (it is a host-side stand-in): the address is
+// looked up per device with cudaGetSymbolAddress, with that device current, and
+// passed to the kernel. Only a successful lookup is kept; after a failure the
+// next call looks again. The kernel writes every scratch word before reading
+// it, so stale contents from the previous call do no harm; concurrent calls on
+// one device share the array and race.
 namespace gdr2 {
 namespace {
 
 static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[GDR2_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxNoAllocDevices = 64;
-void *g_noalloc_ptr[kMaxNoAllocDevices];
-cudaError_t g_noalloc_err[kMaxNoAllocDevices];
-std::once_flag g_noalloc_once[kMaxNoAllocDevices];
+void *g_noalloc_ptr[kMaxNoAllocDevices];  // null until a lookup on that device succeeds
+std::mutex g_noalloc_mu;
 
 }  // namespace
 
@@ -357,16 +373,20 @@ cudaError_t launch_backward_noalloc(const BwdArgs &a_in, cudaStream_t s)
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxNoAllocDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_noalloc_once[dev], [dev] {
-        void *ptr = nullptr;
-        g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch);
-        g_noalloc_ptr[dev] = ptr;
-    });
-    if (g_noalloc_err[dev] != cudaSuccess) return g_noalloc_err[dev];
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        scratch = g_noalloc_ptr[dev];
+        if (!scratch) {
+            e = cudaGetSymbolAddress(&scratch, g_bwd_noalloc_scratch);
+            if (e != cudaSuccess) return e;
+            g_noalloc_ptr[dev] = scratch;
+        }
+    }
     BwdArgs a = a_in;
-    a.workspace = g_noalloc_ptr[dev];
+    a.workspace = scratch;
     a.workspace_bytes = GDR2_NOALLOC_SCRATCH_BYTES;
-    return launch_backward(a, s);
+    return launch_backward_simt(a, s);
 }
 
 }  // namespace gdr2

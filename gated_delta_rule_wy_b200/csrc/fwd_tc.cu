@@ -59,18 +59,15 @@
 #include "gdr2_common.cuh"
 #include "gdr2_launch.h"
 #include "sm100_ptx.cuh"
+#include "tc_common.cuh"
 
 namespace gdr2 {
 namespace {
 
 using namespace sm100;
+using namespace tc;
 
-constexpr int C = 64;
-constexpr int DK = 128;
-constexpr int DV = 128;
 constexpr int NT = 256;                           // 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr float kFactorLimit = 70.f;              // |exponent| of one decay factor
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_STG_Q = 0;       // q  [64][128] bf16
@@ -114,58 +111,6 @@ struct Misc {
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 static_assert(offsetof(Misc, gC) % 16 == 0, "per-channel vectors are 16-byte aligned");
 
-// Offset of the 16-byte chunk holding columns [8*o8, 8*o8 + 8) of `row`.
-__device__ __forceinline__ uint32_t sw_chunk(int row, int o8, int rows)
-{
-    const int blk = o8 >> 3, ch = o8 & 7;
-    return (uint32_t)(blk * rows * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&f)[8])
-{
-    uint4 u;
-    __nv_bfloat162 h;
-    h = __floats2bfloat162_rn(f[0], f[1]); u.x = *reinterpret_cast<uint32_t *>(&h);
-    h = __floats2bfloat162_rn(f[2], f[3]); u.y = *reinterpret_cast<uint32_t *>(&h);
-    h = __floats2bfloat162_rn(f[4], f[5]); u.z = *reinterpret_cast<uint32_t *>(&h);
-    h = __floats2bfloat162_rn(f[6], f[7]); u.w = *reinterpret_cast<uint32_t *>(&h);
-    return u;
-}
-
-__device__ __forceinline__ void unpack8(uint4 u, float (&f)[8])
-{
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 x = __bfloat1622float2(h[i]);
-        f[2 * i] = x.x;
-        f[2 * i + 1] = x.y;
-    }
-}
-
-__device__ __forceinline__ void load8f(const float *p, float (&f)[8])
-{
-    const float4 a = *reinterpret_cast<const float4 *>(p);
-    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
-__device__ __forceinline__ void store8f(float *p, const float (&f)[8])
-{
-    *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
-    *reinterpret_cast<float4 *>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
-}
-
-// ---- workspace slot written by the chunk kernel, read by the scan kernel ----
-// (one per (batch, head, chunk); operand images in the scan kernel's layouts)
-constexpr uint32_t SLOT_B1 = 0;       // [Q'; M]  [c' block][64 t + 128 c rows][64 c'] (K-major B, N = 192)
-constexpr uint32_t SLOT_KT = 49152;   // K~       [c block][t rows][64 c]   (MN-major B)
-constexpr uint32_t SLOT_U = 65536;    // U~^T     [j rows][64 t]            (K-major A)
-constexpr uint32_t SLOT_P = 81920;    // P        [t rows][64 i]            (K-major B)
-constexpr uint32_t SLOT_BYTES = 90112;
-constexpr int B1_ROWS = 192;          // rows of [Q'; M]: t first, then c
-constexpr uint32_t GAMMA_BYTES = DK * 4;  // exp(G_C), stored after all slots
-
 struct ChunkParams {
     int B, T, H, NC;
     int ntasks;            // slot capacity: B * H * NC (dense), task = bh * NC + n
@@ -179,6 +124,7 @@ struct ChunkParams {
     const int *ntasks_dev;  // H * cu_chunks[B], written by the prefix kernel
     int gates;              // kGate* bits: a scalar gate is read here, not by the copy engine
     const __nv_bfloat16 *bg, *wg;
+    unsigned char *ext;     // backward: T and W of every task (EXT_BYTES each), else null
 };
 
 // Where a task's chunk lives: tensor-map coordinates (token t0, sequence bb), head h, and the
@@ -186,18 +132,6 @@ struct ChunkParams {
 struct ChunkLoc {
     int h, t0, bb, Cn;
 };
-
-// 1 / d for 2^-126 <= d < 2^126 (normal, positive). Seed: the bit pattern of a float is close to 2^23 (log2 d + 127),
-// so subtracting it from a constant negates log2 d: one integer operation gives 1 / d to
-// within 5.1% in every binade (the constant minimises that error over one binade). Two
-// Newton steps r <- r + r (1 - d r), each squaring the relative error, leave 6.6e-6.
-// All of it on the FMA and integer pipes: the special-function unit is the scarce one.
-__device__ __forceinline__ float recip_newton2(float d)
-{
-    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
-    r = fmaf(r, fmaf(-d, r, 1.f), r);
-    return fmaf(r, fmaf(-d, r, 1.f), r);
-}
 
 template <bool GENERAL>
 __device__ __forceinline__ ChunkLoc locate_chunk(const ChunkParams &p, int task)
@@ -271,8 +205,9 @@ constexpr uint32_t CK_M = 0, CK_U = 128, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384,
 constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W_0, W_1 once those are read
 
 // GENERAL: packed sequences and/or scalar gates may be in use; the other instantiation is
-// the dense, vector-gate kernel with those branches compiled away.
-template <bool GENERAL>
+// the dense, vector-gate kernel with those branches compiled away. BWD (dense, vector gates):
+// T and W of each task also go to p.ext for the backward.
+template <bool GENERAL, bool BWD = false>
 __global__ void __launch_bounds__(NT, 1)
 fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
@@ -935,6 +870,11 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // U~^T is staged: to the slot in the background (from warp 2, which has nothing to issue)
         if (tid == 64) {
             bulk_store(slot + SLOT_U, sm + OFF_Z, 16384);
+            if (BWD) {
+                unsigned char *ext = p.ext + (size_t)task * EXT_BYTES;
+                bulk_store(ext + EXT_T, sm + OFF_TB, 8192);
+                bulk_store(ext + EXT_W, sm + OFF_STACK, 16384);
+            }
             bulk_commit_group();
         }
         // ================= Q' - Q^ = -P W (M = 64) ;  M = -K~^T W =================
@@ -951,6 +891,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             mma_commit(&ms.bar_mma);
         }
+        if (BWD && tid == 64) bulk_wait_group_read0();  // T and W have left STACK and R
         if (!wait_bar(&ms.bar_mma, ph_mma)) { timed_out = true; break; }
         tc_fence_after_sync();
         // ================= [Q'; M] -> [c' block][192 rows][64 c'] over STACK and R (for the slot) =================
@@ -1051,23 +992,6 @@ constexpr int kEpiNorm = 1, kEpiGate = 2;
 constexpr uint32_t scan_smem_bytes(int epi)
 {
     return ((epi & kEpiGate) ? SC_G + 16384 : (epi & kEpiNorm) ? SC_EPI + 1280 : SC_MISC + 1280) + 1024;
-}
-
-// Sum vals over the 32 lanes of a warp for each of its N entries; on return lane L holds, in
-// vals[0 .. N/32), the sums of the N/32 entries from (N/32) L on.
-template <int N>
-__device__ __forceinline__ void transpose_reduce32(float (&vals)[N], int lane)
-{
-#pragma unroll
-    for (int o = 16, n = N; o >= 1; o >>= 1, n >>= 1) {
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < n / 2; ++i) {
-            const float send = upper ? vals[i] : vals[i + n / 2];
-            const float keep = upper ? vals[i + n / 2] : vals[i];
-            vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-    }
 }
 
 template <int EPI>
@@ -1345,43 +1269,6 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
 }
 
 // ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// [B, T, H, D] token-major tensor as a 4-D map {D, H, T, B}; box = D x 1 head x 64
-// tokens x 1 sequence. The per-sequence extent T makes loads past the end of a
-// sequence read zeros and stores past it drop.
-bool make_map(CUtensorMap *m, const void *base, bool f32, int B, int T, int H, int D)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t esz = f32 ? 4 : 2;
-    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)D * esz, (cuuint64_t)H * D * esz, (cuuint64_t)T * H * D * esz};
-    cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool forward_tc_supported(const FwdArgs &a)
@@ -1420,8 +1307,12 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     // the output gate has the layout of o; without one the o map stands in, unused
     if (!a.out_gate) mg = mo; else if (!make_map(&mg, a.out_gate, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
     const bool general = varlen || bsc || wsc;
-    cudaError_t e = cudaFuncSetAttribute(general ? fwd_chunk_kernel<true> : fwd_chunk_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    const bool bwd = a.bwd_ext != nullptr;
+    if (bwd && general) return cudaErrorInvalidValue;
+    void (*chunk)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                  const CUtensorMap, ChunkParams) =
+        general ? fwd_chunk_kernel<true> : bwd ? fwd_chunk_kernel<false, true> : fwd_chunk_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int epi = (a.norm_weight ? kEpiNorm : 0) | (a.out_gate ? kEpiGate : 0);
     void (*scan)(const CUtensorMap, const CUtensorMap, ScanParams) =
@@ -1445,14 +1336,11 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     ChunkParams cp{a.B,         a.T,       a.H,        NC,
                    ntasks,      ws,        a.status,   a.cu_seqlens,
                    cu_chunks,   ntasks_dev, a.gates,   static_cast<const __nv_bfloat16 *>(a.b),
-                   static_cast<const __nv_bfloat16 *>(a.w)};
+                   static_cast<const __nv_bfloat16 *>(a.w), a.bwd_ext};
     const int grid = ntasks < nsm ? ntasks : nsm;
-    if (general)
-        fwd_chunk_kernel<true><<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
-    else
-        fwd_chunk_kernel<false><<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
+    chunk<<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || a.chunks_only) return e;
     ScanParams sp{a.B,          a.T,          a.H,    NC,       ntasks,    ws,
                   a.S0,         a.S_T,        a.saved_states, a.status, a.cu_seqlens, cu_chunks,
                   static_cast<__nv_bfloat16 *>(a.o), a.norm_weight, a.norm_eps};

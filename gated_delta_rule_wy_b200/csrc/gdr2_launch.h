@@ -26,6 +26,10 @@ struct FwdArgs {
     const void *out_gate;      // bf16, the layout of o, or null
     const float *norm_weight;  // [dv], or null for no norm
     float norm_eps;
+    // backward's use of the tensor-core forward (dense, vector gates): the chunk kernel also
+    // writes T and W of every task here; chunks_only leaves out the scan kernel
+    unsigned char *bwd_ext = nullptr;
+    bool chunks_only = false;
 };
 
 struct DecodeArgs {
@@ -104,5 +108,8 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf16);
 cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s);
 size_t backward_noalloc_scratch_needed(int B, int T, int H, int dk, int dv, bool have_saved_states);
 cudaError_t launch_backward_noalloc(const BwdArgs &a, cudaStream_t s);
+bool backward_tc_supported(const BwdArgs &a);
+size_t backward_tc_workspace_bytes(int B, int T, int H);
+cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s);
 
 }  // namespace gdr2

@@ -226,10 +226,15 @@ def _regrouped_backward(q, k, v, la, b, w, S0, dO, dS_T, C, bf=None, diag_split=
         dq = XdqS * eG + (dPb @ r(kh)) * eG
         de = -XdeS * eG + (dAb @ r(kh)) * eG
         dkAP = (dAb.T @ r(eh) + dPb.T @ r(qh)) * np.exp(-G)
-        dG = de * e - dkAP * kk + dq * qq - Xdkt * kk * kcf
-        dG[-1] += rowsum * np.exp(GC) + np.sum(Xdkt * kk * kcf, axis=0)
+        # dlog alpha: a suffix sum of dG, the state term, and the dK~ term as a prefix sum
+        # (the same total as suffix sums of -dK~ k~ plus their chunk total, without the
+        # cancellation that form suffers under strong decay)
+        dG = de * e - dkAP * kk + dq * qq
+        ktk = Xdkt * kk * kcf
+        dla = (np.cumsum(dG[::-1], axis=0)[::-1] + rowsum * np.exp(GC)
+               + np.concatenate([np.zeros((1, ktk.shape[1])), np.cumsum(ktk, axis=0)[:-1]]))
         out = (dq + dPd[:, None] * kk, dkAP + dPd[:, None] * qq + Xdkt * kcf + de * bb,
-               dz * ww, np.cumsum(dG[::-1], axis=0)[::-1], de * kk, dz * vv)
+               dz * ww, dla, de * kk, dz * vv)
         for acc, g in zip(grads, out):
             acc[s:t] = g
     return (*grads, dS)
