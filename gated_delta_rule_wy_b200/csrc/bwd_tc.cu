@@ -114,13 +114,13 @@ __global__ void __launch_bounds__(RS_NT, 1) bwd_scan_kernel(const __grid_constan
     const uint32_t tm = ms.tmem_base;
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
 
-    bool pend[2] = {false, false};  // thread 0: a buffer's loads were issued and not yet waited for
+    unsigned pend = 0;  // thread 0: bit b set while buffer b's loads are issued and not yet waited for
     auto issue = [&](int n, int sl) {
         const size_t task = base + n;
         unsigned char *buf = sm + sl * RS_BUF;
         mbar_arrive_expect_tx(&ms.bar_full[sl], 2 * B1_ROWS * 128 + GAMMA_BYTES + C * DV * 2);
         bulk_load(buf, p.ws + task * SLOT_BYTES + SLOT_B1, 2 * B1_ROWS * 128, &ms.bar_full[sl]);
-        pend[sl] = true;
+        pend |= 1u << sl;
         bulk_load(ms.gam[sl], p.ws + (size_t)p.ntasks * SLOT_BYTES + task * GAMMA_BYTES, GAMMA_BYTES,
                   &ms.bar_full[sl]);
         tma_load_4d(buf + RS_DO, &tm_do, &ms.bar_full[sl], 0, h, n * C, bb);
@@ -143,11 +143,12 @@ __global__ void __launch_bounds__(RS_NT, 1) bwd_scan_kernel(const __grid_constan
     tc_fence_before_sync();
     __syncthreads();
 
-    uint32_t ph_full[2] = {0, 0}, ph_mma = 0;
+    unsigned phf = 0;  // bit b: the parity of buffer b's next load phase
+    uint32_t ph_mma = 0;
     bool timed_out = false;
     if (NC > 0) {
         const bool ok = mbar_wait_bounded(&ms.bar_full[0], 0, kWaitLimitNs);
-        if (ok) ph_full[0] = 1, pend[0] = false;
+        if (ok) phf ^= 1u, pend &= ~1u;
         if (__syncthreads_or(!ok)) timed_out = true;
     }
     for (int k = 0; k < NC && !timed_out; ++k) {
@@ -214,8 +215,9 @@ __global__ void __launch_bounds__(RS_NT, 1) bwd_scan_kernel(const __grid_constan
         {
             bool ok = true;
             if (k + 1 < NC) {
-                ok = mbar_wait_bounded(&ms.bar_full[sl ^ 1], ph_full[sl ^ 1], kWaitLimitNs);
-                if (ok) ph_full[sl ^ 1] ^= 1u, pend[sl ^ 1] = false;
+                const unsigned nb = (unsigned)(sl ^ 1);
+                ok = mbar_wait_bounded(&ms.bar_full[nb], (phf >> nb) & 1u, kWaitLimitNs);
+                if (ok) phf ^= 1u << nb, pend &= ~(1u << nb);
             }
             ok = mbar_wait_bounded(&ms.bar_mma, ph_mma, kWaitLimitNs) && ok;
             ph_mma ^= 1u;
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(RS_NT, 1) bwd_scan_kernel(const __grid_constan
     if (timed_out && tid == 0) {
         // loads still in flight (issued, never waited for) land before shared memory goes
         for (int b2 = 0; b2 < 2; ++b2)
-            if (pend[b2]) mbar_wait_bounded(&ms.bar_full[b2], ph_full[b2], kWaitLimitNs);
+            if (pend & (1u << b2)) mbar_wait_bounded(&ms.bar_full[b2], (phf >> b2) & 1u, kWaitLimitNs);
         atomicOr(p.status, kStatusTimeout);
     }
     tc_fence_before_sync();

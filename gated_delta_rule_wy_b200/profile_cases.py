@@ -1,6 +1,7 @@
 """Run one libgdr2.so kernel on its benchmark workload, for profilers.
 
     python -m gated_delta_rule_wy_b200.profile_cases {fwd,decode,bwd,prologue} [--launches N] [--batch B] [--epilogue]
+        [--recompute]
 
 fwd     gdr2_forward   B=4 H=16 T=4096 d=128 bf16 (the 1.3B-model layer)
 decode  gdr2_decode_step  256 sequences x 16 heads, d=128, fp32 state (256 MiB)
@@ -11,7 +12,8 @@ Inputs are drawn once (seeded) and stay on the device; the kernel is then
 launched N times back to back (use ncu -s/-c to pick one launch). --batch
 overrides B of the forward and backward cases (a smaller capture whose inputs
 still exceed the 126 MB L2 at B >= 2). --epilogue runs the forward with the block's
-output epilogue (RMSNorm weight and SiLU gate, seeded like the bench's).
+output epilogue (RMSNorm weight and SiLU gate, seeded like the bench's). --recompute runs
+the backward without saved chunk states (the call recomputes them).
 """
 from __future__ import annotations
 
@@ -29,6 +31,7 @@ def main():
     ap.add_argument("--launches", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--epilogue", action="store_true")
+    ap.add_argument("--recompute", action="store_true")
     args = ap.parse_args()
     torch.cuda.set_device(0)
     if args.kernel == "fwd":
@@ -73,7 +76,7 @@ def main():
         dO = I.make_upstream_grad(c["B"], c["T"], c["H"], c["dv"], c["seed"], dtype=c["dtype"]).cuda()
         _, _, saved = gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, None, save_states=True)
         for _ in range(args.launches):
-            gdr2_backward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, dO, None, None, saved)
+            gdr2_backward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, dO, None, None, None if args.recompute else saved)
     gdr2_sync_status()
     print(f"profile_cases {args.kernel}: {args.launches} launches ok")
 
