@@ -9,6 +9,7 @@ fallback: if ``libgdr2.so`` is missing or cannot be loaded, every call raises.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import threading
 
@@ -27,8 +28,8 @@ EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspa
                     "gdr2_forward_gated", "gdr2_forward_varlen_workspace_bytes", "gdr2_forward_varlen",
                     "gdr2_forward_ex", "gdr2_short_conv_silu", "gdr2_gate_activations", "gdr2_segment_states",
                     "gdr2_decode_step", "gdr2_decode_step_gated",
-                    "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_noalloc",
-                    "gdr2_sync_status")
+                    "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_gated", "gdr2_backward_noalloc",
+                    "gdr2_sync_status", "gdr2_debug_force_timeout", "gdr2_debug_recip")
 NOALLOC_SCRATCH_BYTES = 64 << 20  # GDR2_NOALLOC_SCRATCH_BYTES
 
 
@@ -84,12 +85,56 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
         lib.gdr2_backward.restype = I
         lib.gdr2_backward.argtypes = [I, I, I, I, I, I] + [P] * 18 + [Z, P]
+        lib.gdr2_backward_gated.restype = I
+        lib.gdr2_backward_gated.argtypes = [I, I, I, I, I, I, I] + [P] * 18 + [Z, P]
         lib.gdr2_backward_noalloc.restype = I
         lib.gdr2_backward_noalloc.argtypes = [I, I, I, I, I, I] + [P] * 18
         lib.gdr2_sync_status.restype = I
         lib.gdr2_sync_status.argtypes = [P]
+        lib.gdr2_debug_force_timeout.restype = None
+        lib.gdr2_debug_force_timeout.argtypes = [I]
+        lib.gdr2_debug_recip.restype = I
+        lib.gdr2_debug_recip.argtypes = [P, P, ctypes.c_longlong, P]
         _lib = lib
         return lib
+
+
+def _tensors_in(args, kwargs):
+    for a in list(args) + list(kwargs.values()):
+        if isinstance(a, torch.Tensor):
+            yield a
+        elif isinstance(a, (list, tuple)):
+            yield from (x for x in a if isinstance(x, torch.Tensor))
+
+
+def _device_of(tensors):
+    """The one device the tensors live on (None without tensors); raises if they span several."""
+    devs = {t.device for t in tensors}
+    if len(devs) > 1:
+        names = ", ".join(sorted(str(d) for d in devs))
+        raise ValueError(f"all tensors of a call must be on one CUDA device; got {names}")
+    return next(iter(devs)) if devs else None
+
+
+def _one_device(fn):
+    """Run a library call on the device that holds its tensors.
+
+    The library launches on the current CUDA device and stream, so tensors on another
+    device would reach kernels as foreign pointers: the call is made under that device
+    (its current stream unless one is given), after checking that every tensor argument
+    and the stream share it.
+    """
+    @functools.wraps(fn)
+    def call(*args, **kwargs):
+        dev = _device_of(_tensors_in(args, kwargs))
+        if dev is None or dev.type != "cuda":
+            return fn(*args, **kwargs)  # the argument checks reject host tensors
+        stream = kwargs.get("stream")
+        if stream is not None and stream.device != dev:
+            raise ValueError(f"the stream is on {stream.device}, the tensors on {dev}: one CUDA device per call")
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return call
 
 
 def _ptr(t):
@@ -175,6 +220,7 @@ def gdr2_forward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
     return int(lib.gdr2_forward_workspace_bytes(B, T, H, dk, dv, GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
 
 
+@_one_device
 def gdr2_forward(q, k, v, log_alpha, b, w, S0=None, *, final_state=True, save_states=False,
                  out=None, workspace=None, stream=None, out_gate=None, norm_weight=None, norm_eps=1e-6):
     """Chunkwise forward. Returns (o, S_T, saved_states); S_T / saved_states may be None.
@@ -226,6 +272,7 @@ def gdr2_forward_varlen_workspace_bytes(N, T, H, dk, dv, dtype=torch.bfloat16) -
                                                        GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
 
 
+@_one_device
 def gdr2_forward_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, final_state=True, save_states=False,
                         out=None, workspace=None, stream=None, out_gate=None, norm_weight=None, norm_eps=1e-6):
     """Forward over packed sequences. Returns (o, S_T, saved_states).
@@ -285,6 +332,7 @@ def _check_cu_seqlens(cu_seqlens, device):
         raise ValueError("cu_seqlens must be a contiguous 1-D int32 tensor on the inputs' device")
 
 
+@_one_device
 def gdr2_short_conv_silu(x, weight, state=None, *, l2norm=False, eps=1e-6, cu_seqlens=None, final_state=False,
                          state_out=None, out=None, stream=None):
     """Block prologue of one branch: SiLU(causal depthwise convolution of x), then with
@@ -321,6 +369,7 @@ def gdr2_short_conv_silu(x, weight, state=None, *, l2norm=False, eps=1e-6, cu_se
     return y, state_out
 
 
+@_one_device
 def gdr2_gate_activations(a=None, b=None, w=None, *, stream=None):
     """The decay and gate branches' activations, element by element, any of them None:
     log_alpha = -softplus(a) (fp32), sigmoid(b) and sigmoid(w) in the inputs' dtype."""
@@ -342,6 +391,7 @@ def gdr2_gate_activations(a=None, b=None, w=None, *, stream=None):
     return la, bo, wo
 
 
+@_one_device
 def gdr2_block_prologue(xq, xk, xv, conv_q, conv_k, conv_v, a, b, w, *, states=None, eps=1e-6, cu_seqlens=None,
                         final_state=False, stream=None):
     """The whole prologue: q, k = L2(SiLU(conv(x))) per head, v = SiLU(conv(x)), and the
@@ -356,6 +406,7 @@ def gdr2_block_prologue(xq, xk, xv, conv_q, conv_k, conv_v, a, b, w, *, states=N
     return q, k, v, la, bo, wo, ((nq, nk, nv) if final_state else None)
 
 
+@_one_device
 def gdr2_segment_states(A, Bst, S0=None, *, final_state=True, stream=None):
     """States entering the segments of split sequences (see include/gdr2.h).
 
@@ -375,6 +426,7 @@ def gdr2_segment_states(A, Bst, S0=None, *, final_state=True, stream=None):
     return S_starts, S_T
 
 
+@_one_device
 def gdr2_decode_step(q, k, v, log_alpha, b, w, S, *, out=None, stream=None):
     """One decode token; S [N, H, dk, dv] fp32 is updated in place. Returns o [N, H, dv].
 
@@ -405,15 +457,23 @@ def gdr2_backward_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
     return int(lib.gdr2_backward_workspace_bytes(B, T, H, dk, dv, GDR2_BF16 if dtype == torch.bfloat16 else GDR2_F32))
 
 
+@_one_device
 def gdr2_backward(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, saved_states=None, *,
                   want_dS0=True, workspace=None, stream=None):
-    """Gradients of <o, dO> + <S_T, dS_T>. Returns dict dq, dk, dv, dlog_alpha, db, dw, dS0."""
+    """Gradients of <o, dO> + <S_T, dS_T>. Returns dict dq, dk, dv, dlog_alpha, db, dw, dS0.
+
+    b or w shaped [B, T, H] (one value per token-head) are scalar gates; their gradients
+    have the same shape (the tensor-core path: bf16 with dk = dv = 128).
+    """
     lib = load_library()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("b", b, (B, T, H, dk)),
-                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H, dv)), ("dO", dO, (B, T, H, dv))):
+    gates = _gates(b, w, (B, T, H))
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)),
+                         ("b", b, (B, T, H) if gates & GATE_SCALAR_B else (B, T, H, dk)),
+                         ("v", v, (B, T, H, dv)), ("w", w, (B, T, H) if gates & GATE_SCALAR_W else (B, T, H, dv)),
+                         ("dO", dO, (B, T, H, dv))):
         _check(t, name, shp, dt)
     _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32)
     _check(S0, "S0", (B, H, dk, dv), torch.float32)
@@ -427,14 +487,16 @@ def gdr2_backward(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, saved_states
     need = gdr2_backward_workspace_bytes(B, T, H, dk, dv, dt)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-    st = lib.gdr2_backward(B, T, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
-                           _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(saved_states), _ptr(g["dq"]),
-                           _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["db"]), _ptr(g["dw"]),
-                           _ptr(g["dS0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    st = lib.gdr2_backward_gated(B, T, H, dk, dv, _dt(q), gates, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                 _ptr(b), _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(saved_states),
+                                 _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["db"]),
+                                 _ptr(g["dw"]), _ptr(g["dS0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                 _stream(stream))
     _raise(lib, st)
     return g
 
 
+@_one_device
 def gdr2_backward_noalloc(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, saved_states=None, *,
                           want_dS0=True, stream=None):
     """gdr2_backward through the entry point that allocates nothing on the device.

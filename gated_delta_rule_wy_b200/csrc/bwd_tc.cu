@@ -293,6 +293,7 @@ struct VaParams {
     unsigned char *dpa;         // [ntasks][DPA_IMG]
     unsigned char *xrec;        // [ntasks][XREC_BYTES]
     unsigned *status;
+    int wsc;                    // w (and dw) one value per token-head: [B][T][H]
 };
 
 __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant__ CUtensorMap tm_do, VaParams p)
@@ -491,9 +492,9 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
 #pragma unroll
         for (int s = 0; s < 32; ++s) {
             const int t = 32 * colhalf + s;
-            const size_t o = (((size_t)bb * p.T + t0 + t) * p.H + hh) * DV + row;
-            vv[s] = t < Cn ? p.v[o] : __float2bfloat16_rn(0.f);
-            wv[s] = t < Cn ? p.w[o] : __float2bfloat16_rn(0.f);
+            const size_t th = ((size_t)bb * p.T + t0 + t) * p.H + hh;
+            vv[s] = t < Cn ? p.v[th * DV + row] : __float2bfloat16_rn(0.f);
+            wv[s] = t < Cn ? p.w[p.wsc ? th : th * DV + row] : __float2bfloat16_rn(0.f);
         }
         if (!wait_bar(&ms.bar_c, ph_c)) { timed_out = true; break; }
         tc_fence_after_sync();
@@ -506,8 +507,17 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
                 if (t < Cn) {
                     const size_t o = (((size_t)bb * p.T + t0 + t) * p.H + hh) * DV + row;
                     p.gv[o] = __float2bfloat16_rn(dz[s] * __bfloat162float(wv[s]));
-                    p.gw[o] = __float2bfloat16_rn(dz[s] * __bfloat162float(vv[s]));
+                    if (!p.wsc) p.gw[o] = __float2bfloat16_rn(dz[s] * __bfloat162float(vv[s]));
                 }
+            }
+            if (p.wsc) {
+                // a scalar write gate: dw_t = sum_j dz[t][j] v[t][j], this warp's 32 channels first
+                // (lane L ends with token 32 colhalf + L), then the four warp quarters below
+                float dw[32];
+#pragma unroll
+                for (int s = 0; s < 32; ++s) dw[s] = dz[s] * __bfloat162float(vv[s]);
+                transpose_reduce32<32>(dw, lane);
+                ms.red[warp][lane] = dw[0];
             }
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
@@ -518,6 +528,11 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
             }
         }
         mma_sync_point();
+        if (p.wsc && tid < C && tid < Cn) {
+            const int g = tid >> 5, l = tid & 31;
+            const float dw = ms.red[4 * g][l] + ms.red[4 * g + 1][l] + ms.red[4 * g + 2][l] + ms.red[4 * g + 3][l];
+            p.gw[((size_t)bb * p.T + t0 + tid) * p.H + hh] = __float2bfloat16_rn(dw);
+        }
         // ---- dA' = dz U^T (M = 64) ;  X_e = S dz^T ----
         if (tid == 0) {
             const uint32_t ida = idesc_bf16(64, 64, true, true);
@@ -624,6 +639,7 @@ struct KbMisc {
     float gC[DK];                   // G at the chunk's end
     float hsum[2][DK];              // sum of dG over each half-chunk
     float kts[2][DK];               // sum of dk_t (.) k over each half-chunk
+    float red[4][C];                // a scalar erase gate: per-warp-quarter sums of de (.) k per token
 };
 constexpr uint32_t KB_SMEM = KB_MISC + sizeof(KbMisc) + 1024;
 static_assert(offsetof(KbMisc, g0) % 16 == 0 && offsetof(KbMisc, g1) % 16 == 0, "float4 reads of the references");
@@ -638,6 +654,8 @@ struct KbParams {
     const unsigned char *dpa;
     const unsigned char *xrec;
     unsigned *status;
+    const __nv_bfloat16 *bsc;  // b one value per token-head [B][T][H] (its tile map unused), or null
+    __nv_bfloat16 *gbsc;       // db for such a b, [B][T][H]
 };
 
 // element (row, col) of a 128-row, 64-column bf16 image
@@ -676,13 +694,14 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tm = ms.tmem_base;
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
 
+    const bool bsc = p.bsc != nullptr;
     auto issue_loads = [&](int task) {
         const int bhh = task / p.NC, n = task % p.NC;
         const int bb = bhh / p.H, hh = bhh % p.H;
-        mbar_arrive_expect_tx(&ms.bar_ld, KB_TX);
+        mbar_arrive_expect_tx(&ms.bar_ld, KB_TX - (bsc ? 16384u : 0u));
         tma_load_4d(sm + KB_Q, &tm_q, &ms.bar_ld, 0, hh, n * C, bb);
         tma_load_4d(sm + KB_K, &tm_k, &ms.bar_ld, 0, hh, n * C, bb);
-        tma_load_4d(sm + KB_B, &tm_b, &ms.bar_ld, 0, hh, n * C, bb);
+        if (!bsc) tma_load_4d(sm + KB_B, &tm_b, &ms.bar_ld, 0, hh, n * C, bb);
         tma_load_4d(sm + KB_LA, &tm_la, &ms.bar_ld, 0, hh, n * C, bb);
         bulk_load(sm + KB_DPA, p.dpa + (size_t)task * DPA_IMG, DPA_IMG, &ms.bar_ld);
         bulk_load(sm + KB_X, p.xrec + (size_t)task * XREC_BYTES, XREC_BYTES, &ms.bar_ld);
@@ -702,12 +721,34 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
         const int bhh = task / p.NC, n = task % p.NC;
         const int bb = bhh / p.H, hh = bhh % p.H;
+        const int t0 = n * C, Cn = min(C, p.T - t0);
+        // a scalar erase gate: this thread's four rows (t = tid / 16 + 16 k), read while the copies land
+        __nv_bfloat16 gb4[4];
+        if (bsc) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = (tid >> 4) + 16 * k;
+                gb4[k] = t < Cn ? p.bsc[((size_t)bb * p.T + t0 + t) * p.H + hh] : __float2bfloat16_rn(0.f);
+            }
+        }
         {
             const bool ok = mbar_wait_bounded(&ms.bar_ld, ph_ld, kWaitLimitNs);
             if (__syncthreads_or(!ok)) { timed_out = true; break; }
             ph_ld ^= 1u;
         }
         loads_pending = false;
+        if (bsc) {
+            // its rows of the b tile hold that value in every channel (first read after the
+            // barrier that ends the decay scan below)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = (tid >> 4) + 16 * k;
+                const __nv_bfloat162 g2 = __halves2bfloat162(gb4[k], gb4[k]);
+                uint4 u;
+                u.x = u.y = u.z = u.w = *reinterpret_cast<const uint32_t *>(&g2);
+                *reinterpret_cast<uint4 *>(sm + KB_B + t * 256 + (tid & 15) * 16) = u;
+            }
+        }
         // ================= prep: cumulative decay, references, decay-weighted operands =================
         float G[4][8];
 #pragma unroll
@@ -873,12 +914,23 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float dpt = dpd[t];
                 oq[t * DK + c] = __float2bfloat16_rn(fmaf(dpt, kf, dq));
                 ok_[t * DK + c] = __float2bfloat16_rn(dkAP + dpt * qf + dkt + de * bf_);
-                ob[t * DK + c] = __float2bfloat16_rn(de * kf);
+                if (!bsc) {
+                    ob[t * DK + c] = __float2bfloat16_rn(de * kf);
+                } else {
+                    // db_t = sum_c de[t][c] k[t][c]: this warp's 32 channels here, the quarters below
+                    float x = de * kf;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                    if (lane == 0) ms.red[quarter][t] = x;
+                }
             }
         }
         ms.hsum[hf][c] = hs;
         ms.kts[hf][c] = kts;
         __syncthreads();  // every read of G (the exact path reads the other half's) is done
+        if (bsc && tid < Cn)
+            p.gbsc[((size_t)bb * p.T + t0 + tid) * p.H + hh] =
+                __float2bfloat16_rn(ms.red[0][tid] + ms.red[1][tid] + ms.red[2][tid] + ms.red[3][tid]);
         // dlog_alpha[t] = sum_{t' >= t} dG[t'] + sum_j dS' (.) S e^{G_C} + sum_{t' < t} dk~ (.) k~:
         // the last sum as a prefix (as total minus suffix it cancels: the last token's term is
         // O(1) while under strong decay every other term, and the result, are near e^-32)
@@ -906,7 +958,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (tid == 0) {
             tma_store_4d(&tm_gq, sm + KB_STACK, 0, hh, n * C, bb);
             tma_store_4d(&tm_gk, sm + KB_STACK + 16384, 0, hh, n * C, bb);
-            tma_store_4d(&tm_gb, sm + KB_R, 0, hh, n * C, bb);
+            if (!bsc) tma_store_4d(&tm_gb, sm + KB_R, 0, hh, n * C, bb);
             tma_store_4d(&tm_gla, sm + KB_LA, 0, hh, n * C, bb);
             bulk_commit_group();
             if (task + (int)gridDim.x < ntasks) {
@@ -982,7 +1034,7 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     fa.workspace_bytes = L.ext;
     fa.status = a.status;
     fa.cu_seqlens = nullptr;
-    fa.gates = 0;
+    fa.gates = a.gates;
     fa.out_gate = nullptr;
     fa.norm_weight = nullptr;
     fa.norm_eps = 0.f;
@@ -991,13 +1043,20 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     cudaError_t e = launch_forward_tc(fa, s);
     if (e != cudaSuccess) return e;
 
+    const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
     CUtensorMap mdo, mq, mk, mb, mla, mgq, mgk, mgb, mgla;
     if (!make_map(&mdo, a.dO, false, a.B, a.T, a.H, DV, 64, true) ||
         !make_map(&mq, a.q, false, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, false, a.B, a.T, a.H, DK) ||
-        !make_map(&mb, a.b, false, a.B, a.T, a.H, DK) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK) ||
-        !make_map(&mgq, a.gq, false, a.B, a.T, a.H, DK) || !make_map(&mgk, a.gk, false, a.B, a.T, a.H, DK) ||
-        !make_map(&mgb, a.gb, false, a.B, a.T, a.H, DK) || !make_map(&mgla, a.glog_alpha, true, a.B, a.T, a.H, DK))
+        !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK) || !make_map(&mgq, a.gq, false, a.B, a.T, a.H, DK) ||
+        !make_map(&mgk, a.gk, false, a.B, a.T, a.H, DK) || !make_map(&mgla, a.glog_alpha, true, a.B, a.T, a.H, DK))
         return cudaErrorInvalidValue;
+    // a scalar erase gate has no tiles to copy: the q and dq maps stand in, unused
+    if (bsc) {
+        mb = mq;
+        mgb = mgq;
+    } else if (!make_map(&mb, a.b, false, a.B, a.T, a.H, DK) || !make_map(&mgb, a.gb, false, a.B, a.T, a.H, DK)) {
+        return cudaErrorInvalidValue;
+    }
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const int grid = ntasks < nsm ? ntasks : nsm;
@@ -1016,7 +1075,7 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     VaParams vp{a.B, a.T, a.H, NC, ntasks, ws, ws + L.ext, ws + L.dsc, states,
                 static_cast<const __nv_bfloat16 *>(a.v), static_cast<const __nv_bfloat16 *>(a.w),
                 static_cast<__nv_bfloat16 *>(a.gv), static_cast<__nv_bfloat16 *>(a.gw), ws + L.dpa, ws + L.xrec,
-                a.status};
+                a.status, wsc ? 1 : 0};
     bwd_value_kernel<<<grid, 256, VA_SMEM, s>>>(mdo, vp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1024,7 +1083,10 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     // 4. key side
     e = cudaFuncSetAttribute(bwd_key_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KB_SMEM);
     if (e != cudaSuccess) return e;
-    KbParams kp{a.B, a.T, a.H, NC, ntasks, ws + L.dpa, ws + L.xrec, a.status};
+    KbParams kp{a.B,      a.T,         a.H,      NC,
+                ntasks,   ws + L.dpa,  ws + L.xrec, a.status,
+                bsc ? static_cast<const __nv_bfloat16 *>(a.b) : nullptr,
+                bsc ? static_cast<__nv_bfloat16 *>(a.gb) : nullptr};
     bwd_key_kernel<<<grid, 256, KB_SMEM, s>>>(mq, mk, mb, mla, mgq, mgk, mgb, mgla, kp);
     return cudaGetLastError();
 }

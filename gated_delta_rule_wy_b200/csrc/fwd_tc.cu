@@ -125,6 +125,7 @@ struct ChunkParams {
     int gates;              // kGate* bits: a scalar gate is read here, not by the copy engine
     const __nv_bfloat16 *bg, *wg;
     unsigned char *ext;     // backward: T and W of every task (EXT_BYTES each), else null
+    int debug_giveup;       // test hook: give up a 1 us wait before the first copy
 };
 
 // Where a task's chunk lives: tensor-map coordinates (token t0, sequence bb), head h, and the
@@ -205,7 +206,7 @@ constexpr uint32_t CK_M = 0, CK_U = 128, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384,
 constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W_0, W_1 once those are read
 
 // GENERAL: packed sequences and/or scalar gates may be in use; the other instantiation is
-// the dense, vector-gate kernel with those branches compiled away. BWD (dense, vector gates):
+// the dense, vector-gate kernel with those branches compiled away. BWD (dense sequences):
 // T and W of each task also go to p.ext for the backward.
 template <bool GENERAL, bool BWD = false>
 __global__ void __launch_bounds__(NT, 1)
@@ -251,13 +252,19 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wsc) tma_load_4d(sm + OFF_STG_W, &tm_w, &ms.bar_tma, 0, L.h, L.t0, L.bb);
         tma_load_4d(sm + OFF_STG_LA, &tm_la, &ms.bar_tma, 0, L.h, L.t0, L.bb);
     };
-    if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
+    bool timed_out = false;
+    if (p.debug_giveup) {
+        // test hook: nothing has been issued yet and nothing arrives on bar_mma, so this
+        // bounded wait runs out and the CTA takes its give-up path below
+        const bool ok = mbar_wait_bounded(&ms.bar_mma, 0, 1000);
+        timed_out = __syncthreads_or(!ok) != 0;
+    }
+    if (!timed_out && tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
     // the scan kernel may be scheduled now: its CTAs take an SM only once this (persistent) CTA
     // has left it, and they read the workspace only after this whole grid has completed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     uint32_t ph_tma = 0, ph_mma = 0;
-    bool timed_out = false;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
         const bool ok = mbar_wait_bounded(bar, ph, kWaitLimitNs);
         ph ^= 1u;
@@ -1271,6 +1278,21 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
 // ---------------------------------------------------------------- host side
 }  // namespace
 
+namespace {
+__global__ void recip_eval_kernel(const float *x, float *y, long long n)
+{
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        y[i] = recip_newton2(x[i]);
+}
+}  // namespace
+
+cudaError_t launch_recip_eval(const float *x, float *y, long long n, cudaStream_t s)
+{
+    const long long blocks = (n + 255) / 256;
+    recip_eval_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, s>>>(x, y, n);
+    return cudaGetLastError();
+}
+
 bool forward_tc_supported(const FwdArgs &a)
 {
     return a.bf16 && a.dk == DK && a.dv == DV && a.T > 0 && encode_fn() != nullptr;
@@ -1308,10 +1330,11 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     if (!a.out_gate) mg = mo; else if (!make_map(&mg, a.out_gate, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
     const bool general = varlen || bsc || wsc;
     const bool bwd = a.bwd_ext != nullptr;
-    if (bwd && general) return cudaErrorInvalidValue;
+    if (bwd && varlen) return cudaErrorInvalidValue;
     void (*chunk)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                   const CUtensorMap, ChunkParams) =
-        general ? fwd_chunk_kernel<true> : bwd ? fwd_chunk_kernel<false, true> : fwd_chunk_kernel<false>;
+        general ? (bwd ? fwd_chunk_kernel<true, true> : fwd_chunk_kernel<true>)
+                : (bwd ? fwd_chunk_kernel<false, true> : fwd_chunk_kernel<false>);
     cudaError_t e = cudaFuncSetAttribute(chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int epi = (a.norm_weight ? kEpiNorm : 0) | (a.out_gate ? kEpiGate : 0);
@@ -1336,7 +1359,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     ChunkParams cp{a.B,         a.T,       a.H,        NC,
                    ntasks,      ws,        a.status,   a.cu_seqlens,
                    cu_chunks,   ntasks_dev, a.gates,   static_cast<const __nv_bfloat16 *>(a.b),
-                   static_cast<const __nv_bfloat16 *>(a.w), a.bwd_ext};
+                   static_cast<const __nv_bfloat16 *>(a.w), a.bwd_ext, debug_giveup_flag()};
     const int grid = ntasks < nsm ? ntasks : nsm;
     chunk<<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
     e = cudaGetLastError();

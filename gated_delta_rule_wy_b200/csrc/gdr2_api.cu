@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/gdr2.h"
@@ -31,17 +32,22 @@ __device__ unsigned g_status_word;
 
 constexpr int kMaxDevices = 64;
 unsigned *g_status_ptr[kMaxDevices];
-std::once_flag g_status_once[kMaxDevices];
 
+std::mutex g_status_mu;
+
+// The status word's device address on `dev` (current). Only a successful lookup is kept.
 unsigned *status_ptr(int dev)
 {
     if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::call_once(g_status_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) g_status_ptr[dev] = static_cast<unsigned *>(p);
-    });
+    }
     return g_status_ptr[dev];
 }
+
+std::atomic<int> g_debug_giveup{0};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -114,9 +120,23 @@ gdr2_status launched(cudaError_t e, const char *what)
 
 }  // namespace
 
+namespace gdr2 {
+int debug_giveup_flag() { return g_debug_giveup.load(); }
+}  // namespace gdr2
+
 extern "C" {
 
 int gdr2_abi_version(void) { return GDR2_ABI_VERSION; }
+
+void gdr2_debug_force_timeout(int enable) { g_debug_giveup.store(enable != 0 ? 1 : 0); }
+
+gdr2_status gdr2_debug_recip(const float *x, float *y, long long n, void *stream)
+{
+    if (n < 0) return fail(GDR2_ERR_INVALID_ARG, "n must not be negative (n=%lld)", n);
+    if (n == 0) return GDR2_OK;
+    if (!x || !y) return fail(GDR2_ERR_INVALID_ARG, "x and y must not be NULL");
+    return launched(gdr2::launch_recip_eval(x, y, n, static_cast<cudaStream_t>(stream)), "gdr2_debug_recip");
+}
 
 const char *gdr2_last_error(void) { return g_last_error; }
 
@@ -364,18 +384,25 @@ size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_d
     return gdr2::backward_workspace_bytes(B, T, H, dk, dv, dt == GDR2_BF16);
 }
 
-gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
-                          const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
-                          const void *dO, const float *dS_T, const float *saved_states, void *dq, void *dk_,
-                          void *dv_, float *dlog_alpha, void *db, void *dw, float *dS0, void *workspace,
-                          size_t workspace_bytes, void *stream)
+gdr2_status gdr2_backward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates, const void *q,
+                                const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                                const float *S0, const void *dO, const float *dS_T, const float *saved_states,
+                                void *dq, void *dk_, void *dv_, float *dlog_alpha, void *db, void *dw, float *dS0,
+                                void *workspace, size_t workspace_bytes, void *stream)
 {
     GDR2_TRY(check_dims(B, T, H, dk, dv));
     GDR2_TRY(check_dtype(dt));
+    GDR2_TRY(check_gates(gates));
+    if (gates && !(dt == GDR2_BF16 && dk == 128 && dv == 128))
+        return fail(GDR2_ERR_UNSUPPORTED, "scalar gates in the backward need bf16 inputs with dk = dv = 128");
     const bool has_tokens = (long long)B * T * H > 0;
-    const char *names[] = {"q", "k", "v", "log_alpha", "b", "w", "dO", "dq", "dk", "dv", "dlog_alpha", "db", "dw"};
-    const void *ptrs[] = {q, k, v, log_alpha, b, w, dO, dq, dk_, dv_, dlog_alpha, db, dw};
-    for (int i = 0; i < 13; ++i) GDR2_TRY(check_ptr(ptrs[i], names[i], !has_tokens));
+    const char *names[] = {"q", "k", "v", "log_alpha", "dO", "dq", "dk", "dv", "dlog_alpha"};
+    const void *ptrs[] = {q, k, v, log_alpha, dO, dq, dk_, dv_, dlog_alpha};
+    for (int i = 0; i < 9; ++i) GDR2_TRY(check_ptr(ptrs[i], names[i], !has_tokens));
+    GDR2_TRY(check_gate_ptr(b, "b", !has_tokens, gates & GDR2_GATE_SCALAR_B, dt));
+    GDR2_TRY(check_gate_ptr(db, "db", !has_tokens, gates & GDR2_GATE_SCALAR_B, dt));
+    GDR2_TRY(check_gate_ptr(w, "w", !has_tokens, gates & GDR2_GATE_SCALAR_W, dt));
+    GDR2_TRY(check_gate_ptr(dw, "dw", !has_tokens, gates & GDR2_GATE_SCALAR_W, dt));
     GDR2_TRY(check_ptr(S0, "S0", true));
     GDR2_TRY(check_ptr(dS_T, "dS_T", true));
     GDR2_TRY(check_ptr(saved_states, "saved_states", true));
@@ -397,9 +424,21 @@ gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, co
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(GDR2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
     gdr2::BwdArgs a{B, T, H, dk, dv, dt == GDR2_BF16, q, k, v, log_alpha, b, w, S0, dO, dS_T, saved_states,
-                    dq, dk_, dv_, dlog_alpha, db, dw, dS0, workspace, workspace_bytes, nullptr};
+                    dq, dk_, dv_, dlog_alpha, db, dw, dS0, workspace, workspace_bytes, nullptr, gates};
     GDR2_TRY(device_status(&a.status));
+    if (gates && !gdr2::backward_tc_supported(a))
+        return fail(GDR2_ERR_UNSUPPORTED, "scalar gates in the backward need the tensor-core path (no driver entry)");
     return launched(gdr2::launch_backward(a, s), "gdr2_backward");
+}
+
+gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,
+                          const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                          const void *dO, const float *dS_T, const float *saved_states, void *dq, void *dk_,
+                          void *dv_, float *dlog_alpha, void *db, void *dw, float *dS0, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    return gdr2_backward_gated(B, T, H, dk, dv, dt, 0, q, k, v, log_alpha, b, w, S0, dO, dS_T, saved_states, dq,
+                               dk_, dv_, dlog_alpha, db, dw, dS0, workspace, workspace_bytes, stream);
 }
 
 gdr2_status gdr2_backward_noalloc(int B, int T, int H, int dk, int dv, gdr2_dtype dt, const void *q, const void *k,

@@ -61,6 +61,7 @@ struct BwdArgs {
     void *workspace;
     size_t workspace_bytes;
     unsigned *status;
+    int gates = 0;  // kGate* bits: b (and db) and/or w (and dw) one value per token-head
 };
 
 // Block prologue (csrc/prologue.cu).
@@ -96,6 +97,8 @@ struct SegArgs {
 };
 
 cudaError_t launch_segment_states(const SegArgs &a, cudaStream_t s);
+int debug_giveup_flag();  // gdr2_debug_force_timeout's setting
+cudaError_t launch_recip_eval(const float *x, float *y, long long n, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t s);
 cudaError_t launch_gate_activations(const ActArgs &a, cudaStream_t s);
 cudaError_t launch_forward_simt(const FwdArgs &a, cudaStream_t s);

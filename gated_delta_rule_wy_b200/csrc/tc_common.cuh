@@ -66,11 +66,15 @@ __device__ __forceinline__ void store8f(float *p, const float (&f)[8])
     *reinterpret_cast<float4 *>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
 }
 
-// 1 / d for 2^-126 <= d < 2^126 (normal, positive). Seed: the bit pattern of a float is close to 2^23 (log2 d + 127),
-// so subtracting it from a constant negates log2 d: one integer operation gives 1 / d to
-// within 5.1% in every binade (the constant minimises that error over one binade). Two
-// Newton steps r <- r + r (1 - d r), each squaring the relative error, leave 6.6e-6.
-// All of it on the FMA and integer pipes: the special-function unit is the scarce one.
+// 1 / d for normal 2^-126 <= d < 2^125, relative error at most 6.6e-6. The method: the
+// bit pattern of a positive float is close to 2^23 (log2 d + 127), so subtracting it from
+// a constant negates log2 d and one integer operation gives a seed for 1 / d (the
+// integer-arithmetic approximations of J. Blinn, "Floating-point tricks", IEEE Computer
+// Graphics and Applications 17(4), 1997). The constant 0x7EF311C2 makes the seed's relative
+// error equioscillate at +-5.051% over a binade, hence in every binade. Two Newton-Raphson
+// steps r <- r + r (1 - d r), each squaring the relative error, leave 6.6e-6. (At d >= 2^125
+// the seed is subnormal and the bound fails; the callers stay below e^80 < 2^116.) All of it
+// on the FMA and integer pipes: the special-function unit is the scarce one.
 __device__ __forceinline__ float recip_newton2(float d)
 {
     float r = __int_as_float(0x7EF311C2 - __float_as_int(d));

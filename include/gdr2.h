@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 7
+#define GDR2_ABI_VERSION 8
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -298,10 +298,15 @@ size_t gdr2_backward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_d
  * out: dq, dk_, db [B,T,H,dk] dt; dv_, dw [B,T,H,dv] dt;
  *      dlog_alpha [B,T,H,dk] fp32; dS0 [B,H,dk,dv] fp32 or NULL.
  * scratch: workspace of at least gdr2_backward_workspace_bytes(...) bytes,
- *      256-byte aligned; its contents on entry do not matter (the call clears
- *      the part it accumulates into, on `stream`).
- * The per-key-channel gradients (dq, dk, db, dlog_alpha) are summed over the
- * value columns with fp32 atomics, so their last bits may differ between calls.
+ *      256-byte aligned; its contents on entry do not matter.
+ * Paths: bf16 inputs with dk = dv = 128 run the chunkwise tensor-core backward
+ *      (the forward's chunk kernel again, a reverse scan of the state gradient
+ *      over the chunks, then the chunk gradients of every chunk in parallel;
+ *      deterministic, bf16 tensor-core operands with fp32 accumulation and an
+ *      fp32 state gradient). Other inputs run a token-level kernel in fp32,
+ *      whose per-key-channel gradients (dq, dk, db, dlog_alpha) are summed over
+ *      the value columns with fp32 atomics, so their last bits may differ
+ *      between calls.
  */
 gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
                           const void *q, const void *k, const void *v,
@@ -311,6 +316,25 @@ gdr2_status gdr2_backward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
                           void *dq, void *dk_, void *dv_, float *dlog_alpha,
                           void *db, void *dw, float *dS0,
                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdr2_backward_gated -- gdr2_backward with the gate layouts of `gates`
+ * (GDR2_GATE_* bits): a scalar gate b or w is [B, T, H] in the dtype dt (one
+ * value per token-head, the scalar-erase and scalar-write ablations of the
+ * note's sec. 4; both scalar and equal are the KDA and Gated DeltaNet gates of
+ * sec. 2), and its gradient db or dw has the same layout: the sum over the
+ * channels of the vector gate's gradient. Everything else as gdr2_backward;
+ * gates = 0 is gdr2_backward. Scalar gates need bf16 inputs with
+ * dk = dv = 128 (GDR2_ERR_UNSUPPORTED otherwise).
+ */
+gdr2_status gdr2_backward_gated(int B, int T, int H, int dk, int dv, gdr2_dtype dt, int gates,
+                                const void *q, const void *k, const void *v,
+                                const float *log_alpha, const void *b, const void *w,
+                                const float *S0, const void *dO, const float *dS_T,
+                                const float *saved_states,
+                                void *dq, void *dk_, void *dv_, float *dlog_alpha,
+                                void *db, void *dw, float *dS0,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /* Size of the device scratch array behind gdr2_backward_noalloc (64 MiB). */
 #define GDR2_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
@@ -355,6 +379,29 @@ gdr2_status gdr2_backward_noalloc(int B, int T, int H, int dk, int dv, gdr2_dtyp
  * error, GDR2_OK otherwise.
  */
 gdr2_status gdr2_sync_status(void *stream);
+
+/*
+ * Test hooks. Neither has a counterpart in the paper; they exist so that
+ * tests can reach code that normal inputs never run.
+ *
+ * gdr2_debug_force_timeout -- while `enable` is nonzero, the chunk kernel of
+ * every tensor-core forward launch (also the one inside gdr2_backward) first
+ * waits, with a 1 us limit, on an mbarrier that nothing arrives on, before it
+ * issues any copy or MMA. The wait runs out and the kernel takes its normal
+ * give-up path: it frees its tensor memory, records the timeout in the device
+ * status word and returns. The call's outputs are then undefined, and the next
+ * gdr2_sync_status returns GDR2_ERR_TIMEOUT. The setting is process-wide;
+ * concurrent callers see it too. 0 (the default) turns it off.
+ */
+void gdr2_debug_force_timeout(int enable);
+
+/*
+ * gdr2_debug_recip -- y[i] = the device reciprocal the kernels use in place of
+ * 1 / x[i] for positive normal x below 2^125 (a bit-pattern seed and two
+ * Newton steps, relative error at most 6.6e-6). x and y are device arrays of
+ * n floats; asynchronous on `stream`. INVALID_ARG for a NULL pointer or n < 0.
+ */
+gdr2_status gdr2_debug_recip(const float *x, float *y, long long n, void *stream);
 
 #ifdef __cplusplus
 }

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 7
+    assert lib.gdr2_abi_version() == 8
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -250,3 +250,20 @@ def test_new_binding_functions_validate_before_calling():
         g.gdr2_segment_states(torch.zeros(1, 2, 2, 64, 64), torch.zeros(1, 2, 2, 64, 64))
     with pytest.raises(ValueError, match="CUDA"):
         g.gdr2_gate_activations(torch.zeros(16))
+
+
+def test_binding_rejects_tensors_on_several_devices():
+    """Every tensor of a call and its stream must be on one device: the library launches on
+    the current device, so a tensor elsewhere would reach a kernel as a foreign pointer."""
+    import torch
+
+    from gated_delta_rule_wy_b200.binding import _device_of
+
+    host, meta = torch.zeros(1, 4, 1, 64), torch.zeros(1, 4, 1, 64, device="meta")
+    with pytest.raises(ValueError, match="one CUDA device"):
+        _device_of([host, meta])
+    with pytest.raises(ValueError, match="one CUDA device"):
+        g.gdr2_forward(host, host, meta, host, host, host)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        g.gdr2_backward(host, host, host, host, host, host, meta)
+    assert _device_of([host, host]) == torch.device("cpu")

@@ -99,3 +99,56 @@ def test_kda_gates_match_the_oracle():
     o_ref, S_ref = oracle.forward(n["q"], n["k"], n["v"], n["log_alpha"], bv, bv, S0=n["S0"])
     assert_close(o, o_ref, TOL[torch.bfloat16], "KDA gates: o")
     assert_close(S_T, S_ref, TOL[torch.bfloat16], "KDA gates: S_T")
+
+
+def _oracle_backward(x, b_vec, w_vec, dO, dST):
+    n = x.as_numpy64()
+    return oracle.backward(n["q"], n["k"], n["v"], n["log_alpha"], b_vec, w_vec, dO.double().numpy(), S0=n["S0"],
+                           dS_T=None if dST is None else dST.double().numpy())
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("shape", [(2, 16, 256, False), (1, 3, 150, True)])
+def test_backward_scalar_gates_match_the_oracle(mode, shape):
+    """Scalar erase and/or write gates through the tensor-core backward (the first shape is
+    the T = 256 slice of the backward workload, the second a ragged one with S0 and dS_T):
+    each gradient against the oracle's for the broadcast vector gates, a scalar gate's
+    gradient against the sum of the vector gradient over its channels; the other
+    gradients equal those of the broadcast-vector call."""
+    from gated_delta_rule_wy_b200 import gdr2_backward
+
+    B, H, T, with_state = shape
+    sb_on, sw_on = MODES[mode]
+    x = I.make_forward_inputs(B=B, H=H, T=T, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=2.0, seed=89,
+                              with_S0=with_state)
+    sb, sw = _scalar_gates((B, T, H), torch.bfloat16, 90)
+    dO = I.make_upstream_grad(B, T, H, 128, 91, dtype=torch.bfloat16)
+    dST = torch.randn((B, H, 128, 128), generator=torch.Generator().manual_seed(92)) if with_state else None
+    bv = _vec(sb, 128) if sb_on else x.b
+    wv = _vec(sw, 128) if sw_on else x.w
+    d_ = x.to("cuda")
+    dev = lambda t: None if t is None else t.cuda()  # noqa: E731
+    g = gdr2_backward(d_.q, d_.k, d_.v, d_.log_alpha, dev(sb if sb_on else x.b), dev(sw if sw_on else x.w),
+                      dO.cuda(), d_.S0, dev(dST))
+    gv = gdr2_backward(d_.q, d_.k, d_.v, d_.log_alpha, bv.cuda(), wv.cuda(), dO.cuda(), d_.S0, dev(dST))
+    gdr2_sync_status()
+    assert g["db"].shape == ((B, T, H) if sb_on else (B, T, H, 128))
+    assert g["dw"].shape == ((B, T, H) if sw_on else (B, T, H, 128))
+    ref = _oracle_backward(x, bv.double().numpy(), wv.double().numpy(), dO, dST)
+    for name in ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0"):
+        r = ref[name]
+        if (name == "db" and sb_on) or (name == "dw" and sw_on):
+            r = r.sum(axis=-1)
+        assert_close(g[name], r, TOL[torch.bfloat16], f"{mode} {shape}: {name}")
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dS0"):
+        assert torch.equal(g[name], gv[name]), f"{mode} {shape}: {name} differs from the broadcast-vector call"
+
+
+def test_backward_scalar_gates_need_the_tensor_core_path():
+    from gated_delta_rule_wy_b200 import binding, gdr2_backward
+
+    x = I.make_forward_inputs(B=1, H=2, T=70, dk=64, dv=64, dtype=torch.float32, seed=93).to("cuda")
+    sb, _ = _scalar_gates((1, 70, 2), torch.float32, 94)
+    dO = I.make_upstream_grad(1, 70, 2, 64, 95).cuda()
+    with pytest.raises(binding.GDR2Error, match="UNSUPPORTED"):
+        gdr2_backward(x.q, x.k, x.v, x.log_alpha, sb.cuda(), x.w, dO)
