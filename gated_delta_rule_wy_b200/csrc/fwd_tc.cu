@@ -75,7 +75,7 @@ constexpr uint32_t OFF_STG_K = 16384;   // k
 constexpr uint32_t OFF_STG_B = 32768;   // b
 constexpr uint32_t OFF_STG_V = 49152;   // v; exact path: A (fp32 [64][68]) over V and W
 constexpr uint32_t OFF_STG_W = 65536;   // w
-constexpr uint32_t OFF_STG_LA = 81920;  // log_alpha [64][128] fp32; then per-channel references; exact path: G
+constexpr uint32_t OFF_STG_LA = 81920;  // log_alpha [64][128] fp32; then G
 constexpr uint32_t OFF_STACK = 114688;  // [L^e_0; L^q_0; L^e_1; L^q_1] 128 x 128; later W as [c][64 t]
 constexpr uint32_t OFF_R0 = 147456;     // [R_0; R_1] (32 + 64 rows) x 128 as one B operand (24 KB); then
                                         // A and T (fp32 [64][68]) with the block-product scratch, then
@@ -84,7 +84,7 @@ constexpr uint32_t OFF_R0 = 147456;     // [R_0; R_1] (32 + 64 rows) x 128 as on
 constexpr uint32_t OFF_Z = 172032;      // Z 64 x 128 (value side); later U~^T as [j][64 t] for the slot
 constexpr uint32_t OFF_QH = 188416;     // Q^ = Q (.) exp G, [t rows][128 c] (K-major chunks)
 constexpr uint32_t OFF_KT = 204800;     // K (.) exp(G_C - G), 64 x 128
-constexpr uint32_t OFF_P = 221184;      // prefix-scan scratch during prep; then P 64 x 64
+constexpr uint32_t OFF_P = 221184;      // per-channel references during prep; then P 64 x 64
 constexpr uint32_t OFF_MISC = 229376;   // barriers, per-channel vectors
 constexpr uint32_t MISC_BYTES = 1664;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
@@ -345,55 +345,45 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
         // ================= prep: cumulative decay and decay-weighted operands =================
         // Rows beyond T are zero-filled by TMA (per-sequence extent): padded tokens are inert.
-        float G[4][8];
-        float *scan = reinterpret_cast<float *>(sm + OFF_P);       // [16 groups][128]
-        float *refs = reinterpret_cast<float *>(sm + OFF_STG_LA);  // g0, g1, gC after the scan
+        // Thread (key channel c, half-chunk hc) sums its channel over its 32 tokens in
+        // registers; the second half adds the first half's total. G replaces log_alpha in
+        // shared memory (each thread overwrites only what it read).
+        float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
+        float *refs = reinterpret_cast<float *>(sm + OFF_P);  // g0, g1, G_C, first-half totals (until P)
         {
-            const float *la_s = reinterpret_cast<const float *>(sm + OFF_STG_LA);
+            const int c = tid & (DK - 1), hc = tid >> 7;
+            float g[32];
+            float run = 0.f;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                float la[8];
-                load8f(la_s + (tg * 4 + m) * DK + o8 * 8, la);
-#pragma unroll
-                for (int x = 0; x < 8; ++x) G[m][x] = (m == 0 ? 0.f : G[m - 1][x]) + clamp_log_alpha(la[x]);
+            for (int i = 0; i < 32; ++i) {
+                run += clamp_log_alpha(Gs[(32 * hc + i) * DK + c]);
+                g[i] = run;
             }
-            store8f(scan + tg * DK + o8 * 8, G[3]);
-        }
-        __syncthreads();
-        if (tid < DK) {
-            // exclusive prefix over the 16 token groups of channel c
-            const int c = tid;
-            float run = 0.f, g0 = 0.f, g1 = 0.f;
+            if (hc == 0) refs[3 * DK + c] = run;  // G at token 31
+            __syncthreads();
+            const float off = hc ? refs[3 * DK + c] : 0.f;
 #pragma unroll
-            for (int g = 0; g < 16; ++g) {
-                if (g == 4) g0 = run;   // G at token 15
-                if (g == 12) g1 = run;  // G at token 47
-                const float v = scan[g * DK + c];
-                scan[g * DK + c] = run;
-                run += v;
+            for (int i = 0; i < 32; ++i) Gs[(32 * hc + i) * DK + c] = g[i] + off;
+            if (hc == 0) {
+                refs[c] = g[15];  // G at token 15: reference of half-chunk 0
+                ms.eg0[c] = __expf(g[15]);
+            } else {
+                refs[DK + c] = g[15] + off;       // G at token 47: reference of half-chunk 1
+                refs[2 * DK + c] = g[31] + off;   // G_C
+                ms.eg1[c] = __expf(g[15] + off);
+                ms.gC[c] = __expf(g[31] + off);
             }
-            refs[c] = g0;
-            refs[DK + c] = g1;
-            refs[2 * DK + c] = run;  // G_C
-            ms.gC[c] = __expf(run);
-            ms.eg0[c] = __expf(g0);
-            ms.eg1[c] = __expf(g1);
         }
         if (tid == 0) bulk_wait_group_read0();  // ... and [Q'; M] too, before the operands are rebuilt
         __syncthreads();
         bool risky = false;
+        float G[4][8];
         float g0[8], g1[8], gC[8];
         load8f(refs + o8 * 8, g0);
         load8f(refs + DK + o8 * 8, g1);
         load8f(refs + 2 * DK + o8 * 8, gC);
-        {
-            float ex[8];
-            load8f(scan + tg * DK + o8 * 8, ex);
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) G[m][x] += ex[x];
-        }
+        for (int m = 0; m < 4; ++m) load8f(Gs + (tg * 4 + m) * DK + o8 * 8, G[m]);
         {
             const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_Q);
             const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
@@ -461,11 +451,7 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         const bool exact = __syncthreads_or(risky) != 0;
         if (exact) {
-            // ---- exact path: G to shared memory, pairwise exponentials ----
-            float *Gs = reinterpret_cast<float *>(sm + OFF_STG_LA);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) store8f(Gs + (tg * 4 + m) * DK + o8 * 8, G[m]);
-            __syncthreads();
+            // ---- exact path: pairwise exponentials (G is in shared memory already) ----
             const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_Q);
             const __nv_bfloat16 *ks = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_K);
             const __nv_bfloat16 *bs = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG_B);
