@@ -941,10 +941,6 @@ constexpr uint32_t SC_SLOT0 = 0;
 constexpr uint32_t SC_SLOT1 = SLOT_BYTES;          // 90112, 1024-aligned
 constexpr uint32_t SC_O = 2 * SLOT_BYTES;          // O tile [64 t][128 j] bf16
 constexpr uint32_t SC_MISC = SC_O + 16384;
-constexpr uint32_t SC_EPI = SC_MISC + 1280;        // output norm: per-warp sums [4][64], then 1/rms [64]
-constexpr uint32_t SC_G = SC_MISC + 4096;          // output gate tile [64 t][128 j] bf16 (1024-aligned)
-static_assert(SC_EPI + 1280 <= SC_G, "norm scratch overlaps the gate tile");
-static_assert(SC_G % 1024 == 0, "gate tile alignment");
 constexpr int SC_NT = NT + 32;  // 8 warps on the TMEM lanes + warp 8, which issues the MMAs
 constexpr uint32_t SC_REG = 256;                    // region r at columns 256 r: O^T then S^T
 constexpr uint32_t SC_OT = 0, SC_ST = 64;           // offsets within a region
@@ -954,9 +950,7 @@ constexpr uint32_t SC_COLS = 512;
 struct ScanMisc {
     uint64_t bar_full[2];
     uint64_t bar_mma;
-    uint64_t bar_g;   // the output gate tile of the chunk being stored
     uint32_t tmem_base;
-    int g_ok;         // that tile arrived (as seen by thread 0, for warps 0-3)
     alignas(16) float gam[2][DK];  // bulk-copy destination and float4 reads: 16-byte aligned
 };
 static_assert(sizeof(ScanMisc) <= 1280, "scan misc region");
@@ -972,24 +966,12 @@ struct ScanParams {
     const int *cu_seqlens;  // packed sequences (null when dense), as in ChunkParams
     const int *cu_chunks;
     __nv_bfloat16 *o;       // for the row-by-row store of a packed sequence's last, partial tile
-    // block epilogue on the way out: o <- o / rms(o) * norm_weight (.) silu(gate), each optional
-    const float *norm_weight;  // [DV] (with kEpiNorm)
-    float norm_eps;
 };
 
-// Output epilogue of fwd_scan_kernel (template bits): RMSNorm with a weight, SiLU gate.
-constexpr int kEpiNorm = 1, kEpiGate = 2;
+constexpr uint32_t SC_SMEM = SC_MISC + 1280 + 1024;  // + alignment slack
 
-// Dynamic shared memory of an instantiation (+1 KB for aligning the base): the regions
-// an epilogue does not use are left out.
-constexpr uint32_t scan_smem_bytes(int epi)
-{
-    return ((epi & kEpiGate) ? SC_G + 16384 : (epi & kEpiNorm) ? SC_EPI + 1280 : SC_MISC + 1280) + 1024;
-}
-
-template <int EPI>
 __global__ void __launch_bounds__(SC_NT, 1)  // 168 registers: allocation rounds 9 warps up to 12
-fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g, ScanParams p)
+fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm =
@@ -1009,7 +991,6 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         mbar_init(&ms.bar_full[0], 1);
         mbar_init(&ms.bar_full[1], 1);
         mbar_init(&ms.bar_mma, 1);
-        mbar_init(&ms.bar_g, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1042,19 +1023,10 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         bulk_load(ms.gam[sl], p.ws + (size_t)p.ntasks * SLOT_BYTES + task * GAMMA_BYTES, GAMMA_BYTES,
                   &ms.bar_full[sl]);
     };
-    bool g_inflight = false;  // thread 0: a gate tile was issued and not yet seen to land
-    auto issue_gate = [&](int m) {  // the output gate tile of chunk m (rows past the sequence unused)
-        mbar_arrive_expect_tx(&ms.bar_g, C * DV * 2);
-        tma_load_4d(sm + SC_G, &tm_g, &ms.bar_g, 0, h, tstart + m * C, tb);
-        g_inflight = true;
-    };
     if (tid == 0) {
         if (NC > 0) issue_slot(0);
         if (NC > 1) issue_slot(1);
-        if ((EPI & kEpiGate) && NC > 0) issue_gate(0);
     }
-    uint32_t ph_g = 0;
-    bool g_failed = false;  // a gate tile that never arrived: stop waiting for the later ones
     // initial state S^T[j][c] = S0[c][j] into region 1 (chunk 0 reads the region of "chunk -1")
     if (warp < 8) {
         float v[32];
@@ -1081,7 +1053,7 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         return __syncthreads_or(!ok) == 0;
     };
 
-    // O^T of chunk m -> (epilogue) -> bf16 tile [t][j] -> one TMA store (rows past T are
+    // O^T of chunk m -> bf16 tile [t][j] -> one TMA store (rows past T are
     // clipped). Warps 0-7 under named barrier 1, while warp 8 keeps the tensor core busy with
     // the next chunk: warp quarter q reads TMEM lanes (value channels) j = 32 q + lane, warp
     // group colhalf the tokens t = 32 colhalf .. 32 colhalf + 31.
@@ -1091,53 +1063,12 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         const int t0 = colhalf * 32;
         float o0[32];
         tmem_ld32(tm_lane + SC_REG * (m & 1) + SC_OT + t0, o0);
-        if constexpr ((EPI & kEpiNorm) != 0) {
-            // RMSNorm over the value channels of each token: sums of squares over a warp's
-            // 32 channels (lane L ends with token t0 + L), then over the 4 warp quarters
-            float *red = reinterpret_cast<float *>(sm + SC_EPI);  // [4][64], then 1/rms at [256 ..)
-            float sq[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sq[i] = o0[i] * o0[i];
-            transpose_reduce32<32>(sq, lane);
-            red[quarter * 64 + t0 + lane] = sq[0];
-            named_barrier(1, 256);
-            if (tid < 64)
-                red[256 + tid] = rsqrtf((red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid]) * (1.f / DV) +
-                                        p.norm_eps);
-            named_barrier(1, 256);
-            const float wj = p.norm_weight[j];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o0[i] *= red[256 + t0 + i] * wj;
-        }
-        if constexpr ((EPI & kEpiGate) != 0) {
-            if (tid == 0) {
-                ms.g_ok = (!g_failed && mbar_wait_bounded(&ms.bar_g, ph_g, kWaitLimitNs)) ? 1 : 0;
-                if (ms.g_ok) g_inflight = false;
-            }
-            named_barrier(1, 256);
-            ph_g ^= 1u;
-            if (ms.g_ok) {
-                const __nv_bfloat16 *gt = reinterpret_cast<const __nv_bfloat16 *>(sm + SC_G) + t0 * DV + j;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    // silu(g) = g / (1 + exp(-g)), exp argument kept below 80 so 1 + exp stays
-                    // finite (for g < -80, silu(g) is below 2e-33 in magnitude either way)
-                    const float g = __bfloat162float(gt[i * DV]);
-                    o0[i] *= g * recip_newton2(1.f + __expf(-fmaxf(g, -80.f)));
-                }
-            } else {
-                g_failed = true;
-                if (tid == 0) atomicOr(p.status, kStatusTimeout);
-            }
-        }
         __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
 #pragma unroll
         for (int i = 0; i < 32; ++i) ot[(t0 + i) * DV + j] = __float2bfloat16_rn(o0[i]);
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_barrier(1, 256);
-        // every read of this chunk's gate tile is done: the next one may land
-        if ((EPI & kEpiGate) && !g_failed && tid == 0 && m + 1 < NC) issue_gate(m + 1);
         const int rows = min(C, len - m * C);
         if (p.cu_seqlens && rows < C) {
             // a packed sequence's partial last tile: its rows only (a tile store would write
@@ -1253,8 +1184,6 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
         }
     }
     if (tid == 0) bulk_wait_group0();
-    // a gate tile still on its way (only after a timeout): let it land before shared memory goes
-    if (tid == 0 && g_inflight) mbar_wait_bounded(&ms.bar_g, ph_g, kWaitLimitNs);
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
@@ -1265,6 +1194,65 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant_
 }  // namespace
 
 namespace {
+// Block output epilogue as its own pass over o (bf16 [rows][DV], one row per token-head):
+// y = o / sqrt(mean_j o_j^2 + eps) * weight (.) silu(g), each factor optional, in place.
+// A half-warp per row, eight channels per lane (16-byte loads), each thread with two rows in
+// flight. Run inside the scan kernel's per-chunk chain, the same arithmetic lengthened that
+// serial chain by more than this extra pass over o and g costs in HBM time.
+__device__ __forceinline__ void epilogue_row(uint4 &ov, uint4 gv, const float (&w)[8], bool norm, bool gate,
+                                             float eps)
+{
+    float o[8], gg[8];
+    unpack8(ov, o);
+    if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(o[i], o[i], ss);
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);  // within the half-warp
+        const float rinv = rsqrtf(ss * (1.f / DV) + eps);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] *= rinv * w[i];
+    }
+    if (gate) {
+        unpack8(gv, gg);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            // silu(g) = g / (1 + exp(-g)), exp argument kept below 80 so 1 + exp stays finite
+            // (for g < -80, silu(g) is below 2e-33 in magnitude either way)
+            o[i] *= gg[i] * recip_newton2(1.f + __expf(-fmaxf(gg[i], -80.f)));
+    }
+    ov = pack8(o);
+}
+
+__global__ void __launch_bounds__(256) output_epilogue_kernel(__nv_bfloat16 *y, const __nv_bfloat16 *g,
+                                                              const float *weight, float eps, long long nrows)
+{
+    static_assert(DV == 128, "eight channels per lane of a half-warp");
+    const int lane = threadIdx.x & 31, hl = lane & 15, half = lane >> 4;
+    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    float w[8];  // weight is only 4-byte aligned: scalar loads
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = weight ? weight[8 * hl + i] : 1.f;
+    const bool norm = weight != nullptr, gate = g != nullptr;
+    // each warp takes four rows per step (base is the same for all its lanes, so every lane
+    // runs the half-warp shuffles): this half-warp's rows base + half and base + 2 + half
+    for (long long base = 4 * wid; base < nrows; base += 4 * nw) {
+        const long long r0 = base + half, r1 = base + 2 + half;
+        const bool v0 = r0 < nrows, v1 = r1 < nrows;
+        uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0, g0 = o0, g1 = o0;
+        if (v0) o0 = reinterpret_cast<const uint4 *>(y + r0 * DV)[hl];
+        if (v1) o1 = reinterpret_cast<const uint4 *>(y + r1 * DV)[hl];
+        if (gate && v0) g0 = reinterpret_cast<const uint4 *>(g + r0 * DV)[hl];
+        if (gate && v1) g1 = reinterpret_cast<const uint4 *>(g + r1 * DV)[hl];
+        epilogue_row(o0, g0, w, norm, gate, eps);
+        epilogue_row(o1, g1, w, norm, gate, eps);
+        if (v0) reinterpret_cast<uint4 *>(y + r0 * DV)[hl] = o0;
+        if (v1) reinterpret_cast<uint4 *>(y + r1 * DV)[hl] = o1;
+    }
+}
+
 __global__ void recip_eval_kernel(const float *x, float *y, long long n)
 {
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
@@ -1304,7 +1292,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     const bool varlen = a.cu_seqlens != nullptr;
     const int Bm = varlen ? 1 : a.B;  // tensor-map batch extent: packed sequences share one
     const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
-    CUtensorMap mq, mk, mb, mv, mw, mla, mo, mg;
+    CUtensorMap mq, mk, mb, mv, mw, mla, mo;
     if (!make_map(&mq, a.q, false, Bm, a.T, a.H, DK) || !make_map(&mk, a.k, false, Bm, a.T, a.H, DK) ||
         !make_map(&mv, a.v, false, Bm, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, Bm, a.T, a.H, DK) ||
         !make_map(&mo, a.o, false, Bm, a.T, a.H, DV))
@@ -1312,8 +1300,6 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     // a scalar gate has no tile to copy: its map slot is never used (the q map stands in)
     if (bsc) mb = mq; else if (!make_map(&mb, a.b, false, Bm, a.T, a.H, DK)) return cudaErrorInvalidValue;
     if (wsc) mw = mq; else if (!make_map(&mw, a.w, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
-    // the output gate has the layout of o; without one the o map stands in, unused
-    if (!a.out_gate) mg = mo; else if (!make_map(&mg, a.out_gate, false, Bm, a.T, a.H, DV)) return cudaErrorInvalidValue;
     const bool general = varlen || bsc || wsc;
     const bool bwd = a.bwd_ext != nullptr;
     if (bwd && varlen) return cudaErrorInvalidValue;
@@ -1323,11 +1309,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
                 : (bwd ? fwd_chunk_kernel<false, true> : fwd_chunk_kernel<false>);
     cudaError_t e = cudaFuncSetAttribute(chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const int epi = (a.norm_weight ? kEpiNorm : 0) | (a.out_gate ? kEpiGate : 0);
-    void (*scan)(const CUtensorMap, const CUtensorMap, ScanParams) =
-        epi == 0 ? fwd_scan_kernel<0> : epi == kEpiNorm ? fwd_scan_kernel<kEpiNorm>
-        : epi == kEpiGate ? fwd_scan_kernel<kEpiGate> : fwd_scan_kernel<kEpiNorm | kEpiGate>;
-    e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem_bytes(epi));
+    e = cudaFuncSetAttribute(fwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC_SMEM);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1352,18 +1334,27 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     if (e != cudaSuccess || a.chunks_only) return e;
     ScanParams sp{a.B,          a.T,          a.H,    NC,       ntasks,    ws,
                   a.S0,         a.S_T,        a.saved_states, a.status, a.cu_seqlens, cu_chunks,
-                  static_cast<__nv_bfloat16 *>(a.o), a.norm_weight, a.norm_eps};
+                  static_cast<__nv_bfloat16 *>(a.o)};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.H);
     cfg.blockDim = dim3(SC_NT);
-    cfg.dynamicSmemBytes = scan_smem_bytes(epi);
+    cfg.dynamicSmemBytes = SC_SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, scan, mo, mg, sp);
+    e = cudaLaunchKernelEx(&cfg, fwd_scan_kernel, mo, sp);
+    if (e != cudaSuccess || (!a.out_gate && !a.norm_weight)) return e;
+    const long long nrows = (long long)(varlen ? 1 : a.B) * a.T * a.H;
+    if (nrows == 0) return cudaSuccess;
+    const long long blocks = (nrows + 31) / 32;  // 8 warps of four rows per block
+    const int eg = (int)(blocks < (long long)nsm * 16 ? blocks : (long long)nsm * 16);
+    output_epilogue_kernel<<<eg, 256, 0, s>>>(static_cast<__nv_bfloat16 *>(a.o),
+                                              static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight,
+                                              a.norm_eps, nrows);
+    return cudaGetLastError();
 }
 
 }  // namespace gdr2

@@ -197,7 +197,8 @@ gdr2_status gdr2_forward_varlen(int N, int T, int H, int dk, int dv, gdr2_dtype 
  * (cu_seqlens as in gdr2_forward_varlen; B = N sequences), the gate layouts of
  * `gates`, and the output epilogue of the Gated DeltaNet-2 block (note sec. 3,
  * block data-flow paragraph: the mixer output goes through an RMSNorm combined
- * with a SiLU output gate), applied to o in fp32 before its bf16 rounding:
+ * with a SiLU output gate), applied to the bf16 o in fp32 arithmetic by a pass
+ * over o and out_gate after the forward's kernels, on the same stream:
  *
  *   o[t, j] <- o[t, j] / sqrt(mean_j' o[t, j']^2 + norm_eps) * norm_weight[j]
  *              * silu(out_gate[t, j]),        silu(x) = x / (1 + exp(-x))
