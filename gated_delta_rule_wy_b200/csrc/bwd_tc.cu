@@ -264,6 +264,9 @@ constexpr uint32_t VA_U = 147456;    // U^T     [j 128][i]
 constexpr uint32_t VA_X = 163840;    // record staging: 3 x [64 t][128 c] bf16, plain rows
 constexpr uint32_t VA_MISC = VA_X + 3 * X_ARR;
 constexpr uint32_t VA_DU = VA_W, VA_DZ = VA_UT, VA_DPA = VA_KT;
+constexpr uint32_t VA_GV = VA_DU;  // dv tile [64 t][128 j] bf16, once dU~^T's product is done
+constexpr uint32_t VA_GW = VA_T;   // dw tile over T and P (16 KB), once their products are done
+static_assert(VA_P == VA_T + 8192, "T and P are one 16 KB region");
 constexpr uint32_t VA_TX = 16384 + 32768 + 8192 + 8192 + 16384 + 16384 + 16384;
 
 struct VaMisc {
@@ -296,7 +299,9 @@ struct VaParams {
     int wsc;                    // w (and dw) one value per token-head: [B][T][H]
 };
 
-__global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant__ CUtensorMap tm_do, VaParams p)
+__global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant__ CUtensorMap tm_do,
+                                                          const __grid_constant__ CUtensorMap tm_gv,
+                                                          const __grid_constant__ CUtensorMap tm_gw, VaParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm =
@@ -499,16 +504,17 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
         if (!wait_bar(&ms.bar_c, ph_c)) { timed_out = true; break; }
         tc_fence_after_sync();
         {
+            // dv = dz (.) w and dw = dz (.) v as [t][j] tiles over dU~^T and T, P (their products
+            // are done), stored by TMA below (rows past T clipped)
             float dz[32];
             tmem_ld32(tm_lane + VT_DZ + 32 * colhalf, dz);
+            __nv_bfloat16 *tv = reinterpret_cast<__nv_bfloat16 *>(sm + VA_GV);
+            __nv_bfloat16 *tw = reinterpret_cast<__nv_bfloat16 *>(sm + VA_GW);
 #pragma unroll
             for (int s = 0; s < 32; ++s) {
                 const int t = 32 * colhalf + s;
-                if (t < Cn) {
-                    const size_t o = (((size_t)bb * p.T + t0 + t) * p.H + hh) * DV + row;
-                    p.gv[o] = __float2bfloat16_rn(dz[s] * __bfloat162float(wv[s]));
-                    if (!p.wsc) p.gw[o] = __float2bfloat16_rn(dz[s] * __bfloat162float(vv[s]));
-                }
+                tv[t * DV + row] = __float2bfloat16_rn(dz[s] * __bfloat162float(wv[s]));
+                if (!p.wsc) tw[t * DV + row] = __float2bfloat16_rn(dz[s] * __bfloat162float(vv[s]));
             }
             if (p.wsc) {
                 // a scalar write gate: dw_t = sum_j dz[t][j] v[t][j], this warp's 32 channels first
@@ -528,6 +534,11 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
             }
         }
         mma_sync_point();
+        if (tid == 0) {
+            tma_store_4d(&tm_gv, sm + VA_GV, 0, hh, t0, bb);
+            if (!p.wsc) tma_store_4d(&tm_gw, sm + VA_GW, 0, hh, t0, bb);
+            bulk_commit_group();
+        }
         if (p.wsc && tid < C && tid < Cn) {
             const int g = tid >> 5, l = tid & 31;
             const float dw = ms.red[4 * g][l] + ms.red[4 * g + 1][l] + ms.red[4 * g + 2][l] + ms.red[4 * g + 3][l];
@@ -857,17 +868,50 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __nv_bfloat16 *ok_ = reinterpret_cast<__nv_bfloat16 *>(sm + KB_STACK + 16384);
         __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(sm + KB_R);
         const unsigned char *dpa = sm + KB_DPA;
+        if (exact) {
+            // A chunk past the decay guard: the four decay products with one exponential per token
+            // pair (exponents never positive), written where the tensor-core path leaves D and E,
+            // with every decay factor 1 below. Kept out of the unrolled loop: it is rare, and its
+            // code there would be repeated for every token.
+            for (int blk = 0; blk < 2; ++blk) {
+                uint32_t pq[16], pe[16], pk[16], zz[16];
+                for (int u = 0; u < 16; ++u) {
+                    const int t = 32 * hf + 16 * blk + u;
+                    const float Gt = Gs[t * DK + c];
+                    float dqP = 0.f, deA = 0.f, dkAP = 0.f;
+                    const int rA = 64 * (t >> 5) + (t & 31);
+                    for (int i = 0; i < t; ++i) {
+                        const float f = __bfloat162float(ks_[i * DK + c]) * __expf(Gt - Gs[i * DK + c]);
+                        dqP = fmaf(img64(dpa, rA + 32, i), f, dqP);
+                        deA = fmaf(img64(dpa, rA, i), f, deA);
+                    }
+                    for (int s2 = t + 1; s2 < C; ++s2) {
+                        const int rs = 64 * (s2 >> 5) + (s2 & 31);
+                        const float ksv = __bfloat162float(ks_[s2 * DK + c]);
+                        const float x = img64(dpa, rs, t) * __bfloat162float(bs[s2 * DK + c]) * ksv +
+                                        img64(dpa, rs + 32, t) * __bfloat162float(qs[s2 * DK + c]);
+                        dkAP = fmaf(x, __expf(Gs[s2 * DK + c] - Gt), dkAP);
+                    }
+                    pq[u] = __float_as_uint(dqP);
+                    pe[u] = __float_as_uint(deA);
+                    pk[u] = __float_as_uint(dkAP);
+                    zz[u] = 0u;
+                }
+                tmem_st16u(tm_lane + (hf ? KT_D1 : KT_D0) + 16 * blk, pe);
+                tmem_st16u(tm_lane + (hf ? KT_D1 : KT_D0) + 32 + 16 * blk, pq);
+                tmem_st16u(tm_lane + KT_E1 + 32 * hf + 16 * blk, pk);
+                tmem_st16u(tm_lane + KT_E0 + 32 * hf + 16 * blk, zz);
+            }
+        }
         float dG[32];
         float hs = 0.f, kts = 0.f;
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
             float De[16], Dq[16], E1[16], E0[16];
-            if (!exact) {
-                tmem_ld16(tm_lane + (hf ? KT_D1 : KT_D0) + 16 * blk, De);
-                tmem_ld16(tm_lane + (hf ? KT_D1 : KT_D0) + 32 + 16 * blk, Dq);
-                tmem_ld16(tm_lane + KT_E1 + 32 * hf + 16 * blk, E1);
-                tmem_ld16(tm_lane + KT_E0 + 32 * hf + 16 * blk, E0);
-            }
+            tmem_ld16(tm_lane + (hf ? KT_D1 : KT_D0) + 16 * blk, De);
+            tmem_ld16(tm_lane + (hf ? KT_D1 : KT_D0) + 32 + 16 * blk, Dq);
+            tmem_ld16(tm_lane + KT_E1 + 32 * hf + 16 * blk, E1);
+            tmem_ld16(tm_lane + KT_E0 + 32 * hf + 16 * blk, E0);
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int tl = 16 * blk + u, t = 32 * hf + tl;
@@ -879,30 +923,12 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float xe = __bfloat162float(X[(64 + t) * DK + c]);
                 const float xk = __bfloat162float(X[(128 + t) * DK + c]);
                 const float eG = __expf(Gt), kcf = __expf(gCc - Gt);
-                float dqP, deA, dkAP;
-                if (!exact) {
-                    const float Lf = __expf(Gt - ghc);
-                    dqP = Dq[u] * Lf;
-                    deA = De[u] * Lf;
-                    dkAP = E1[u] * __expf(g1c - Gt);
-                    if (hf == 0) dkAP = fmaf(E0[u], __expf(g0c - Gt), dkAP);
-                } else {
-                    // one exponential per token pair (exponents never positive)
-                    dqP = 0.f, deA = 0.f, dkAP = 0.f;
-                    const int rA = 64 * (t >> 5) + (t & 31);
-                    for (int i = 0; i < t; ++i) {
-                        const float f = __bfloat162float(ks_[i * DK + c]) * __expf(Gt - Gs[i * DK + c]);
-                        dqP = fmaf(img64(dpa, rA + 32, i), f, dqP);
-                        deA = fmaf(img64(dpa, rA, i), f, deA);
-                    }
-                    for (int s = t + 1; s < C; ++s) {
-                        const int rs = 64 * (s >> 5) + (s & 31);
-                        const float ksv = __bfloat162float(ks_[s * DK + c]);
-                        const float x = img64(dpa, rs, t) * __bfloat162float(bs[s * DK + c]) * ksv +
-                                        img64(dpa, rs + 32, t) * __bfloat162float(qs[s * DK + c]);
-                        dkAP = fmaf(x, __expf(Gs[s * DK + c] - Gt), dkAP);
-                    }
-                }
+                // the decay factors of the products' half-chunk references (1 on the exact path)
+                const float Lf = exact ? 1.f : __expf(Gt - ghc);
+                const float dqP = Dq[u] * Lf;
+                const float deA = De[u] * Lf;
+                float dkAP = E1[u] * (exact ? 1.f : __expf(g1c - Gt));
+                if (hf == 0 && !exact) dkAP = fmaf(E0[u], __expf(g0c - Gt), dkAP);
                 const float dq = fmaf(xq, eG, dqP);
                 const float de = fmaf(-xe, eG, deA);
                 const float dkt = xk * kcf;
@@ -1072,11 +1098,15 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     // 3. value side
     e = cudaFuncSetAttribute(bwd_value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VA_SMEM);
     if (e != cudaSuccess) return e;
+    CUtensorMap mgv, mgw;
+    if (!make_map(&mgv, a.gv, false, a.B, a.T, a.H, DV)) return cudaErrorInvalidValue;
+    if (wsc) mgw = mgv;  // a scalar write gate's dw is reduced in the kernel: no tile
+    else if (!make_map(&mgw, a.gw, false, a.B, a.T, a.H, DV)) return cudaErrorInvalidValue;
     VaParams vp{a.B, a.T, a.H, NC, ntasks, ws, ws + L.ext, ws + L.dsc, states,
                 static_cast<const __nv_bfloat16 *>(a.v), static_cast<const __nv_bfloat16 *>(a.w),
                 static_cast<__nv_bfloat16 *>(a.gv), static_cast<__nv_bfloat16 *>(a.gw), ws + L.dpa, ws + L.xrec,
                 a.status, wsc ? 1 : 0};
-    bwd_value_kernel<<<grid, 256, VA_SMEM, s>>>(mdo, vp);
+    bwd_value_kernel<<<grid, 256, VA_SMEM, s>>>(mdo, mgv, mgw, vp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
