@@ -330,7 +330,10 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
     const uint32_t tm = ms.tmem_base;
     const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
 
-    auto issue_loads = [&](int task) {
+    // A task's copies, in three groups: dO, dS'^T and U~^T land where no store reads; T, P and
+    // W where the dv and dw tiles were staged; K~ where the dA/dP image was (thread 0 waits
+    // for those stores to have read their source before the later groups).
+    auto issue_loads = [&](int task, bool first) {
         const int bhh = task / p.NC, n = task % p.NC;
         const int bb = bhh / p.H, hh = bhh % p.H;
         const unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
@@ -339,14 +342,16 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
         tma_load_4d(sm + VA_DO, &tm_do, &ms.bar_ld, 0, hh, n * C, bb);
         tma_load_4d(sm + VA_DO + 8192, &tm_do, &ms.bar_ld, 64, hh, n * C, bb);
         bulk_load(sm + VA_DS, p.dsc + (size_t)task * DS_IMG, DS_IMG, &ms.bar_ld);
+        bulk_load(sm + VA_UT, slot + SLOT_U, 16384, &ms.bar_ld);
+        if (!first) bulk_wait_group_read1();  // the dv and dw tiles have left W, T and P
         bulk_load(sm + VA_T, ext + EXT_T, 8192, &ms.bar_ld);
         bulk_load(sm + VA_P, slot + SLOT_P, 8192, &ms.bar_ld);
         bulk_load(sm + VA_W, ext + EXT_W, 16384, &ms.bar_ld);
-        bulk_load(sm + VA_UT, slot + SLOT_U, 16384, &ms.bar_ld);
+        if (!first) bulk_wait_group_read0();  // the dA/dP image has left K~
         bulk_load(sm + VA_KT, slot + SLOT_KT, 16384, &ms.bar_ld);
     };
     const int ntasks = p.ntasks;
-    if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
+    if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x, true);
 
     uint32_t ph_ld = 0, ph_a = 0, ph_b = 0, ph_c = 0, ph_d = 0;
     bool timed_out = false, loads_pending = (int)blockIdx.x < ntasks;
@@ -609,8 +614,7 @@ __global__ void __launch_bounds__(256, 1) bwd_value_kernel(const __grid_constant
             bulk_store(p.xrec + (size_t)task * XREC_BYTES + 3 * X_ARR, ms.dpd, 64 * 4 + 128 * 4);
             bulk_commit_group();
             if (task + (int)gridDim.x < ntasks) {
-                bulk_wait_group_read0();  // the next loads overwrite the image just stored
-                issue_loads(task + gridDim.x);
+                issue_loads(task + gridDim.x, false);
                 loads_pending = true;
             }
         }
@@ -638,11 +642,11 @@ constexpr uint32_t KB_DPA = 139264;   // [dA_0; dP_0; dA_1; dP_1]
 constexpr uint32_t KB_X = 155648;     // the value kernel's record
 constexpr uint32_t KB_SCAN = KB_X + al1k(XREC_BYTES);  // prefix-scan scratch [16][128] fp32
 constexpr uint32_t KB_MISC = KB_SCAN + 8192;
-constexpr uint32_t KB_TX = 3 * 16384 + 32768 + DPA_IMG + XREC_BYTES;
+constexpr uint32_t KB_TX = 3 * 16384 + 32768 + DPA_IMG;  // q, k, b, log_alpha and the dA/dP image
 constexpr int R_ROWS = 96;
 
 struct KbMisc {
-    uint64_t bar_ld, bar_mma;
+    uint64_t bar_ld, bar_mma, bar_x;  // bar_x: the value kernel's record
     uint32_t tmem_base;
     int pad;
     alignas(16) float g0[DK];       // G at tokens 15 and 47 (half-chunk references; float4 reads)
@@ -693,6 +697,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (tid == 0) {
         mbar_init(&ms.bar_ld, 1);
         mbar_init(&ms.bar_mma, 1);
+        mbar_init(&ms.bar_x, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -715,13 +720,20 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!bsc) tma_load_4d(sm + KB_B, &tm_b, &ms.bar_ld, 0, hh, n * C, bb);
         tma_load_4d(sm + KB_LA, &tm_la, &ms.bar_ld, 0, hh, n * C, bb);
         bulk_load(sm + KB_DPA, p.dpa + (size_t)task * DPA_IMG, DPA_IMG, &ms.bar_ld);
-        bulk_load(sm + KB_X, p.xrec + (size_t)task * XREC_BYTES, XREC_BYTES, &ms.bar_ld);
+    };
+    // the record lands over the previous task's dlog_alpha tile: issued once that has left
+    auto issue_record = [&](int task) {
+        mbar_arrive_expect_tx(&ms.bar_x, XREC_BYTES);
+        bulk_load(sm + KB_X, p.xrec + (size_t)task * XREC_BYTES, XREC_BYTES, &ms.bar_x);
     };
     const int ntasks = p.ntasks;
-    if (tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
+    if (tid == 0 && (int)blockIdx.x < ntasks) {
+        issue_loads(blockIdx.x);
+        issue_record(blockIdx.x);
+    }
 
-    uint32_t ph_ld = 0, ph_mma = 0;
-    bool timed_out = false, loads_pending = (int)blockIdx.x < ntasks;
+    uint32_t ph_ld = 0, ph_mma = 0, ph_x = 0;
+    bool timed_out = false, loads_pending = (int)blockIdx.x < ntasks, x_pending = loads_pending;
     const int o8 = tid & 15, tg = tid >> 4, HI = tg >> 3;  // prep: channels 8 o8.., tokens 4 tg..
     const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + KB_Q);
     const __nv_bfloat16 *ks_ = reinterpret_cast<const __nv_bfloat16 *>(sm + KB_K);
@@ -784,6 +796,11 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ms.g0[tid] = g0;
             ms.g1[tid] = g1;
             ms.gC[tid] = run;
+        }
+        if (tid == 0 && task != (int)blockIdx.x) {
+            bulk_wait_group_read0();  // the previous task's gradient tiles have left STACK, R and X
+            issue_record(task);
+            x_pending = true;
         }
         __syncthreads();
         bool risky = false;
@@ -856,6 +873,12 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ph_mma ^= 1u;
             if (__syncthreads_or(!ok)) { timed_out = true; break; }
             tc_fence_after_sync();
+        }
+        {
+            const bool ok = mbar_wait_bounded(&ms.bar_x, ph_x, kWaitLimitNs);
+            if (__syncthreads_or(!ok)) { timed_out = true; break; }
+            ph_x ^= 1u;
+            x_pending = false;
         }
         // ================= per channel: thread (c, half hf) walks tokens 32 hf .. 32 hf + 31 =================
         const int c = quarter * 32 + lane;
@@ -960,7 +983,10 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // dlog_alpha[t] = sum_{t' >= t} dG[t'] + sum_j dS' (.) S e^{G_C} + sum_{t' < t} dk~ (.) k~:
         // the last sum as a prefix (as total minus suffix it cancels: the last token's term is
         // O(1) while under strong decay every other term, and the result, are near e^-32)
+        // (staged as a [64 t][128 c] fp32 tile over X_q and X_e, whose reads ended at the barrier)
         {
+            float *Dl = reinterpret_cast<float *>(sm + KB_X);
+            static_assert(2 * X_ARR == C * DK * 4, "the dlog_alpha tile fits X_q and X_e");
             float pre = hf ? ms.kts[0][c] : 0.f;
 #pragma unroll 4
             for (int tl = 0; tl < 32; ++tl) {
@@ -968,14 +994,14 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float Gt = Gs[t * DK + c];
                 const float ktk = __bfloat162float(X[(128 + t) * DK + c]) * __expf(gCc - Gt) *
                                   __bfloat162float(ks_[t * DK + c]);
-                Gs[t * DK + c] = pre;
+                Dl[t * DK + c] = pre;
                 pre += ktk;
             }
             float run = rowsum * __expf(gCc) + (hf == 0 ? ms.hsum[1][c] : 0.f);
 #pragma unroll
             for (int tl = 31; tl >= 0; --tl) {
                 run += dG[tl];
-                Gs[(32 * hf + tl) * DK + c] += run;
+                Dl[(32 * hf + tl) * DK + c] += run;
             }
         }
         fence_proxy_async_smem();
@@ -985,10 +1011,11 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_store_4d(&tm_gq, sm + KB_STACK, 0, hh, n * C, bb);
             tma_store_4d(&tm_gk, sm + KB_STACK + 16384, 0, hh, n * C, bb);
             if (!bsc) tma_store_4d(&tm_gb, sm + KB_R, 0, hh, n * C, bb);
-            tma_store_4d(&tm_gla, sm + KB_LA, 0, hh, n * C, bb);
+            tma_store_4d(&tm_gla, sm + KB_X, 0, hh, n * C, bb);
             bulk_commit_group();
+            // q, k, b, log_alpha and the dA/dP image are no store's source: the next task's
+            // copies go out now, under the stores (its record follows once they have left)
             if (task + (int)gridDim.x < ntasks) {
-                bulk_wait_group_read0();  // the staged gradients have left before the next loads land
                 issue_loads(task + gridDim.x);
                 loads_pending = true;
             }
@@ -998,6 +1025,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         bulk_wait_group0();
         if (timed_out) {
             if (loads_pending) mbar_wait_bounded(&ms.bar_ld, ph_ld, kWaitLimitNs);
+            if (x_pending) mbar_wait_bounded(&ms.bar_x, ph_x, kWaitLimitNs);
             atomicOr(p.status, kStatusTimeout);
         }
     }
