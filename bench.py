@@ -49,7 +49,7 @@ BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 2 * 256 + 256  # q,k,v bf16 + log_alpha f
 FLOP_PER_TOKEN_HEAD = 139_264  # chunk products at C=64, d=128, triangular parts counted once
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-LAUNCHES_PER_STEP = 2  # chunk kernel + scan kernel (tensor-core path)
+LAUNCHES_PER_STEP = 1  # the fused forward kernel (chunk tasks, then the scans), after a memset of its flags
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -498,10 +498,11 @@ def run_ours(args, world, rank, local):
     achieved = alg_bytes / t_launch / 1e9
     rec = committed_record("fwd")
     traffic = float(rec["dram_bytes_per_launch"]) if rec else None
-    kernel = "one gdr2_forward call: fwd_chunk_kernel + fwd_scan_kernel"
+    # the call's kernels and their shares of its device time, from the committed ncu record
+    kernel = "one gdr2_forward call"
     if rec and "device_time_share" in rec:
-        kernel += " (" + ", ".join(f"{k} {100 * v:.0f}%" for k, v in rec["device_time_share"].items()) + \
-                  " of its device time under ncu)"
+        kernel += ": " + " + ".join(f"{k} ({100 * v:.0f}% of its device time under ncu)"
+                                    for k, v in rec["device_time_share"].items())
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": alg_bytes, "kernel": kernel}

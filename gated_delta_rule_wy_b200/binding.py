@@ -29,7 +29,8 @@ EXPORTED_SYMBOLS = ("gdr2_abi_version", "gdr2_last_error", "gdr2_forward_workspa
                     "gdr2_forward_ex", "gdr2_short_conv_silu", "gdr2_gate_activations", "gdr2_segment_states",
                     "gdr2_decode_step", "gdr2_decode_step_gated",
                     "gdr2_backward_workspace_bytes", "gdr2_backward", "gdr2_backward_gated", "gdr2_backward_noalloc",
-                    "gdr2_sync_status", "gdr2_debug_force_timeout", "gdr2_debug_recip")
+                    "gdr2_sync_status", "gdr2_debug_force_timeout", "gdr2_debug_recip",
+                    "gdr2_debug_forward_unfused")
 NOALLOC_SCRATCH_BYTES = 64 << 20  # GDR2_NOALLOC_SCRATCH_BYTES
 
 
@@ -93,6 +94,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.gdr2_sync_status.argtypes = [P]
         lib.gdr2_debug_force_timeout.restype = None
         lib.gdr2_debug_force_timeout.argtypes = [I]
+        lib.gdr2_debug_forward_unfused.restype = None
+        lib.gdr2_debug_forward_unfused.argtypes = [I]
         lib.gdr2_debug_recip.restype = I
         lib.gdr2_debug_recip.argtypes = [P, P, ctypes.c_longlong, P]
         _lib = lib

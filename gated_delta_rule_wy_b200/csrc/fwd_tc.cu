@@ -25,6 +25,13 @@
 //   2. scan kernel (one CTA per (batch, head), chunks in order): S^T stays in
 //      TMEM as fp32; per chunk one pass copies it to a bf16 TMEM operand and
 //      scales it by gamma, then one batch of MMAs produces S'^T and O^T.
+// A scan's chunks are a serial chain (about 2.3 K cycles each) on one SM, so run
+// after the chunk kernel the scans leave most SMs idle. Where B H leaves at least
+// 32 SMs free, both run as one cooperative launch instead (fwd_fused_kernel):
+// every CTA takes chunk tasks from a queue in chunk-major order, and CTA b < B H
+// leaves the queue near its end for the scan of (batch, head) b, which copies a
+// chunk's workspace slot only once that task's flag says it is written. The scans
+// then overlap the last quarter or so of the chunk tasks.
 //
 // Decay range. exp(G_t - G_i) is formed as a product of two factors around a
 // per-channel reference g_I, the cumulative decay at the midpoint of the
@@ -98,12 +105,17 @@ constexpr int R_ROWS = 96;               // rows of the stacked [R_0; R_1] opera
 static_assert(OFF_STACK + 2 * 192 * 128 <= OFF_Z, "[Q'; M] (48 KB) is staged over STACK and R, clear of Z");
 
 constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
+// Fused kernel: at least this many CTAs stay on the chunk queue while B H of them scan, and the
+// ratio of a scan's time per chunk to a chunk task's time that places the switch.
+constexpr int kFusedMinQueueCtas = 32;
+constexpr double kScanToTaskTime = 0.25;
 
 struct Misc {
     uint64_t bar_tma;
     uint64_t bar_mma;
     uint32_t tmem_base;
-    int pad[3];
+    int q_next;      // fused kernel: the queue index this CTA takes next
+    int pad[2];
     float gC[DK];    // exp(G_C)
     float eg0[DK];   // W combine factor of half-chunk 0: exp(g_0)
     float eg1[DK];   // ... of half-chunk 1: exp(g_1)
@@ -126,6 +138,12 @@ struct ChunkParams {
     const __nv_bfloat16 *bg, *wg;
     unsigned char *ext;     // backward: T and W of every task (EXT_BYTES each), else null
     int debug_giveup;       // test hook: give up a 1 us wait before the first copy
+    // fused kernel (dense, vector gates): a task queue in chunk-major order and one ready flag
+    // per task (both zero at launch); CTA b < BH leaves the queue for the scan of (sequence,
+    // head) b once the queue index it holds reaches switch_at
+    int *queue = nullptr;
+    unsigned *flags = nullptr;
+    int BH = 0, switch_at = 0;
 };
 
 // Where a task's chunk lives: tensor-map coordinates (token t0, sequence bb), head h, and the
@@ -205,19 +223,18 @@ __global__ void __launch_bounds__(1024) varlen_prefix_kernel(const int *cu, int 
 constexpr uint32_t CK_M = 0, CK_U = 128, CK_W0 = 256, CK_W1 = 320, CK_AP0 = 384, CK_AP1 = 416;
 constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W_0, W_1 once those are read
 
-// GENERAL: packed sequences and/or scalar gates may be in use; the other instantiation is
-// the dense, vector-gate kernel with those branches compiled away. BWD (dense sequences):
-// T and W of each task also go to p.ext for the backward.
-template <bool GENERAL, bool BWD = false>
-__global__ void __launch_bounds__(NT, 1)
-fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
-                 ChunkParams p)
+// The chunk kernel's work. GENERAL: packed sequences and/or scalar gates may be in use; the
+// other instantiation is the dense, vector-gate kernel with those branches compiled away. BWD
+// (dense sequences): T and W of each task also go to p.ext for the backward. FUSED (dense
+// sequences): the first role of the fused kernel -- tasks come from a queue in chunk-major
+// order, each finished task is published by its flag, and the TMEM allocation is kept for the
+// scan role (tm_out). Returns whether a bounded wait gave up (the same on every thread).
+template <bool GENERAL, bool BWD, bool FUSED>
+__device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_b,
+                                           const CUtensorMap &tm_v, const CUtensorMap &tm_w, const CUtensorMap &tm_la,
+                                           const ChunkParams &p, unsigned char *sm, uint32_t &tm_out)
 {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *sm =
-        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    static_assert(!FUSED || !BWD, "the fused kernel is the dense forward without the backward's extras");
     Misc &ms = *reinterpret_cast<Misc *>(sm + OFF_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -259,7 +276,15 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool ok = mbar_wait_bounded(&ms.bar_mma, 0, 1000);
         timed_out = __syncthreads_or(!ok) != 0;
     }
-    if (!timed_out && tid == 0 && (int)blockIdx.x < ntasks) issue_loads(blockIdx.x);
+    // queue index -> task (slot): FUSED takes chunk n of every (sequence, head) before chunk n + 1
+    auto task_of = [&](int qi) -> int { return FUSED ? (qi % p.BH) * p.NC + qi / p.BH : qi; };
+    int q0 = blockIdx.x;
+    if (FUSED) {
+        if (tid == 0) ms.q_next = atomicAdd(p.queue, 1);
+        __syncthreads();
+        q0 = ms.q_next;
+    }
+    if (!timed_out && tid == 0 && q0 < ntasks) issue_loads(task_of(q0));
     // the scan kernel may be scheduled now: its CTAs take an SM only once this (persistent) CTA
     // has left it, and they read the workspace only after this whole grid has completed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -284,7 +309,9 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float *A32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
 
-    for (int task = blockIdx.x; task < ntasks && !timed_out; task += gridDim.x) {
+    int prev_task = -1;  // FUSED: the task finished last, whose flag is still to be set
+    for (int qi = q0; qi < ntasks && !timed_out;) {
+        const int task = task_of(qi);
         const ChunkLoc loc = locate_chunk<GENERAL>(p, task);
         const int Cn = loc.Cn;
         // a scalar gate: this thread's four rows (t = tid / 16 + 16 k), read while the copies land
@@ -301,7 +328,16 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // this task's workspace slot: each section is staged in shared memory and bulk-copied
         unsigned char *slot = p.ws + (size_t)task * SLOT_BYTES;
-        if (tid == 64) bulk_wait_group_read0();  // K~, P and U~ of the previous task have left shared memory
+        if (tid == 64) {
+            // K~, P and U~ of the previous task have left shared memory (FUSED: and reached
+            // global memory, for its flag)
+            if (FUSED) {
+                bulk_wait_group0();
+                fence_proxy_async_global();
+            } else {
+                bulk_wait_group_read0();
+            }
+        }
         if (!wait_bar(&ms.bar_tma, ph_tma)) { timed_out = true; break; }
         if (GENERAL && Cn < C) {
             // a packed sequence's partial chunk: the rows past its end hold the next sequence's
@@ -374,8 +410,20 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 ms.gC[c] = __expf(g[31] + off);
             }
         }
-        if (tid == 0) bulk_wait_group_read0();  // ... and [Q'; M] too, before the operands are rebuilt
+        if (tid == 0) {  // ... and [Q'; M] too, before the operands are rebuilt
+            if (FUSED) {
+                bulk_wait_group0();
+                fence_proxy_async_global();
+            } else {
+                bulk_wait_group_read0();
+            }
+        }
         __syncthreads();
+        if (FUSED && tid == 0 && prev_task >= 0) {
+            // every section of the previous task's slot and its gamma are in global memory
+            __threadfence();
+            st_release_gpu(p.flags + prev_task, 1u);
+        }
         bool risky = false;
         float G[4][8];
         float g0[8], g1[8], gC[8];
@@ -610,7 +658,13 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // The staging buffers are free: prefetch the next task. K~ and P are final: copy them to
         // the slot in the background. Both are issued from warp 2, idle in the first solve levels.
         if (tid == 64) {
-            if (task + (int)gridDim.x < ntasks) issue_loads(task + gridDim.x);
+            int qn = qi + (int)gridDim.x;
+            if (FUSED) {
+                // a CTA that will run a scan leaves the queue once its index reaches switch_at
+                qn = ((int)blockIdx.x < p.BH && qi >= p.switch_at) ? ntasks : atomicAdd(p.queue, 1);
+                ms.q_next = qn;  // read by every thread after the barriers below
+            }
+            if (qn < ntasks) issue_loads(task_of(qn));
             bulk_store(slot + SLOT_KT, sm + OFF_KT, 16384);
             bulk_store(slot + SLOT_P, sm + OFF_P, 8192);
             bulk_commit_group();
@@ -923,12 +977,40 @@ fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bulk_store(slot + SLOT_B1, sm + OFF_STACK, 2 * B1_ROWS * 128);
             bulk_commit_group();
         }
+        prev_task = task;
+        qi = FUSED ? ms.q_next : qi + (int)gridDim.x;
     }
-    if (tid == 0 || tid == 64) bulk_wait_group0();  // each waits for the bulk groups it committed
+    if (tid == 0 || tid == 64) {
+        bulk_wait_group0();  // each waits for the bulk groups it committed
+        if (FUSED) fence_proxy_async_global();
+    }
+    if (FUSED) {
+        __syncthreads();
+        if (!timed_out && tid == 0 && prev_task >= 0) {
+            __threadfence();
+            st_release_gpu(p.flags + prev_task, 1u);
+        }
+    }
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, TM_COLS);
+    if (!FUSED && warp == 0) tmem_dealloc(tm, TM_COLS);
+    tm_out = tm;
+    return timed_out;
+}
+
+template <bool GENERAL, bool BWD = false>
+__global__ void __launch_bounds__(NT, 1)
+fwd_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
+                 ChunkParams p)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t tm;
+    chunk_body<GENERAL, BWD, false>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, p, sm, tm);
 }
 
 // ---- scan kernel ----
@@ -1190,6 +1272,205 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     if (warp == 0) tmem_dealloc(tm, SC_COLS);
 }
 
+// ---- fused kernel: chunk tasks, then (CTA b < B H) the scan of (sequence, head) b ----
+// One cooperative launch of one CTA per SM, so every CTA is resident and a scan that waits for
+// a chunk task only waits for CTAs that are running and never wait themselves. All CTAs first
+// take chunk tasks from a queue in chunk-major order; CTA b < B H leaves the queue near its
+// end (switch_at) and runs the scan of (sequence, head) b, whose first chunks are long done,
+// while the other CTAs finish the queue. The scan copies a slot only after its task's flag is
+// set. The scan's steps are those of fwd_scan_kernel, on eight warps: thread 0 issues the
+// products and the slot copies.
+__device__ __forceinline__ void fused_scan(const CUtensorMap &tm_o, const ScanParams &p, const unsigned *flags,
+                                           unsigned char *sm, uint32_t tm, int bh, bool &timed_out)
+{
+    ScanMisc &ms = *reinterpret_cast<ScanMisc *>(sm + SC_MISC);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quarter = warp & 3, colhalf = warp >> 2;
+    const int bb = bh / p.H, h = bh % p.H;
+    const int c0 = colhalf * 64;  // this thread's 64 state columns c (S^T columns)
+    const int NC = p.NC;
+    const size_t base = (size_t)bh * p.NC;
+    const uint32_t tm_lane = tm + ((uint32_t)(quarter * 32) << 16);
+    const int j = quarter * 32 + lane;  // this thread's TMEM lane = value channel
+
+    if (tid == 0) {
+        mbar_init(&ms.bar_full[0], 1);
+        mbar_init(&ms.bar_full[1], 1);
+        mbar_init(&ms.bar_mma, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // thread 0: a task's slot is copied once its flag is set; if a flag never comes, the copy is
+    // not issued and the wait for it below gives up as well
+    auto issue_slot = [&](int n) {
+        const int sl = n & 1;
+        const size_t task = base + n;
+        if (!flag_wait_bounded(flags + task, kWaitLimitNs)) return;
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(&ms.bar_full[sl], SLOT_BYTES + GAMMA_BYTES);
+        bulk_load(sm + (sl ? SC_SLOT1 : SC_SLOT0), p.ws + task * SLOT_BYTES, SLOT_BYTES, &ms.bar_full[sl]);
+        bulk_load(ms.gam[sl], p.ws + (size_t)p.ntasks * SLOT_BYTES + task * GAMMA_BYTES, GAMMA_BYTES,
+                  &ms.bar_full[sl]);
+    };
+    if (tid == 0) {
+        if (NC > 0) issue_slot(0);
+        if (NC > 1) issue_slot(1);
+    }
+    // initial state S^T[j][c] = S0[c][j] into region 1 (chunk 0 reads the region of "chunk -1")
+    {
+        float v[32];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = p.S0 ? p.S0[((size_t)bh * DK + c0 + q2 * 32 + i) * DV + j] : 0.f;
+            tmem_st32(tm_lane + SC_REG + SC_ST + c0 + q2 * 32, v);
+        }
+        float zz[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) zz[i] = 0.f;
+        tmem_st32(tm_lane + SC_OT + colhalf * 32, zz);  // chunk 0's O^T starts at zero
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+
+    uint32_t ph_full = 0, ph_mma = 0;  // bit s: phase of bar_full[s]
+    auto store_o = [&](int m) {  // as in fwd_scan_kernel: O^T of chunk m -> bf16 tile -> TMA store
+        if (tid == 0) bulk_wait_group_read0();
+        named_barrier(1, NT);
+        const int t0 = colhalf * 32;
+        float o0[32];
+        tmem_ld32(tm_lane + SC_REG * (m & 1) + SC_OT + t0, o0);
+        __nv_bfloat16 *ot = reinterpret_cast<__nv_bfloat16 *>(sm + SC_O);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ot[(t0 + i) * DV + j] = __float2bfloat16_rn(o0[i]);
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        named_barrier(1, NT);
+        if (tid == 0) {
+            tma_store_4d(&tm_o, sm + SC_O, 0, h, m * C, bb);
+            bulk_commit_group();
+        }
+    };
+
+    if (NC > 0) {
+        const bool ok = mbar_wait_bounded(&ms.bar_full[0], 0, kWaitLimitNs);
+        ph_full ^= 1u;
+        if (__syncthreads_or(!ok)) timed_out = true;
+    }
+    for (int n = 0; n < NC && !timed_out; ++n) {
+        const int sl = n & 1;
+        const uint32_t slot = sbase + (sl ? SC_SLOT1 : SC_SLOT0);
+        const uint32_t rg = SC_REG * (uint32_t)sl, rg_prev = SC_REG * (uint32_t)(sl ^ 1);
+        // ---- S^T (previous region) -> bf16 operand; gamma-scaled S^T -> this region ----
+        {
+            float s0[32], s1[32];
+            tmem_ld32x2(tm_lane + rg_prev + SC_ST + c0, tm_lane + rg_prev + SC_ST + c0 + 32, s0, s1);
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(s0[2 * i], s0[2 * i + 1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(s1[2 * i], s1[2 * i + 1]);
+                pk[i] = *reinterpret_cast<uint32_t *>(&h0);
+                pk[16 + i] = *reinterpret_cast<uint32_t *>(&h1);
+            }
+            tmem_st32u_nw(tm_lane + SC_SA + (uint32_t)(c0 >> 1), pk);
+            const float4 *g4 = reinterpret_cast<const float4 *>(&ms.gam[sl][c0]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 ga = g4[i], gb = g4[8 + i];
+                s0[4 * i] *= ga.x; s0[4 * i + 1] *= ga.y; s0[4 * i + 2] *= ga.z; s0[4 * i + 3] *= ga.w;
+                s1[4 * i] *= gb.x; s1[4 * i + 1] *= gb.y; s1[4 * i + 2] *= gb.z; s1[4 * i + 3] *= gb.w;
+            }
+            tmem_st32_nw(tm_lane + rg + SC_ST + c0, s0);
+            tmem_st32_nw(tm_lane + rg + SC_ST + c0 + 32, s1);
+            tmem_wait_st();
+        }
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
+        // ---- [O^T | S^T] += S_bf16^T [Q'; M]^T ;  S^T += U~^T K~ ;  O^T += U~^T P^T ----
+        if (tid == 0) {
+            const uint32_t id1 = idesc_bf16(128, B1_ROWS, false, false);
+            const uint32_t idS = idesc_bf16(128, 128, false, true);
+            const uint32_t idO = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t b1 =
+                    sdesc_sw128(slot + SLOT_B1 + (ks >> 2) * (B1_ROWS * 128) + (ks & 3) * 32, 16, 1024);
+                mma_bf16_ts(tm + rg + SC_OT, tm + SC_SA + ks * 8, b1, id1, 1);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t au = sdesc_sw128(slot + SLOT_U + ks * 32, 16, 1024);
+                const uint64_t bk = sdesc_sw128(slot + SLOT_KT + ks * 2048, 8192, 1024);
+                mma_bf16(tm + rg + SC_ST, au, bk, idS, 1);
+                const uint64_t bp = sdesc_sw128(slot + SLOT_P + ks * 32, 16, 1024);
+                mma_bf16(tm + rg + SC_OT, au, bp, idO, 1);
+            }
+            mma_commit(&ms.bar_mma);
+        }
+        // overlaps this chunk's MMAs (the other region), then clears that region's O^T for
+        // chunk n + 1 (each thread rewrites only the lane and columns it has just read)
+        if (n > 0) store_o(n - 1);
+        {
+            float zz[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) zz[i] = 0.f;
+            tmem_st32_nw(tm_lane + rg_prev + SC_OT + colhalf * 32, zz);
+            tmem_wait_st();
+        }
+        // the next slot and this chunk's MMAs, one barrier for both
+        {
+            bool ok = true;
+            if (n + 1 < NC) {
+                ok = mbar_wait_bounded(&ms.bar_full[sl ^ 1], (ph_full >> (sl ^ 1)) & 1u, kWaitLimitNs);
+                ph_full ^= 1u << (sl ^ 1);
+            }
+            ok = mbar_wait_bounded(&ms.bar_mma, ph_mma, kWaitLimitNs) && ok;
+            ph_mma ^= 1u;
+            tc_fence_before_sync();
+            if (__syncthreads_or(!ok)) { timed_out = true; break; }
+            tc_fence_after_sync();
+        }
+        if (tid == 0 && n + 2 < NC) issue_slot(n + 2);  // this slot's MMAs are done
+    }
+    if (!timed_out && NC > 0) store_o(NC - 1);
+    if (!timed_out && p.S_T) {
+        const uint32_t rg_last = SC_REG * (uint32_t)((NC + 1) & 1);  // region of chunk NC - 1 (region 1 if NC = 0)
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int cb = c0 + q2 * 32;
+            float sv[32];
+            tmem_ld32(tm_lane + rg_last + SC_ST + cb, sv);
+            float *dst = p.S_T + ((size_t)bh * DK + cb) * DV + j;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dst[(size_t)i * DV] = sv[i];
+        }
+    }
+    if (tid == 0) bulk_wait_group0();
+    if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
+}
+
+template <bool GENERAL>
+__global__ void __launch_bounds__(NT, 1)
+fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
+                 const __grid_constant__ CUtensorMap tm_o, ChunkParams cp, ScanParams sp)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t tm = 0;
+    bool timed_out = chunk_body<GENERAL, false, true>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, cp, sm, tm);
+    if (!timed_out && (int)blockIdx.x < cp.BH) fused_scan(tm_o, sp, cp.flags, sm, tm, blockIdx.x, timed_out);
+    tc_fence_before_sync();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tm, TM_COLS);
+}
+
 // ---------------------------------------------------------------- host side
 }  // namespace
 
@@ -1272,10 +1553,13 @@ bool forward_tc_supported(const FwdArgs &a)
     return a.bf16 && a.dk == DK && a.dv == DV && a.T > 0 && encode_fn() != nullptr;
 }
 
+// Dense: the slots, the gammas, then the fused kernel's queue counter (16 bytes) and task flags.
+static size_t fused_sync_bytes(size_t ntasks) { return (16 + ntasks * 4 + 255) / 256 * 256; }
+
 size_t forward_tc_workspace_bytes(int B, int T, int H)
 {
     const size_t ntasks = (size_t)B * H * ((T + C - 1) / C);
-    return ntasks * (SLOT_BYTES + GAMMA_BYTES);
+    return ntasks * (SLOT_BYTES + GAMMA_BYTES) + fused_sync_bytes(ntasks);
 }
 
 // Packed sequences: at most H (ceil(T / 64) + N) tasks (each sequence adds at most one
@@ -1285,6 +1569,20 @@ static size_t varlen_task_capacity(int N, int T, int H) { return (size_t)H * ((T
 size_t forward_tc_varlen_workspace_bytes(int N, int T, int H)
 {
     return varlen_task_capacity(N, T, H) * (SLOT_BYTES + GAMMA_BYTES) + (((size_t)N + 2) * sizeof(int) + 255) / 256 * 256;
+}
+
+// The block's output epilogue, a pass over o after the forward's kernels (when asked for).
+static cudaError_t launch_output_epilogue(const FwdArgs &a, int nsm, cudaStream_t s)
+{
+    if (!a.out_gate && !a.norm_weight) return cudaSuccess;
+    const long long nrows = (long long)(a.cu_seqlens ? 1 : a.B) * a.T * a.H;
+    if (nrows == 0) return cudaSuccess;
+    const long long blocks = (nrows + 31) / 32;  // 8 warps of four rows per block
+    const int eg = (int)(blocks < (long long)nsm * 16 ? blocks : (long long)nsm * 16);
+    output_epilogue_kernel<<<eg, 256, 0, s>>>(static_cast<__nv_bfloat16 *>(a.o),
+                                              static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight,
+                                              a.norm_eps, nrows);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
@@ -1328,6 +1626,51 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
                    ntasks,      ws,        a.status,   a.cu_seqlens,
                    cu_chunks,   ntasks_dev, a.gates,   static_cast<const __nv_bfloat16 *>(a.b),
                    static_cast<const __nv_bfloat16 *>(a.w), a.bwd_ext, debug_giveup_flag()};
+    // The fused kernel (chunk tasks, then the scans on B H of the CTAs) when the scans leave
+    // enough SMs to the queue's tail: dense sequences, nothing saved for a backward, and a
+    // workspace with room for the queue and flags.
+    const int BH = a.B * a.H;
+    int coop = 0;
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    const bool fused = !varlen && !bwd && !a.chunks_only && !a.saved_states && coop != 0 && !debug_unfused_flag() &&
+                       BH + kFusedMinQueueCtas <= nsm &&
+                       a.workspace_bytes >= forward_tc_workspace_bytes(a.B, a.T, a.H);
+    if (fused) {
+        void (*fk)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                   const CUtensorMap, const CUtensorMap, ChunkParams, ScanParams) =
+            general ? fwd_fused_kernel<true> : fwd_fused_kernel<false>;
+        e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fk, NT, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        unsigned char *sync = ws + (size_t)ntasks * (SLOT_BYTES + GAMMA_BYTES);
+        e = cudaMemsetAsync(sync, 0, fused_sync_bytes(ntasks), s);
+        if (e != cudaSuccess) return e;
+        cp.queue = reinterpret_cast<int *>(sync);
+        cp.flags = reinterpret_cast<unsigned *>(sync + 16);
+        cp.BH = BH;
+        // The scans start once (nsm - BH) CTAs can finish the rest of the queue in about the
+        // time of one scan: rest ~ (nsm - BH) * NC * (scan time per chunk / chunk task time).
+        const double rest = (double)(nsm - BH) * NC * kScanToTaskTime;
+        cp.switch_at = rest >= ntasks ? 0 : ntasks - (int)rest;
+        ScanParams sp{a.B, a.T, a.H, NC, ntasks, ws, a.S0, a.S_T, nullptr, a.status, nullptr, nullptr,
+                      static_cast<__nv_bfloat16 *>(a.o)};
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(nsm);
+        cfg.blockDim = dim3(NT);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the scans wait on the others
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, fk, mq, mk, mb, mv, mw, mla, mo, cp, sp);
+        if (e != cudaSuccess) return e;
+        return launch_output_epilogue(a, nsm, s);
+    }
     const int grid = ntasks < nsm ? ntasks : nsm;
     chunk<<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
     e = cudaGetLastError();
@@ -1346,15 +1689,8 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, fwd_scan_kernel, mo, sp);
-    if (e != cudaSuccess || (!a.out_gate && !a.norm_weight)) return e;
-    const long long nrows = (long long)(varlen ? 1 : a.B) * a.T * a.H;
-    if (nrows == 0) return cudaSuccess;
-    const long long blocks = (nrows + 31) / 32;  // 8 warps of four rows per block
-    const int eg = (int)(blocks < (long long)nsm * 16 ? blocks : (long long)nsm * 16);
-    output_epilogue_kernel<<<eg, 256, 0, s>>>(static_cast<__nv_bfloat16 *>(a.o),
-                                              static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight,
-                                              a.norm_eps, nrows);
-    return cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_output_epilogue(a, nsm, s);
 }
 
 }  // namespace gdr2

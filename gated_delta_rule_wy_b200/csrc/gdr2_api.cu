@@ -48,6 +48,7 @@ unsigned *status_ptr(int dev)
 }
 
 std::atomic<int> g_debug_giveup{0};
+std::atomic<int> g_debug_unfused{0};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -122,6 +123,7 @@ gdr2_status launched(cudaError_t e, const char *what)
 
 namespace gdr2 {
 int debug_giveup_flag() { return g_debug_giveup.load(); }
+int debug_unfused_flag() { return g_debug_unfused.load(); }
 }  // namespace gdr2
 
 extern "C" {
@@ -129,6 +131,8 @@ extern "C" {
 int gdr2_abi_version(void) { return GDR2_ABI_VERSION; }
 
 void gdr2_debug_force_timeout(int enable) { g_debug_giveup.store(enable != 0 ? 1 : 0); }
+
+void gdr2_debug_forward_unfused(int enable) { g_debug_unfused.store(enable != 0 ? 1 : 0); }
 
 gdr2_status gdr2_debug_recip(const float *x, float *y, long long n, void *stream)
 {

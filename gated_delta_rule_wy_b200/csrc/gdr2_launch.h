@@ -98,6 +98,7 @@ struct SegArgs {
 
 cudaError_t launch_segment_states(const SegArgs &a, cudaStream_t s);
 int debug_giveup_flag();  // gdr2_debug_force_timeout's setting
+int debug_unfused_flag();  // gdr2_debug_forward_unfused's setting
 cudaError_t launch_recip_eval(const float *x, float *y, long long n, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t s);
 cudaError_t launch_gate_activations(const ActArgs &a, cudaStream_t s);

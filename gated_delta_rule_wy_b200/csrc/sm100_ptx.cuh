@@ -129,6 +129,39 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy accesses of global memory with its async-proxy ones (bulk
+// copies): between a completed bulk store and a flag release, and between a flag acquire and a
+// bulk load.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// A 32-bit flag in global memory, released / acquired at GPU scope.
+__device__ __forceinline__ void st_release_gpu(unsigned *f, unsigned v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *f)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+// Waits until *f is nonzero, for at most limit_ns; false if it gave up.
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned *f, uint64_t limit_ns)
+{
+    if (ld_acquire_gpu(f) != 0u) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(f) != 0u) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+}
+
 // ---------------------------------------------------------------- TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols)
 {

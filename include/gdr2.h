@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define GDR2_ABI_VERSION 8
+#define GDR2_ABI_VERSION 9
 #define GDR2_CHUNK 64 /* tokens per chunk of the chunkwise forward */
 
 typedef enum {
@@ -115,7 +115,10 @@ size_t gdr2_forward_workspace_bytes(int B, int T, int H, int dk, int dv, gdr2_dt
  * scratch: workspace of at least gdr2_forward_workspace_bytes(...) bytes,
  *      256-byte aligned (may be NULL when that size is 0); contents on entry
  *      do not matter. The bf16 path at d = 128 keeps each chunk's
- *      state-independent intermediates there (88.5 KiB per (b, h, chunk)).
+ *      state-independent intermediates there (88.5 KiB per (b, h, chunk)),
+ *      then a task queue counter and one ready flag per chunk for the fused
+ *      kernel (chunk tasks and the per-(b, h) scans in one launch, used when
+ *      B H leaves at least 32 SMs to the chunk tasks; the call clears them).
  * Input and output buffers must not overlap (S0 == S_T is allowed).
  */
 gdr2_status gdr2_forward(int B, int T, int H, int dk, int dv, gdr2_dtype dt,
@@ -395,6 +398,15 @@ gdr2_status gdr2_sync_status(void *stream);
  * concurrent callers see it too. 0 (the default) turns it off.
  */
 void gdr2_debug_force_timeout(int enable);
+
+/*
+ * gdr2_debug_forward_unfused -- while `enable` is nonzero, every dense bf16
+ * forward runs as its two kernels (all chunk tasks, then one scan per
+ * (sequence, head)) even where it would otherwise run as the fused kernel
+ * (chunk tasks and scans in one cooperative launch). Both give the same bits;
+ * the hook lets a test compare them. Process-wide; 0 (the default) turns it off.
+ */
+void gdr2_debug_forward_unfused(int enable);
 
 /*
  * gdr2_debug_recip -- y[i] = the device reciprocal the kernels use in place of

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gdr2_abi_version() == 8
+    assert lib.gdr2_abi_version() == 9
 
 
 NULL11 = [None] * 11 + [ctypes.c_size_t(0), None]  # 11 tensors + workspace bytes + stream
@@ -150,7 +150,10 @@ def test_noalloc_backward_rejects_oversized_problems_on_the_host(lib):
 def test_forward_workspace_query_and_check(lib):
     # bf16 at d = 128 runs on the tensor cores and needs the chunk workspace
     n = lib.gdr2_forward_workspace_bytes(4, 4096, 16, 128, 128, 1)
-    assert n == 4 * 16 * 64 * (90112 + 512)
+    ntasks = 4 * 16 * 64
+    # per task a slot and its gamma, then the fused kernel's queue counter (16 bytes) and one
+    # 4-byte flag per task, rounded up to 256 bytes
+    assert n == ntasks * (90112 + 512) + (16 + 4 * ntasks + 255) // 256 * 256
     assert lib.gdr2_forward_workspace_bytes(4, 4096, 16, 128, 128, 0) == 0  # fp32: CUDA cores
     assert lib.gdr2_forward_workspace_bytes(4, 4096, 16, 64, 64, 1) == 0
     p = [ctypes.c_void_p(0x10000)] * 11  # 10 tensors + the workspace
