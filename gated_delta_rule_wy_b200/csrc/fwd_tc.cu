@@ -116,6 +116,7 @@ struct Misc {
     uint32_t tmem_base;
     int q_next;      // fused kernel: the queue index this CTA takes next
     int pad[2];
+    int loc_next[4];  // packed sequences: where the next task's chunk lives (h, t0, bb, Cn)
     float gC[DK];    // exp(G_C)
     float eg0[DK];   // W combine factor of half-chunk 0: exp(g_0)
     float eg1[DK];   // ... of half-chunk 1: exp(g_1)
@@ -182,11 +183,17 @@ __device__ __forceinline__ ChunkLoc locate_chunk(const ChunkParams &p, int task)
 
 // Packed sequences: chunk offsets per sequence and the task count, after checking that
 // cu_seqlens runs from 0 to T without decreasing. If it does not, no task runs (the count
-// is 0 and every offset 0) and the status word records it. One block.
+// is 0 and every offset 0) and the status word records it. Also the order in which the scan
+// kernel takes the sequences: longest first (a scan's time is its chunk count, so the long
+// ones must not start last), ties by index; up to kOrderMax sequences, by a bitonic sort in
+// shared memory, else the given order. One block.
+constexpr int kOrderMax = 2048;
+
 __global__ void __launch_bounds__(1024) varlen_prefix_kernel(const int *cu, int N, int T, int H, int *cu_chunks,
-                                                             int *ntasks, unsigned *status)
+                                                             int *ntasks, int *order, unsigned *status)
 {
     __shared__ int part[1024];
+    __shared__ int key[kOrderMax], idx[kOrderMax];
     const int tid = threadIdx.x;
     const int per = (N + 1023) / 1024;
     const int i0 = tid * per, i1 = min(N, i0 + per);
@@ -217,6 +224,33 @@ __global__ void __launch_bounds__(1024) varlen_prefix_kernel(const int *cu, int 
         *ntasks = bad ? 0 : H * part[1023];
         if (bad) atomicOr(status, kStatusBadSeqlens);
     }
+    if (N > kOrderMax || bad) {
+        for (int i = tid; i < N; i += 1024) order[i] = i;
+        return;
+    }
+    int P = 1;
+    while (P < N) P <<= 1;
+    for (int i = tid; i < P; i += 1024) {
+        key[i] = i < N ? (max(cu[i + 1] - cu[i], 0) + C - 1) / C : -1;  // padding sorts last
+        idx[i] = i;
+    }
+    __syncthreads();
+    // "a before b": more chunks, or as many and a smaller index
+    auto before = [&](int a, int b) { return key[a] > key[b] || (key[a] == key[b] && idx[a] < idx[b]); };
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += 1024) {
+                const int l = i ^ j;
+                if (l > i && (((i & k) == 0) ? before(l, i) : before(i, l))) {
+                    const int tk = key[i], ti = idx[i];
+                    key[i] = key[l]; idx[i] = idx[l];
+                    key[l] = tk; idx[l] = ti;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = tid; i < N; i += 1024) order[i] = idx[i];
 }
 
 // TMEM columns of the chunk kernel
@@ -259,8 +293,17 @@ __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtens
     const int ntasks = (GENERAL && p.cu_seqlens) ? *p.ntasks_dev : p.ntasks;
     const bool bsc = GENERAL && (p.gates & kGateScalarB) != 0, wsc = GENERAL && (p.gates & kGateScalarW) != 0;
     const uint32_t tx_bytes = TX_BYTES - (bsc ? 16384u : 0u) - (wsc ? 16384u : 0u);
+    // Packed sequences: a task's location takes a binary search over cu_chunks (dependent global
+    // loads), so the thread that issues its copies also leaves it in shared memory for the rest.
+    const bool varlen = GENERAL && p.cu_seqlens;
     auto issue_loads = [&](int task) {
         const ChunkLoc L = locate_chunk<GENERAL>(p, task);
+        if (varlen) {
+            ms.loc_next[0] = L.h;
+            ms.loc_next[1] = L.t0;
+            ms.loc_next[2] = L.bb;
+            ms.loc_next[3] = L.Cn;
+        }
         mbar_arrive_expect_tx(&ms.bar_tma, tx_bytes);
         tma_load_4d(sm + OFF_STG_Q, &tm_q, &ms.bar_tma, 0, L.h, L.t0, L.bb);
         tma_load_4d(sm + OFF_STG_K, &tm_k, &ms.bar_tma, 0, L.h, L.t0, L.bb);
@@ -285,6 +328,7 @@ __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtens
         q0 = ms.q_next;
     }
     if (!timed_out && tid == 0 && q0 < ntasks) issue_loads(task_of(q0));
+    if (varlen) __syncthreads();  // the first task's location
     // the scan kernel may be scheduled now: its CTAs take an SM only once this (persistent) CTA
     // has left it, and they read the workspace only after this whole grid has completed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -312,7 +356,15 @@ __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtens
     int prev_task = -1;  // FUSED: the task finished last, whose flag is still to be set
     for (int qi = q0; qi < ntasks && !timed_out;) {
         const int task = task_of(qi);
-        const ChunkLoc loc = locate_chunk<GENERAL>(p, task);
+        ChunkLoc loc;
+        if (varlen) {  // left by the thread that issued this task's copies (barriers since)
+            loc.h = ms.loc_next[0];
+            loc.t0 = ms.loc_next[1];
+            loc.bb = ms.loc_next[2];
+            loc.Cn = ms.loc_next[3];
+        } else {
+            loc = locate_chunk<GENERAL>(p, task);
+        }
         const int Cn = loc.Cn;
         // a scalar gate: this thread's four rows (t = tid / 16 + 16 k), read while the copies land
         static_assert(C * 16 == 4 * NT, "four 16-byte pieces of a staging row set per thread");
@@ -1048,6 +1100,7 @@ struct ScanParams {
     const int *cu_seqlens;  // packed sequences (null when dense), as in ChunkParams
     const int *cu_chunks;
     __nv_bfloat16 *o;       // for the row-by-row store of a packed sequence's last, partial tile
+    const int *seq_order = nullptr;  // packed: CTA group g (H CTAs) scans sequence seq_order[g]
 };
 
 constexpr uint32_t SC_SMEM = SC_MISC + 1280 + 1024;  // + alignment slack
@@ -1062,8 +1115,9 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quarter = warp & 3, colhalf = warp >> 2;
-    const int bh = blockIdx.x;  // (sequence, head)
-    const int bb = bh / p.H, h = bh % p.H;
+    int bh = blockIdx.x;  // (sequence, head)
+    int bb = bh / p.H;
+    const int h = bh % p.H;
     const int c0 = colhalf * 64;  // this thread's 64 state columns c (S^T columns)
     // this (sequence, head)'s chunks: count, first task, first token and length, map batch
     int NC = p.NC, tstart = 0, len = p.T, tb = bb;
@@ -1090,6 +1144,8 @@ fwd_scan_kernel(const __grid_constant__ CUtensorMap tm_o, ScanParams p)
     // tail; the workspace is read only after that grid has completed and flushed its memory.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (p.cu_seqlens) {
+        bb = p.seq_order[bb];  // the longest sequences first
+        bh = bb * p.H + h;
         NC = p.cu_chunks[bb + 1] - p.cu_chunks[bb];
         base = (size_t)p.H * p.cu_chunks[bb] + (size_t)h * NC;
         tstart = p.cu_seqlens[bb];
@@ -1568,7 +1624,9 @@ static size_t varlen_task_capacity(int N, int T, int H) { return (size_t)H * ((T
 
 size_t forward_tc_varlen_workspace_bytes(int N, int T, int H)
 {
-    return varlen_task_capacity(N, T, H) * (SLOT_BYTES + GAMMA_BYTES) + (((size_t)N + 2) * sizeof(int) + 255) / 256 * 256;
+    // then cu_chunks (N + 1 ints), the task count and the scan order (N ints)
+    return varlen_task_capacity(N, T, H) * (SLOT_BYTES + GAMMA_BYTES) +
+           ((2 * (size_t)N + 2) * sizeof(int) + 255) / 256 * 256;
 }
 
 // The block's output epilogue, a pass over o after the forward's kernels (when asked for).
@@ -1614,11 +1672,13 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     const int NC = (a.T + C - 1) / C;
     const int ntasks = varlen ? (int)varlen_task_capacity(a.B, a.T, a.H) : a.B * a.H * NC;
     unsigned char *ws = static_cast<unsigned char *>(a.workspace);
-    int *cu_chunks = nullptr, *ntasks_dev = nullptr;
+    int *cu_chunks = nullptr, *ntasks_dev = nullptr, *seq_order = nullptr;
     if (varlen) {
         cu_chunks = reinterpret_cast<int *>(ws + (size_t)ntasks * (SLOT_BYTES + GAMMA_BYTES));
         ntasks_dev = cu_chunks + a.B + 1;
-        varlen_prefix_kernel<<<1, 1024, 0, s>>>(a.cu_seqlens, a.B, a.T, a.H, cu_chunks, ntasks_dev, a.status);
+        seq_order = ntasks_dev + 1;
+        varlen_prefix_kernel<<<1, 1024, 0, s>>>(a.cu_seqlens, a.B, a.T, a.H, cu_chunks, ntasks_dev, seq_order,
+                                                 a.status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1678,6 +1738,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     ScanParams sp{a.B,          a.T,          a.H,    NC,       ntasks,    ws,
                   a.S0,         a.S_T,        a.saved_states, a.status, a.cu_seqlens, cu_chunks,
                   static_cast<__nv_bfloat16 *>(a.o)};
+    sp.seq_order = seq_order;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.H);
     cfg.blockDim = dim3(SC_NT);

@@ -51,9 +51,22 @@ def test_single_sequence_and_one_token_sequences():
     _check_against_oracle([1, 1, 1, 2, 1], H=3, seed=73)
 
 
+def test_lengths_in_ascending_order():
+    # the scans take the sequences longest first: here the reverse of their order in memory
+    _check_against_oracle([1, 5, 63, 64, 100, 300, 700], H=3, seed=77)
+
+
+def test_more_sequences_than_the_scan_order_sort_takes():
+    # beyond 2048 sequences the scans take them in the given order
+    rng = np.random.default_rng(78)
+    lens = rng.integers(0, 24, 2100)
+    lens[[5, 1000, 2099]] = [200, 130, 65]
+    _check_against_oracle(lens.tolist(), H=1, seed=78, which=[0, 5, 17, 1000, 1500, 2098, 2099])
+
+
 def test_equal_lengths_match_the_dense_forward_exactly():
-    """B equal sequences packed, against the [B, T, H, D] forward: the same kernels on
-    the same chunks, so the same bits (including the saved chunk states)."""
+    """B equal sequences packed, against the [B, T, H, D] forward: the same chunk and scan
+    steps on the same chunks, so the same bits (including the saved chunk states)."""
     B, T, H = 3, 200, 4
     x = I.make_forward_inputs(B=B, H=H, T=T, dk=128, dv=128, dtype=torch.bfloat16, decay_shift=2.0, seed=74,
                               with_S0=True)
