@@ -22,7 +22,9 @@
 // Launches (one stream):
 //   1. the forward's chunk kernel (backward instance): the workspace slots ([Q'; M], K~,
 //      U~, P, gamma) plus T and W; and, without saved states, the forward's scan kernel
-//      for the chunk-entry states;
+//      for the chunk-entry states. With saved states, where B H leaves 32 SMs to the chunk
+//      tasks, steps 1 and 2 are one cooperative launch (bwd_front_kernel, fwd_tc.cu): the
+//      chunk tasks from the last chunk back, then the reverse scans on B H of the CTAs;
 //   2. reverse scan (one CTA per (batch, head), chunks last to first): dS^T in TMEM in
 //      fp32; per chunk a bf16 image of dS' for the chunk kernels, then
 //      dS^T = dS'^T Diag(gamma) + dS'^T M + dO^T Q' as 12 MMAs;
@@ -42,6 +44,7 @@
 #include "gdr2_launch.h"
 #include "sm100_ptx.cuh"
 #include "tc_common.cuh"
+#include "bwd_rscan.cuh"
 
 namespace gdr2 {
 namespace {
@@ -49,7 +52,6 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr uint32_t DS_IMG = 32768;   // dS'^T in bf16, [j rows 128][c: 2 blocks of 64]
 constexpr uint32_t DPA_IMG = 16384;  // [dA_0; dP_0; dA_1; dP_1] rows t (32 each) x 64 i, bf16
 constexpr uint32_t X_ARR = 16384;    // one [64 t][128 c] bf16 array of the value kernel's record
 constexpr uint32_t XREC_BYTES = 3 * X_ARR + 64 * 4 + 128 * 4;  // 3 arrays, dP_tt [64], sum_j dS' S [128]
@@ -57,32 +59,7 @@ constexpr uint32_t XREC_BYTES = 3 * X_ARR + 64 * 4 + 128 * 4;  // 3 arrays, dP_t
 __host__ __device__ constexpr size_t al1k(size_t x) { return (x + 1023) & ~size_t(1023); }
 
 // ============================================================ reverse scan
-constexpr int RS_NT = 288;                        // 8 TMEM warps + the MMA warp
-constexpr uint32_t RS_BUF = 65536;                // one chunk: [Q'; M] (49152) then the dO image
-constexpr uint32_t RS_DO = 49152;
-constexpr uint32_t RS_DS = 2 * RS_BUF;            // two dS'^T images
-constexpr uint32_t RS_MISC = RS_DS + 2 * DS_IMG;  // 196608
-constexpr uint32_t RS_SA = 256;                   // TMEM: regions at 0 and 128, bf16 copy at 256
-
-struct RsMisc {
-    uint64_t bar_full[2];
-    uint64_t bar_mma;
-    uint32_t tmem_base;
-    int pad;
-    alignas(16) float gam[2][DK];
-};
-constexpr uint32_t RS_SMEM = RS_MISC + sizeof(RsMisc) + 1024;
-static_assert(offsetof(RsMisc, gam) % 16 == 0, "gamma rows are bulk-copy destinations");
-
-struct RsParams {
-    int B, T, H, NC, ntasks;
-    const unsigned char *ws;  // slots, then gammas
-    const float *dS_T;        // [B][H][DK][DV] or null (zero)
-    float *gS0;               // [B][H][DK][DV] or null
-    unsigned char *dsc;       // [ntasks][DS_IMG]: dS'^T of every chunk, bf16 images
-    unsigned *status;
-};
-
+// (definitions and the fused kernel's eight-warp version in bwd_rscan.cuh)
 __global__ void __launch_bounds__(RS_NT, 1) bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_do, RsParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -1035,7 +1012,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 struct BwdTcLayout {
-    size_t ntasks, ext, dsc, dpa, xrec, states, o, total;
+    size_t ntasks, ext, dsc, dpa, xrec, states, o, sync, total;
 };
 
 BwdTcLayout bwd_tc_layout(int B, int T, int H)
@@ -1056,6 +1033,8 @@ BwdTcLayout bwd_tc_layout(int B, int T, int H)
     off += al1k(L.ntasks * DK * DV * sizeof(float));
     L.o = off;       // the forward's output, unused
     off += al1k((size_t)B * T * H * DV * 2);
+    L.sync = off;    // the fused front's queue counter and task flags
+    off += al1k(fused_sync_bytes_for(L.ntasks));
     L.total = off;
     return L;
 }
@@ -1094,8 +1073,18 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     fa.norm_eps = 0.f;
     fa.bwd_ext = ws + L.ext;
     fa.chunks_only = a.saved_states != nullptr;
-    cudaError_t e = launch_forward_tc(fa, s);
-    if (e != cudaSuccess) return e;
+    // with saved states, the chunk tasks and the reverse scans (step 2) as one launch where it fits
+    bool front_fused = false;
+    cudaError_t e = cudaSuccess;
+    if (a.saved_states) {
+        const BwdFrontArgs r{a.dO, a.dS_T, a.gS0, ws + L.dsc, ws + L.sync};
+        e = launch_backward_front_fused(fa, r, s, &front_fused);
+        if (e != cudaSuccess) return e;
+    }
+    if (!front_fused) {
+        e = launch_forward_tc(fa, s);
+        if (e != cudaSuccess) return e;
+    }
 
     const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
     CUtensorMap mdo, mq, mk, mb, mla, mgq, mgk, mgb, mgla;
@@ -1116,12 +1105,14 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     const int grid = ntasks < nsm ? ntasks : nsm;
 
     // 2. reverse scan
-    e = cudaFuncSetAttribute(bwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RS_SMEM);
-    if (e != cudaSuccess) return e;
-    RsParams rp{a.B, a.T, a.H, NC, ntasks, ws, a.dS_T, a.gS0, ws + L.dsc, a.status};
-    bwd_scan_kernel<<<a.B * a.H, RS_NT, RS_SMEM, s>>>(mdo, rp);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (!front_fused) {
+        e = cudaFuncSetAttribute(bwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RS_SMEM);
+        if (e != cudaSuccess) return e;
+        RsParams rp{a.B, a.T, a.H, NC, ntasks, ws, a.dS_T, a.gS0, ws + L.dsc, a.status};
+        bwd_scan_kernel<<<a.B * a.H, RS_NT, RS_SMEM, s>>>(mdo, rp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
 
     // 3. value side
     e = cudaFuncSetAttribute(bwd_value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VA_SMEM);

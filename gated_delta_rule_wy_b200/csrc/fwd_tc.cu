@@ -67,6 +67,7 @@
 #include "gdr2_launch.h"
 #include "sm100_ptx.cuh"
 #include "tc_common.cuh"
+#include "bwd_rscan.cuh"
 
 namespace gdr2 {
 namespace {
@@ -109,6 +110,7 @@ constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
 // ratio of a scan's time per chunk to a chunk task's time that places the switch.
 constexpr int kFusedMinQueueCtas = 32;
 constexpr double kScanToTaskTime = 0.25;
+constexpr double kRevScanToTaskTime = 0.25;  // the same for the backward's front (reverse scans)
 
 struct Misc {
     uint64_t bar_tma;
@@ -260,7 +262,7 @@ constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W
 // The chunk kernel's work. GENERAL: packed sequences and/or scalar gates may be in use; the
 // other instantiation is the dense, vector-gate kernel with those branches compiled away. BWD
 // (dense sequences): T and W of each task also go to p.ext for the backward. FUSED (dense
-// sequences): the first role of the fused kernel -- tasks come from a queue in chunk-major
+// sequences): the first role of the fused forward or backward-front kernel -- tasks come from a queue in chunk-major
 // order, each finished task is published by its flag, and the TMEM allocation is kept for the
 // scan role (tm_out). Returns whether a bounded wait gave up (the same on every thread).
 template <bool GENERAL, bool BWD, bool FUSED>
@@ -268,7 +270,6 @@ __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtens
                                            const CUtensorMap &tm_v, const CUtensorMap &tm_w, const CUtensorMap &tm_la,
                                            const ChunkParams &p, unsigned char *sm, uint32_t &tm_out)
 {
-    static_assert(!FUSED || !BWD, "the fused kernel is the dense forward without the backward's extras");
     Misc &ms = *reinterpret_cast<Misc *>(sm + OFF_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -319,8 +320,13 @@ __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtens
         const bool ok = mbar_wait_bounded(&ms.bar_mma, 0, 1000);
         timed_out = __syncthreads_or(!ok) != 0;
     }
-    // queue index -> task (slot): FUSED takes chunk n of every (sequence, head) before chunk n + 1
-    auto task_of = [&](int qi) -> int { return FUSED ? (qi % p.BH) * p.NC + qi / p.BH : qi; };
+    // queue index -> task (slot): FUSED takes chunk n of every (sequence, head) before chunk n + 1;
+    // FUSED with BWD (for the backward's reverse scans) from the last chunk back
+    auto task_of = [&](int qi) -> int {
+        if (!FUSED) return qi;
+        const int n = qi / p.BH;
+        return (qi % p.BH) * p.NC + (BWD ? p.NC - 1 - n : n);
+    };
     int q0 = blockIdx.x;
     if (FUSED) {
         if (tid == 0) ms.q_next = atomicAdd(p.queue, 1);
@@ -1527,6 +1533,27 @@ fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if ((threadIdx.x >> 5) == 0) tmem_dealloc(tm, TM_COLS);
 }
 
+// ---- the backward's front as one launch: the forward's chunk tasks (backward instance) from
+// the last chunk back, then (CTA b < B H) the reverse scan of (sequence, head) b, each chunk's
+// slot copied once its flag is set. The same residency argument as fwd_fused_kernel.
+template <bool GENERAL>
+__global__ void __launch_bounds__(NT, 1)
+bwd_front_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_la,
+                 const __grid_constant__ CUtensorMap tm_do, ChunkParams cp, RsParams rp)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t tm = 0;
+    bool timed_out = chunk_body<GENERAL, true, true>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, cp, sm, tm);
+    if (!timed_out && (int)blockIdx.x < cp.BH) rscan_role(tm_do, rp, cp.flags, sm, tm, blockIdx.x, timed_out);
+    tc_fence_before_sync();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tm, TM_COLS);
+}
+
 // ---------------------------------------------------------------- host side
 }  // namespace
 
@@ -1752,6 +1779,65 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
     e = cudaLaunchKernelEx(&cfg, fwd_scan_kernel, mo, sp);
     if (e != cudaSuccess) return e;
     return launch_output_epilogue(a, nsm, s);
+}
+
+size_t fused_sync_bytes_for(size_t ntasks) { return fused_sync_bytes(ntasks); }
+
+cudaError_t launch_backward_front_fused(const FwdArgs &a, const BwdFrontArgs &r, cudaStream_t s, bool *launched)
+{
+    *launched = false;
+    if (a.cu_seqlens || !a.bwd_ext || !a.chunks_only || debug_unfused_flag()) return cudaSuccess;
+    int dev = 0, nsm = 148, coop = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    const int BH = a.B * a.H;
+    if (!coop || BH + kFusedMinQueueCtas > nsm) return cudaSuccess;
+    const bool bsc = (a.gates & kGateScalarB) != 0, wsc = (a.gates & kGateScalarW) != 0;
+    CUtensorMap mq, mk, mb, mv, mw, mla, mdo;
+    if (!make_map(&mq, a.q, false, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, false, a.B, a.T, a.H, DK) ||
+        !make_map(&mv, a.v, false, a.B, a.T, a.H, DV) || !make_map(&mla, a.log_alpha, true, a.B, a.T, a.H, DK) ||
+        !make_map(&mdo, r.dO, false, a.B, a.T, a.H, DV, 64, true))
+        return cudaErrorInvalidValue;
+    if (bsc) mb = mq; else if (!make_map(&mb, a.b, false, a.B, a.T, a.H, DK)) return cudaErrorInvalidValue;
+    if (wsc) mw = mq; else if (!make_map(&mw, a.w, false, a.B, a.T, a.H, DV)) return cudaErrorInvalidValue;
+    const bool general = bsc || wsc;
+    void (*fk)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+               const CUtensorMap, const CUtensorMap, ChunkParams, RsParams) =
+        general ? bwd_front_kernel<true> : bwd_front_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fk, NT, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaSuccess;
+    const int NC = (a.T + C - 1) / C;
+    const int ntasks = BH * NC;
+    e = cudaMemsetAsync(r.sync, 0, fused_sync_bytes(ntasks), s);
+    if (e != cudaSuccess) return e;
+    ChunkParams cp{a.B,     a.T,     a.H,      NC,
+                   ntasks,  static_cast<unsigned char *>(a.workspace), a.status, nullptr,
+                   nullptr, nullptr, a.gates,  static_cast<const __nv_bfloat16 *>(a.b),
+                   static_cast<const __nv_bfloat16 *>(a.w), a.bwd_ext, debug_giveup_flag()};
+    cp.queue = reinterpret_cast<int *>(r.sync);
+    cp.flags = reinterpret_cast<unsigned *>(r.sync + 16);
+    cp.BH = BH;
+    const double rest = (double)(nsm - BH) * NC * kRevScanToTaskTime;
+    cp.switch_at = rest >= ntasks ? 0 : ntasks - (int)rest;
+    RsParams rp{a.B, a.T, a.H, NC, ntasks, static_cast<const unsigned char *>(a.workspace), r.dS_T, r.gS0, r.dsc,
+                a.status};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nsm);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the scans wait on the others
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, fk, mq, mk, mb, mv, mw, mla, mdo, cp, rp);
+    if (e == cudaSuccess) *launched = true;
+    return e;
 }
 
 }  // namespace gdr2

@@ -97,6 +97,20 @@ struct SegArgs {
 };
 
 cudaError_t launch_segment_states(const SegArgs &a, cudaStream_t s);
+
+// The backward's first two steps as one cooperative launch (fwd_tc.cu): the forward's chunk
+// tasks (backward instance, T and W to fa.bwd_ext; chunk-major from the last chunk) and the
+// reverse scans of the state gradient. Runs only for dense sequences with saved chunk states
+// (fa.chunks_only) where B H leaves 32 SMs to the chunk tasks; *launched says whether it ran.
+struct BwdFrontArgs {
+    const void *dO;       // [B][T][H][dv] bf16
+    const float *dS_T;    // [B][H][dk][dv] or null
+    float *gS0;           // [B][H][dk][dv] or null
+    unsigned char *dsc;   // the dS'^T images, one per task
+    unsigned char *sync;  // fused_sync_bytes_for(tasks) bytes: the queue counter and task flags
+};
+cudaError_t launch_backward_front_fused(const FwdArgs &fa, const BwdFrontArgs &r, cudaStream_t s, bool *launched);
+size_t fused_sync_bytes_for(size_t ntasks);
 int debug_giveup_flag();  // gdr2_debug_force_timeout's setting
 int debug_unfused_flag();  // gdr2_debug_forward_unfused's setting
 cudaError_t launch_recip_eval(const float *x, float *y, long long n, cudaStream_t s);

@@ -403,8 +403,10 @@ void gdr2_debug_force_timeout(int enable);
  * gdr2_debug_forward_unfused -- while `enable` is nonzero, every dense bf16
  * forward runs as its two kernels (all chunk tasks, then one scan per
  * (sequence, head)) even where it would otherwise run as the fused kernel
- * (chunk tasks and scans in one cooperative launch). Both give the same bits;
- * the hook lets a test compare them. Process-wide; 0 (the default) turns it off.
+ * (chunk tasks and scans in one cooperative launch), and gdr2_backward with
+ * saved states runs its chunk tasks and reverse scans as two launches instead
+ * of one. Both ways give the same bits; the hook lets a test compare them.
+ * Process-wide; 0 (the default) turns it off.
  */
 void gdr2_debug_forward_unfused(int enable);
 

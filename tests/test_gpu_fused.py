@@ -82,3 +82,41 @@ def test_fused_forward_with_scalar_gates_is_bitwise_the_two_kernel_forward(scala
     finally:
         lib.gdr2_debug_forward_unfused(0)
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+BWD_CASES = [
+    dict(B=1, H=2, T=200, seed=87, with_S0=True, dS_T=True),   # ragged tail, both scans switch at once
+    dict(B=2, H=16, T=4096, seed=88, with_S0=False, dS_T=False),  # the benchmarked backward
+    dict(B=2, H=4, T=1500, seed=89, with_S0=True, dS_T=True, scalar="bw"),
+]
+
+
+@pytest.mark.parametrize("c", BWD_CASES, ids=lambda c: f"B{c['B']}_H{c['H']}_T{c['T']}{'_' + c.get('scalar', '')}")
+def test_fused_backward_front_is_bitwise_the_two_launch_front(c):
+    # with saved states the backward's chunk tasks and reverse scans run as one cooperative launch
+    # (chunk-major from the last chunk); every gradient must be the same bits as with the two
+    # launches it replaces
+    from gated_delta_rule_wy_b200 import gdr2_backward
+    lib = binding.load_library()
+    x = I.make_forward_inputs(B=c["B"], H=c["H"], T=c["T"], dk=128, dv=128, dtype=torch.bfloat16, seed=c["seed"],
+                              with_S0=c["with_S0"]).to("cuda")
+    b = x.b[..., 0].contiguous() if "b" in c.get("scalar", "") else x.b
+    w = x.w[..., 0].contiguous() if "w" in c.get("scalar", "") else x.w
+    dO = I.make_upstream_grad(c["B"], c["T"], c["H"], 128, c["seed"], dtype=torch.bfloat16).cuda()
+    dS_T = (torch.randn((c["B"], c["H"], 128, 128), generator=torch.Generator().manual_seed(c["seed"])) * 0.1).cuda() \
+        if c["dS_T"] else None
+    _, _, saved = gdr2_forward(x.q, x.k, x.v, x.log_alpha, b, w, x.S0, save_states=True)
+    g1 = gdr2_backward(x.q, x.k, x.v, x.log_alpha, b, w, dO, x.S0, dS_T, saved)
+    gdr2_sync_status()
+    lib.gdr2_debug_forward_unfused(1)
+    try:
+        g2 = gdr2_backward(x.q, x.k, x.v, x.log_alpha, b, w, dO, x.S0, dS_T, saved)
+        gdr2_sync_status()
+    finally:
+        lib.gdr2_debug_forward_unfused(0)
+    for name in g1:
+        if g1[name] is None:
+            assert g2[name] is None
+            continue
+        assert torch.isfinite(g1[name].float()).all(), name
+        assert torch.equal(g1[name], g2[name]), f"{name} differs in {(g1[name] != g2[name]).sum().item()} elements"
