@@ -16,11 +16,14 @@ The JSON line carries:
   e2e                  same metric through the C ABI with pinned HOST buffers:
                        host->device copy of the inputs, the forward, device->host
                        copy of o and S_T, all inside the timed region
-  roofline             HBM roofline of the forward kernel (algorithmic bytes / time)
+  roofline             HBM roofline of the forward call (algorithmic bytes / time); at
+                       this size the call is one kernel, the fused chunk-and-scan launch
   tensor               algorithmic FLOP/s against the dense bf16 peak
   components           decode step (256 seq x 16 heads, fp32 state), backward
-                       (B=2, T=4096) and the sequence-length sweep (65,536 tokens
-                       per call, T = 2048 .. 32768), each with its own figures
+                       (B=2, T=4096, with and without saved states), the sequence-length
+                       sweep (65,536 tokens per call, T = 2048 .. 32768), packed sequences,
+                       scalar (KDA) gates, the block's output epilogue and prologue, each
+                       with its own figures
   cpu_baseline         the fp64 oracle on the host cores (rank 0, N = 1)
   clocks               SM clocks and throttle reasons sampled during the timed region
 `--impl reference` times the oracle itself on the same workload (sampled heads).
