@@ -1073,6 +1073,7 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     fa.norm_eps = 0.f;
     fa.bwd_ext = ws + L.ext;
     fa.chunks_only = a.saved_states != nullptr;
+    fa.fused_sync = ws + L.sync;  // without saved states: the forward's fused launch keeps T and W
     // with saved states, the chunk tasks and the reverse scans (step 2) as one launch where it fits
     bool front_fused = false;
     cudaError_t e = cudaSuccess;

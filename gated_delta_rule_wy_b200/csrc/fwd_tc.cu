@@ -265,7 +265,7 @@ constexpr uint32_t CK_Q = CK_W0;  // Q' - Q^ (M = 64 layout, 128 columns) over W
 // sequences): the first role of the fused forward or backward-front kernel -- tasks come from a queue in chunk-major
 // order, each finished task is published by its flag, and the TMEM allocation is kept for the
 // scan role (tm_out). Returns whether a bounded wait gave up (the same on every thread).
-template <bool GENERAL, bool BWD, bool FUSED>
+template <bool GENERAL, bool BWD, bool FUSED, bool REV = false>
 __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_b,
                                            const CUtensorMap &tm_v, const CUtensorMap &tm_w, const CUtensorMap &tm_la,
                                            const ChunkParams &p, unsigned char *sm, uint32_t &tm_out)
@@ -321,11 +321,11 @@ __device__ __forceinline__ bool chunk_body(const CUtensorMap &tm_q, const CUtens
         timed_out = __syncthreads_or(!ok) != 0;
     }
     // queue index -> task (slot): FUSED takes chunk n of every (sequence, head) before chunk n + 1;
-    // FUSED with BWD (for the backward's reverse scans) from the last chunk back
+    // REV (for the backward's reverse scans) from the last chunk back
     auto task_of = [&](int qi) -> int {
         if (!FUSED) return qi;
         const int n = qi / p.BH;
-        return (qi % p.BH) * p.NC + (BWD ? p.NC - 1 - n : n);
+        return (qi % p.BH) * p.NC + (REV ? p.NC - 1 - n : n);
     };
     int q0 = blockIdx.x;
     if (FUSED) {
@@ -1429,6 +1429,14 @@ __device__ __forceinline__ void fused_scan(const CUtensorMap &tm_o, const ScanPa
         {
             float s0[32], s1[32];
             tmem_ld32x2(tm_lane + rg_prev + SC_ST + c0, tm_lane + rg_prev + SC_ST + c0 + 32, s0, s1);
+            if (p.saved_states) {  // the state entering chunk n, for the backward
+                float *dst = p.saved_states + ((base + n) * DK + c0) * DV + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    dst[(size_t)i * DV] = s0[i];
+                    dst[(size_t)(32 + i) * DV] = s1[i];
+                }
+            }
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -1515,7 +1523,7 @@ __device__ __forceinline__ void fused_scan(const CUtensorMap &tm_o, const ScanPa
     if (timed_out && tid == 0) atomicOr(p.status, kStatusTimeout);
 }
 
-template <bool GENERAL>
+template <bool GENERAL, bool BWD>
 __global__ void __launch_bounds__(NT, 1)
 fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
@@ -1526,7 +1534,7 @@ fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint32_t tm = 0;
-    bool timed_out = chunk_body<GENERAL, false, true>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, cp, sm, tm);
+    bool timed_out = chunk_body<GENERAL, BWD, true>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, cp, sm, tm);
     if (!timed_out && (int)blockIdx.x < cp.BH) fused_scan(tm_o, sp, cp.flags, sm, tm, blockIdx.x, timed_out);
     tc_fence_before_sync();
     __syncthreads();
@@ -1547,7 +1555,7 @@ bwd_front_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint32_t tm = 0;
-    bool timed_out = chunk_body<GENERAL, true, true>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, cp, sm, tm);
+    bool timed_out = chunk_body<GENERAL, true, true, true>(tm_q, tm_k, tm_b, tm_v, tm_w, tm_la, cp, sm, tm);
     if (!timed_out && (int)blockIdx.x < cp.BH) rscan_role(tm_do, rp, cp.flags, sm, tm, blockIdx.x, timed_out);
     tc_fence_before_sync();
     __syncthreads();
@@ -1714,25 +1722,29 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
                    cu_chunks,   ntasks_dev, a.gates,   static_cast<const __nv_bfloat16 *>(a.b),
                    static_cast<const __nv_bfloat16 *>(a.w), a.bwd_ext, debug_giveup_flag()};
     // The fused kernel (chunk tasks, then the scans on B H of the CTAs) when the scans leave
-    // enough SMs to the queue's tail: dense sequences, nothing saved for a backward, and a
-    // workspace with room for the queue and flags.
+    // enough SMs to the queue's tail: dense sequences and room for the queue and flags. With
+    // the backward's extras it also keeps T and W (bwd_ext) and the chunk-entry states; a
+    // call for the chunk tasks alone (chunks_only) takes the chunk kernel.
     const int BH = a.B * a.H;
     int coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
-    const bool fused = !varlen && !bwd && !a.chunks_only && !a.saved_states && coop != 0 && !debug_unfused_flag() &&
-                       BH + kFusedMinQueueCtas <= nsm &&
-                       a.workspace_bytes >= forward_tc_workspace_bytes(a.B, a.T, a.H);
+    // the queue and flags: behind the slots in a forward's workspace, or where the caller says
+    unsigned char *sync = a.fused_sync ? a.fused_sync
+                          : (a.workspace_bytes >= forward_tc_workspace_bytes(a.B, a.T, a.H)
+                                 ? ws + (size_t)ntasks * (SLOT_BYTES + GAMMA_BYTES) : nullptr);
+    const bool fused = !varlen && !a.chunks_only && sync != nullptr && coop != 0 && !debug_unfused_flag() &&
+                       BH + kFusedMinQueueCtas <= nsm;
     if (fused) {
         void (*fk)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                    const CUtensorMap, const CUtensorMap, ChunkParams, ScanParams) =
-            general ? fwd_fused_kernel<true> : fwd_fused_kernel<false>;
+            general ? (bwd ? fwd_fused_kernel<true, true> : fwd_fused_kernel<true, false>)
+                    : (bwd ? fwd_fused_kernel<false, true> : fwd_fused_kernel<false, false>);
         e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fk, NT, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) return cudaErrorInvalidConfiguration;
-        unsigned char *sync = ws + (size_t)ntasks * (SLOT_BYTES + GAMMA_BYTES);
         e = cudaMemsetAsync(sync, 0, fused_sync_bytes(ntasks), s);
         if (e != cudaSuccess) return e;
         cp.queue = reinterpret_cast<int *>(sync);
@@ -1742,7 +1754,7 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
         // time of one scan: rest ~ (nsm - BH) * NC * (scan time per chunk / chunk task time).
         const double rest = (double)(nsm - BH) * NC * kScanToTaskTime;
         cp.switch_at = rest >= ntasks ? 0 : ntasks - (int)rest;
-        ScanParams sp{a.B, a.T, a.H, NC, ntasks, ws, a.S0, a.S_T, nullptr, a.status, nullptr, nullptr,
+        ScanParams sp{a.B, a.T, a.H, NC, ntasks, ws, a.S0, a.S_T, a.saved_states, a.status, nullptr, nullptr,
                       static_cast<__nv_bfloat16 *>(a.o)};
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(nsm);

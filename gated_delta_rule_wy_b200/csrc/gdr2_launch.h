@@ -30,6 +30,9 @@ struct FwdArgs {
     // writes T and W of every task here; chunks_only leaves out the scan kernel
     unsigned char *bwd_ext = nullptr;
     bool chunks_only = false;
+    // the fused forward's queue counter and task flags (fused_sync_bytes_for(tasks) bytes), when
+    // the workspace has no room for them behind the slots; null: behind the slots, if it fits
+    unsigned char *fused_sync = nullptr;
 };
 
 struct DecodeArgs {

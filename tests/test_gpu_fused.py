@@ -26,6 +26,16 @@ CASES = [
 ]
 
 
+# edges: B H at the fusion threshold of a 148-SM B200 (116 scans beside 32 queue CTAs), one
+# chunk, one token, one (sequence, head), a chunk count that the scans' switch index hits early
+CASES += [
+    dict(B=4, H=29, T=130, seed=90, with_S0=True),
+    dict(B=3, H=5, T=64, seed=91, with_S0=True),
+    dict(B=2, H=3, T=1, seed=92, with_S0=True),
+    dict(B=1, H=1, T=777, seed=93, with_S0=True, decay_shift=2.0),
+]
+
+
 @pytest.mark.parametrize("c", CASES, ids=lambda c: f"B{c['B']}_H{c['H']}_T{c['T']}")
 def test_fused_forward_is_bitwise_the_two_kernel_forward(c):
     lib = binding.load_library()
@@ -120,3 +130,31 @@ def test_fused_backward_front_is_bitwise_the_two_launch_front(c):
             continue
         assert torch.isfinite(g1[name].float()).all(), name
         assert torch.equal(g1[name], g2[name]), f"{name} differs in {(g1[name] != g2[name]).sum().item()} elements"
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 200), (2, 16, 4096)], ids=["B1_H2_T200", "B2_H16_T4096"])
+def test_fused_forward_with_saved_states_and_the_recomputing_backward(shape):
+    # the forward's saved chunk states, and the backward without them (which recomputes them in
+    # the fused forward launch, keeping T and W for its chunk kernels), against the two kernels
+    from gated_delta_rule_wy_b200 import gdr2_backward
+    lib = binding.load_library()
+    B, H, T = shape
+    x = I.make_forward_inputs(B=B, H=H, T=T, dk=128, dv=128, dtype=torch.bfloat16, seed=94, with_S0=True).to("cuda")
+    dO = I.make_upstream_grad(B, T, H, 128, 94, dtype=torch.bfloat16).cuda()
+    dS_T = (torch.randn((B, H, 128, 128), generator=torch.Generator().manual_seed(95)) * 0.1).cuda()
+    runs = []
+    for unfused in (0, 1):
+        lib.gdr2_debug_forward_unfused(unfused)
+        try:
+            o, S, saved = gdr2_forward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, x.S0, save_states=True)
+            g = gdr2_backward(x.q, x.k, x.v, x.log_alpha, x.b, x.w, dO, x.S0, dS_T, None)
+            gdr2_sync_status()
+        finally:
+            lib.gdr2_debug_forward_unfused(0)
+        runs.append((o, S, saved, g))
+    (o1, S1, sv1, g1), (o2, S2, sv2, g2) = runs
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    assert torch.equal(sv1, sv2), "saved states differ"
+    for name in g1:
+        if g1[name] is not None:
+            assert torch.equal(g1[name], g2[name]), name
