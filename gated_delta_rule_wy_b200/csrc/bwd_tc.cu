@@ -20,11 +20,12 @@
 // dP_tt q_t to dk in fp32, and its two contributions to dG cancel exactly.
 //
 // Launches (one stream):
-//   1. the forward's chunk kernel (backward instance): the workspace slots ([Q'; M], K~,
-//      U~, P, gamma) plus T and W; and, without saved states, the forward's scan kernel
-//      for the chunk-entry states. With saved states, where B H leaves 32 SMs to the chunk
-//      tasks, steps 1 and 2 are one cooperative launch (bwd_front_kernel, fwd_tc.cu): the
-//      chunk tasks from the last chunk back, then the reverse scans on B H of the CTAs;
+//   1. the forward's chunk tasks (backward instance): the workspace slots ([Q'; M], K~,
+//      U~, P, gamma) plus T and W; and, without saved states, the forward's scans for the
+//      chunk-entry states. Where B H leaves 32 SMs to the chunk tasks, both run as one
+//      cooperative launch: with saved states steps 1 and 2 (bwd_front_kernel, fwd_tc.cu:
+//      the chunk tasks from the last chunk back, then the reverse scans on B H of the CTAs),
+//      without them the chunk tasks and the forward's scans (fwd_fused_kernel);
 //   2. reverse scan (one CTA per (batch, head), chunks last to first): dS^T in TMEM in
 //      fp32; per chunk a bf16 image of dS' for the chunk kernels, then
 //      dS^T = dS'^T Diag(gamma) + dS'^T M + dO^T Q' as 12 MMAs;
@@ -1056,7 +1057,7 @@ cudaError_t launch_backward_tc(const BwdArgs &a, cudaStream_t s)
     const int ntasks = (int)L.ntasks;
     float *states = a.saved_states ? const_cast<float *>(a.saved_states) : reinterpret_cast<float *>(ws + L.states);
 
-    // 1. the forward's chunk kernel (and, without saved states, its scan for the states)
+    // 1. the forward's chunk tasks (and, without saved states, its scans for the states)
     FwdArgs fa{};
     fa.B = a.B; fa.T = a.T; fa.H = a.H; fa.dk = DK; fa.dv = DV; fa.bf16 = true;
     fa.q = a.q; fa.k = a.k; fa.v = a.v; fa.log_alpha = a.log_alpha; fa.b = a.b; fa.w = a.w; fa.S0 = a.S0;
