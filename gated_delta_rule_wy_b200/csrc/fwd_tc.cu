@@ -31,7 +31,10 @@
 // every CTA takes chunk tasks from a queue in chunk-major order, and CTA b < B H
 // leaves the queue near its end for the scan of (batch, head) b, which copies a
 // chunk's workspace slot only once that task's flag says it is written. The scans
-// then overlap the last quarter or so of the chunk tasks.
+// then overlap the last quarter or so of the chunk tasks. The same launch serves a
+// forward that saves its chunk-entry states and the backward's recomputation of them
+// (T and W kept); the backward's front (bwd_front_kernel) is fused alike, its queue
+// running from the last chunk back for the reverse scans of the state gradient.
 //
 // Decay range. exp(G_t - G_i) is formed as a product of two factors around a
 // per-channel reference g_I, the cumulative decay at the midpoint of the
