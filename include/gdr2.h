@@ -385,8 +385,8 @@ gdr2_status gdr2_backward_noalloc(int B, int T, int H, int dk, int dv, gdr2_dtyp
 gdr2_status gdr2_sync_status(void *stream);
 
 /*
- * Test hooks. Neither has a counterpart in the paper; they exist so that
- * tests can reach code that normal inputs never run.
+ * Test hooks. None has a counterpart in the paper; they exist so that tests
+ * can reach code that normal inputs never run, or compare two paths bit for bit.
  *
  * gdr2_debug_force_timeout -- while `enable` is nonzero, the chunk kernel of
  * every tensor-core forward launch (also the one inside gdr2_backward) first
