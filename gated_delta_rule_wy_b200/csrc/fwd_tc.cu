@@ -113,6 +113,7 @@ constexpr uint32_t TM_COLS = 512;  // TMEM columns of the chunk kernel
 // ratio of a scan's time per chunk to a chunk task's time that places the switch.
 constexpr int kFusedMinQueueCtas = 32;
 constexpr double kScanToTaskTime = 0.25;
+constexpr double kLongScanToTaskTime = 0.22;    // from 256 chunks per sequence (measured better there)
 constexpr double kSavingScanToTaskTime = 0.35;  // the same when the scans also write the chunk states
 constexpr double kRevScanToTaskTime = 0.25;  // the same for the backward's front (reverse scans)
 
@@ -1756,7 +1757,8 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
         cp.BH = BH;
         // The scans start once (nsm - BH) CTAs can finish the rest of the queue in about the
         // time of one scan: rest ~ (nsm - BH) * NC * (scan time per chunk / chunk task time).
-        const double rest = (double)(nsm - BH) * NC * (a.saved_states ? kSavingScanToTaskTime : kScanToTaskTime);
+        const double ratio = a.saved_states ? kSavingScanToTaskTime : (NC >= 256 ? kLongScanToTaskTime : kScanToTaskTime);
+        const double rest = (double)(nsm - BH) * NC * ratio;
         cp.switch_at = rest >= ntasks ? 0 : ntasks - (int)rest;
         ScanParams sp{a.B, a.T, a.H, NC, ntasks, ws, a.S0, a.S_T, a.saved_states, a.status, nullptr, nullptr,
                       static_cast<__nv_bfloat16 *>(a.o)};
