@@ -1773,8 +1773,14 @@ cudaError_t launch_forward_tc(const FwdArgs &a, cudaStream_t s)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, fk, mq, mk, mb, mv, mw, mla, mo, cp, sp);
-        if (e != cudaSuccess) return e;
-        return launch_output_epilogue(a, nsm, s);
+        if (e == cudaSuccess) return launch_output_epilogue(a, nsm, s);
+        // the device could not hold every CTA at once (another context holds SMs): the two
+        // kernels below do the same work without that requirement
+        if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+        (void)cudaGetLastError();
+        cp.queue = nullptr;
+        cp.flags = nullptr;
+        cp.BH = cp.switch_at = 0;
     }
     const int grid = ntasks < nsm ? ntasks : nsm;
     chunk<<<grid, NT, SMEM_BYTES, s>>>(mq, mk, mb, mv, mw, mla, cp);
@@ -1855,6 +1861,10 @@ cudaError_t launch_backward_front_fused(const FwdArgs &a, const BwdFrontArgs &r,
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, fk, mq, mk, mb, mv, mw, mla, mdo, cp, rp);
     if (e == cudaSuccess) *launched = true;
+    if (e == cudaErrorCooperativeLaunchTooLarge) {  // not every CTA fits at once: the caller's two launches
+        (void)cudaGetLastError();
+        return cudaSuccess;
+    }
     return e;
 }
 
